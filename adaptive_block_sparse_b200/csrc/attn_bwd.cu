@@ -1,0 +1,770 @@
+// Block-sparse flash-attention backward over the kept 64 x 64 tiles (sm_100a).
+//
+// The NABLA pages ("NABLA: Neighborhood Adaptive Block-Level Attention", gist.science,
+// Chinese edition, technical summary, "Core contributions: two-stage acceleration";
+// lsdiaocha.cn article, section 3, pre-training 10.9 s -> 7.5 s per iteration) credit the
+// method with faster training as well as inference.  The binary mask has no gradient,
+// so the backward pass is ordinary softmax-attention backward restricted to the kept
+// tiles, with the mask held constant:
+//   P = exp(scale Q K^T - LSE),  dP = dO V^T,  Dr = rowsum(dO * O),
+//   dS = P * (dP - Dr),  dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Deterministic, no floating-point atomics, three launches:
+//   1. preprocess: Dr = rowsum(dO * O) and LSE in log2 units (HBM-bound);
+//   2. dK/dV: one CTA per pair of key blocks (128 key rows -> M = 128 MMAs) walks the
+//      ascending union of the two blocks' query-block (column) lists.  Per query block:
+//      S^T = K Q^T and dP^T = V dO^T into TMEM (double-buffered), P^T and dS^T in
+//      registers (one key row per thread) -> bf16 in shared memory, then
+//      dV += P^T dO and dK += dS^T Q into TMEM accumulators;
+//   3. dQ: one CTA per pair of query blocks walks the union of the row lists:
+//      S = Q K^T and dP = dO V^T into TMEM, dS in registers -> shared memory,
+//      dQ += dS K.
+// Warp roles as in the forward kernel: warp 0 = TMA producer, warp 1 = MMA issuer and
+// TMEM owner, warps 4-7 = element-wise math and epilogue.  Every wait is bounded.
+#include <math.h>
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace nabla {
+
+bool make_map_bf16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows);
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMathWarp0 = 4;
+constexpr uint32_t kEnd = 0xFFFFFFFFu;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// -------------------------------------------------------------------------------------
+// 1. preprocess: delta = rowsum(dO * O), lse2 = LSE * log2(e)
+// -------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const void* __restrict__ o, int o_f32,
+                                                             const __nv_bfloat16* __restrict__ dout,
+                                                             const float* __restrict__ lse,
+                                                             float* __restrict__ delta,
+                                                             float* __restrict__ lse2, long long rows) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int E = D / 32;  // elements per lane (contiguous)
+  float acc = 0.f;
+  const __nv_bfloat16* g = dout + row * D + lane * E;
+  if (o_f32) {
+    const float* f = static_cast<const float*>(o) + row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(g[e]), f[e], acc);
+  } else {
+    const __nv_bfloat16* f = static_cast<const __nv_bfloat16*>(o) + row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(g[e]), __bfloat162float(f[e]), acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    delta[row] = acc;
+    lse2[row] = lse[row] * kLog2e;
+  }
+}
+
+struct BwdParams {
+  const int32_t* list_idx;   // column lists (dK/dV pass) or row lists (dQ pass)
+  const int32_t* list_cnt;
+  const float* delta;
+  const float* lse2;
+  float* out0;               // dV (dK/dV pass) or dQ (dQ pass)
+  float* out1;               // dK (dK/dV pass)
+  uint32_t* status;
+  int nb;
+  long long S;
+  float scale_log2;
+  float scale;
+};
+
+// Walks the ascending union of two sorted lists; returns -1 at the end.  f: bit0 = in
+// the first list, bit1 = in the second.
+struct UnionWalk {
+  const int32_t* l0;
+  const int32_t* l1;
+  int c0, c1, a, b;
+  __device__ int next(uint32_t* f) {
+    if (a < c0 && b < c1) {
+      const int ja = l0[a], jb = l1[b];
+      if (ja < jb) { *f = 1; ++a; return ja; }
+      if (jb < ja) { *f = 2; ++b; return jb; }
+      *f = 3; ++a; ++b; return ja;
+    }
+    if (a < c0) { *f = 1; return l0[a++]; }
+    if (b < c1) { *f = 2; return l1[b++]; }
+    return -1;
+  }
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kPairBytes = 128 * D * 2;       // one 128-row operand (resident)
+  static constexpr int kTileBytes = 64 * D * 2;        // one 64-row operand (streamed)
+  static constexpr int kPBytes = 128 * 64 * 2;         // one bf16 128 x 64 tile
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM: buffer b at columns [128b, 128b+64) = S (or S^T), [128b+64, 128b+128) = dP.
+  static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
+};
+
+// -------------------------------------------------------------------------------------
+// 2. dK / dV over column lists
+// -------------------------------------------------------------------------------------
+template <int D>
+struct DkdvLayout {
+  using C = BwdCfg<D>;
+  static constexpr int kStages = 2;
+  static constexpr int kStageBytes = 2 * C::kTileBytes + 512;    // Q_i, dO_i, lse2_i, delta_i
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + C::kPairBytes;
+  static constexpr int kOffStage = kOffV + C::kPairBytes;
+  static constexpr int kOffPT = kOffStage + kStages * ((kStageBytes + 1023) / 1024 * 1024);
+  static constexpr int kOffDST = kOffPT + 2 * C::kPBytes;
+  static constexpr int kOffBar = kOffDST + 2 * C::kPBytes;
+  static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_q64,
+                         const __grid_constant__ CUtensorMap map_do64,
+                         const __grid_constant__ CUtensorMap map_k128,
+                         const __grid_constant__ CUtensorMap map_v128, const BwdParams prm) {
+  using C = BwdCfg<D>;
+  using L = DkdvLayout<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sK = smem + L::kOffK;
+  unsigned char* sV = smem + L::kOffV;
+  unsigned char* sStage = smem + L::kOffStage;
+  unsigned char* sPT = smem + L::kOffPT;
+  unsigned char* sDST = smem + L::kOffDST;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;                    // [kStages]
+  uint64_t* empty = bars + L::kStages;      // [kStages]
+  uint64_t* kv_full = bars + 2 * L::kStages;
+  uint64_t* sd_full = kv_full + 1;          // [2]
+  uint64_t* p_full = sd_full + 2;           // [2]
+  uint64_t* acc_bar = p_full + 2;
+  uint64_t* drain = acc_bar + 1;
+  uint32_t* meta = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* tmem_slot = meta + L::kStages;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long bh = blockIdx.y;
+  const int nb = prm.nb;
+  const int j0 = 2 * blockIdx.x;
+  const bool has_j1 = (j0 + 1) < nb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(kv_full, 1);
+    mbar_init(&sd_full[0], 1);
+    mbar_init(&sd_full[1], 1);
+    mbar_init(&p_full[0], 128);
+    mbar_init(&p_full[1], 128);
+    mbar_init(acc_bar, 1);
+    mbar_init(drain, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q64);
+      tma_prefetch_desc(&map_do64);
+      tma_prefetch_desc(&map_k128);
+      tma_prefetch_desc(&map_v128);
+      const int krow = static_cast<int>(bh * prm.S + static_cast<long long>(j0) * 64);
+      mbar_arrive_expect_tx(kv_full, 2 * C::kPairBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_2d(sK + pn * 16384, &map_k128, kv_full, pn * 64, krow);
+        tma_load_2d(sV + pn * 16384, &map_v128, kv_full, pn * 64, krow);
+      }
+      UnionWalk wk;
+      wk.l0 = prm.list_idx + (bh * nb + j0) * static_cast<long long>(nb);
+      wk.l1 = wk.l0 + nb;
+      wk.c0 = min(max(prm.list_cnt[bh * nb + j0], 0), nb);
+      wk.c1 = has_j1 ? min(max(prm.list_cnt[bh * nb + j0 + 1], 0), nb) : 0;
+      wk.a = wk.b = 0;
+      int it = 0;
+      while (true) {
+        uint32_t f = 0;
+        const int i = wk.next(&f);
+        const int s = it % L::kStages;
+        const int n = it / L::kStages;
+        if (n > 0 && !mbar_wait(&empty[s], (n - 1) & 1, prm.status, kDevTimeoutKvEmpty)) break;
+        if (i < 0 || i >= nb) {
+          meta[s] = kEnd;
+          mbar_arrive(&full[s]);
+          break;
+        }
+        meta[s] = static_cast<uint32_t>(i) | (f << 28);
+        unsigned char* st = sStage + s * L::kStageStride;
+        mbar_arrive_expect_tx(&full[s], 2 * C::kTileBytes + 512);
+        const long long qrow = bh * prm.S + static_cast<long long>(i) * 64;
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_2d(st + pn * 8192, &map_q64, &full[s], pn * 64, static_cast<int>(qrow));
+          tma_load_2d(st + C::kTileBytes + pn * 8192, &map_do64, &full[s], pn * 64, static_cast<int>(qrow));
+        }
+        bulk_load(st + 2 * C::kTileBytes, prm.lse2 + qrow, 256, &full[s]);
+        bulk_load(st + 2 * C::kTileBytes + 256, prm.delta + qrow, 256, &full[s]);
+        ++it;
+      }
+      const int first = it > L::kStages ? it - L::kStages : 0;
+      for (int x = first; x < it; ++x)
+        mbar_wait(&full[x % L::kStages], (x / L::kStages) & 1, prm.status, kDevTimeoutDrain);
+      mbar_wait(kv_full, 0, prm.status, kDevTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      const uint32_t st_addr = smem_u32(sStage);
+      const uint32_t pt_addr = smem_u32(sPT), dst_addr = smem_u32(sDST);
+      auto issue_sd = [&](int x) {
+        const int s = x % L::kStages;
+        const uint32_t qa = st_addr + s * L::kStageStride;
+        const uint32_t da = qa + C::kTileBytes;
+        const uint32_t col = (x & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int pn = kk >> 2, w = kk & 3;
+          mma_bf16_ss(tmem + col, sdesc_sw128(k_addr + pn * 16384 + w * 32, 16, 1024),
+                      sdesc_sw128(qa + pn * 8192 + w * 32, 16, 1024), idesc_s, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int pn = kk >> 2, w = kk & 3;
+          mma_bf16_ss(tmem + col + 64, sdesc_sw128(v_addr + pn * 16384 + w * 32, 16, 1024),
+                      sdesc_sw128(da + pn * 8192 + w * 32, 16, 1024), idesc_s, kk > 0);
+        }
+        mma_commit(&sd_full[x & 1]);
+      };
+      auto issue_acc = [&](int x) {
+        const int s = x % L::kStages;
+        const uint32_t qa = st_addr + s * L::kStageStride;
+        const uint32_t da = qa + C::kTileBytes;
+        const uint32_t b = x & 1;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_bf16_ss(tmem + C::kColAcc0, sdesc_sw128(pt_addr + b * C::kPBytes + kk * 32, 16, 1024),
+                      sdesc_sw128(da + kk * 2048, 8192, 1024), idesc_acc, (x > 0 || kk > 0));
+          mma_bf16_ss(tmem + C::kColAcc1, sdesc_sw128(dst_addr + b * C::kPBytes + kk * 32, 16, 1024),
+                      sdesc_sw128(qa + kk * 2048, 8192, 1024), idesc_acc, (x > 0 || kk > 0));
+        }
+      };
+      bool ok = mbar_wait(kv_full, 0, prm.status, kDevTimeoutQFull);
+      if (ok) ok = mbar_wait(&full[0], 0, prm.status, kDevTimeoutTmaFull);
+      if (ok && meta[0] != kEnd) {
+        tc_fence_after();
+        issue_sd(0);
+        for (int it = 0;; ++it) {
+          const int s1 = (it + 1) % L::kStages;
+          if (!mbar_wait(&full[s1], ((it + 1) / L::kStages) & 1, prm.status, kDevTimeoutTmaFull)) break;
+          const bool end1 = meta[s1] == kEnd;
+          tc_fence_after();
+          if (!end1) issue_sd(it + 1);
+          if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutPFull)) break;
+          tc_fence_after();
+          issue_acc(it);
+          mma_commit(&empty[it % L::kStages]);
+          if (end1) break;
+        }
+      }
+      mma_commit(acc_bar);
+      mma_commit(drain);
+      mbar_wait(drain, 0, prm.status, kDevTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp >= kMathWarp0) {
+    const int row = threadIdx.x - kMathWarp0 * 32;          // key row within the pair
+    const uint32_t lane_base = static_cast<uint32_t>((warp - kMathWarp0) * 32) << 16;
+    const bool upper = row >= 64;
+    const float sl2 = prm.scale_log2;
+    unsigned char* ptrow = sPT + row * 128;
+    unsigned char* dsrow = sDST + row * 128;
+    int it = 0;
+    bool ok = true;
+    for (;; ++it) {
+      const int s = it % L::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (it / L::kStages) & 1, prm.status, kDevTimeoutTmaFull));
+      if (!ok) break;
+      const uint32_t mt = meta[s];
+      if (mt == kEnd) break;
+      const bool keep = upper ? ((mt >> 29) & 1u) : ((mt >> 28) & 1u);
+      const float* s_lse = reinterpret_cast<const float*>(sStage + s * L::kStageStride + 2 * C::kTileBytes);
+      const float* s_del = s_lse + 64;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutSFull));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t col = (it & 1) * 128;
+      uint32_t pk[32], dk[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tmem + lane_base + col + half * 32, sv);
+        tmem_ld32(tmem + lane_base + col + 64 + half * 32, dv);
+        tmem_wait_ld();
+        if (keep) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const int q0 = half * 32 + c;
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -s_lse[q0]));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -s_lse[q0 + 1]));
+            const float d0 = p0 * (__uint_as_float(dv[c]) - s_del[q0]);
+            const float d1 = p1 * (__uint_as_float(dv[c + 1]) - s_del[q0 + 1]);
+            pk[half * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
+            dk[half * 16 + (c >> 1)] = pack_bf16x2(d0, d1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) { pk[half * 16 + c] = 0u; dk[half * 16 + c] = 0u; }
+        }
+      }
+      const int b = it & 1;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const int off = b * C::kPBytes + ((ch ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(ptrow + off) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(dsrow + off) = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    // ---- epilogue: dV and scale * dK (fp32) ----------------------------------------------
+    const bool valid = upper ? has_j1 : true;
+    const long long tok = bh * prm.S + static_cast<long long>(j0) * 64 + row;
+    bool have = ok && it > 0;
+    if (have) {
+      have = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, prm.status, kDevTimeoutOBar));
+      tc_fence_after();
+    }
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      float* out = which == 0 ? prm.out0 : prm.out1;
+      const float mul = which == 0 ? 1.f : prm.scale;
+      const uint32_t colbase = which == 0 ? C::kColAcc0 : C::kColAcc1;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ov[32];
+        if (have) {
+          tmem_ld32(tmem + lane_base + colbase + c0, ov);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = 0u;
+        }
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(out + tok * D + c0);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            dst[c] = make_float4(__uint_as_float(ov[4 * c]) * mul, __uint_as_float(ov[4 * c + 1]) * mul,
+                                 __uint_as_float(ov[4 * c + 2]) * mul, __uint_as_float(ov[4 * c + 3]) * mul);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// -------------------------------------------------------------------------------------
+// 3. dQ over row lists
+// -------------------------------------------------------------------------------------
+template <int D>
+struct DqLayout {
+  using C = BwdCfg<D>;
+  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kStageBytes = 2 * C::kTileBytes;        // K_j, V_j
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kOffQ + C::kPairBytes;
+  static constexpr int kOffStage = kOffDO + C::kPairBytes;
+  static constexpr int kOffDS = kOffStage + kStages * kStageBytes;
+  static constexpr int kOffBar = kOffDS + 2 * C::kPBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q128,
+                       const __grid_constant__ CUtensorMap map_do128,
+                       const __grid_constant__ CUtensorMap map_k64,
+                       const __grid_constant__ CUtensorMap map_v64, const BwdParams prm) {
+  using C = BwdCfg<D>;
+  using L = DqLayout<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sQ = smem + L::kOffQ;
+  unsigned char* sDO = smem + L::kOffDO;
+  unsigned char* sStage = smem + L::kOffStage;
+  unsigned char* sDS = smem + L::kOffDS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + L::kStages;
+  uint64_t* q_full = bars + 2 * L::kStages;
+  uint64_t* sd_full = q_full + 1;
+  uint64_t* p_full = sd_full + 2;
+  uint64_t* acc_bar = p_full + 2;
+  uint64_t* drain = acc_bar + 1;
+  uint32_t* meta = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* tmem_slot = meta + L::kStages;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long bh = blockIdx.y;
+  const int nb = prm.nb;
+  const int i0 = 2 * blockIdx.x;
+  const bool has_i1 = (i0 + 1) < nb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(&sd_full[0], 1);
+    mbar_init(&sd_full[1], 1);
+    mbar_init(&p_full[0], 128);
+    mbar_init(&p_full[1], 128);
+    mbar_init(acc_bar, 1);
+    mbar_init(drain, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q128);
+      tma_prefetch_desc(&map_do128);
+      tma_prefetch_desc(&map_k64);
+      tma_prefetch_desc(&map_v64);
+      const int qrow = static_cast<int>(bh * prm.S + static_cast<long long>(i0) * 64);
+      mbar_arrive_expect_tx(q_full, 2 * C::kPairBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_2d(sQ + pn * 16384, &map_q128, q_full, pn * 64, qrow);
+        tma_load_2d(sDO + pn * 16384, &map_do128, q_full, pn * 64, qrow);
+      }
+      UnionWalk wk;
+      wk.l0 = prm.list_idx + (bh * nb + i0) * static_cast<long long>(nb);
+      wk.l1 = wk.l0 + nb;
+      wk.c0 = min(max(prm.list_cnt[bh * nb + i0], 0), nb);
+      wk.c1 = has_i1 ? min(max(prm.list_cnt[bh * nb + i0 + 1], 0), nb) : 0;
+      wk.a = wk.b = 0;
+      int it = 0;
+      while (true) {
+        uint32_t f = 0;
+        const int j = wk.next(&f);
+        const int s = it % L::kStages;
+        const int n = it / L::kStages;
+        if (n > 0 && !mbar_wait(&empty[s], (n - 1) & 1, prm.status, kDevTimeoutKvEmpty)) break;
+        if (j < 0 || j >= nb) {
+          meta[s] = kEnd;
+          mbar_arrive(&full[s]);
+          break;
+        }
+        meta[s] = static_cast<uint32_t>(j) | (f << 28);
+        unsigned char* st = sStage + s * L::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], 2 * C::kTileBytes);
+        const int krow = static_cast<int>(bh * prm.S + static_cast<long long>(j) * 64);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_2d(st + pn * 8192, &map_k64, &full[s], pn * 64, krow);
+          tma_load_2d(st + C::kTileBytes + pn * 8192, &map_v64, &full[s], pn * 64, krow);
+        }
+        ++it;
+      }
+      const int first = it > L::kStages ? it - L::kStages : 0;
+      for (int x = first; x < it; ++x)
+        mbar_wait(&full[x % L::kStages], (x / L::kStages) & 1, prm.status, kDevTimeoutDrain);
+      mbar_wait(q_full, 0, prm.status, kDevTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+      const uint32_t st_addr = smem_u32(sStage), ds_addr = smem_u32(sDS);
+      auto issue_sd = [&](int x) {
+        const int s = x % L::kStages;
+        const uint32_t ka = st_addr + s * L::kStageBytes;
+        const uint32_t va = ka + C::kTileBytes;
+        const uint32_t col = (x & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int pn = kk >> 2, w = kk & 3;
+          mma_bf16_ss(tmem + col, sdesc_sw128(q_addr + pn * 16384 + w * 32, 16, 1024),
+                      sdesc_sw128(ka + pn * 8192 + w * 32, 16, 1024), idesc_s, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int pn = kk >> 2, w = kk & 3;
+          mma_bf16_ss(tmem + col + 64, sdesc_sw128(do_addr + pn * 16384 + w * 32, 16, 1024),
+                      sdesc_sw128(va + pn * 8192 + w * 32, 16, 1024), idesc_s, kk > 0);
+        }
+        mma_commit(&sd_full[x & 1]);
+      };
+      auto issue_acc = [&](int x) {
+        const int s = x % L::kStages;
+        const uint32_t ka = st_addr + s * L::kStageBytes;
+        const uint32_t b = x & 1;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tmem + C::kColAcc0, sdesc_sw128(ds_addr + b * C::kPBytes + kk * 32, 16, 1024),
+                      sdesc_sw128(ka + kk * 2048, 8192, 1024), idesc_acc, (x > 0 || kk > 0));
+      };
+      bool ok = mbar_wait(q_full, 0, prm.status, kDevTimeoutQFull);
+      if (ok) ok = mbar_wait(&full[0], 0, prm.status, kDevTimeoutTmaFull);
+      if (ok && meta[0] != kEnd) {
+        tc_fence_after();
+        issue_sd(0);
+        for (int it = 0;; ++it) {
+          const int s1 = (it + 1) % L::kStages;
+          if (!mbar_wait(&full[s1], ((it + 1) / L::kStages) & 1, prm.status, kDevTimeoutTmaFull)) break;
+          const bool end1 = meta[s1] == kEnd;
+          tc_fence_after();
+          if (!end1) issue_sd(it + 1);
+          if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutPFull)) break;
+          tc_fence_after();
+          issue_acc(it);
+          mma_commit(&empty[it % L::kStages]);
+          if (end1) break;
+        }
+      }
+      mma_commit(acc_bar);
+      mma_commit(drain);
+      mbar_wait(drain, 0, prm.status, kDevTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp >= kMathWarp0) {
+    const int row = threadIdx.x - kMathWarp0 * 32;
+    const uint32_t lane_base = static_cast<uint32_t>((warp - kMathWarp0) * 32) << 16;
+    const bool upper = row >= 64;
+    const bool valid = upper ? has_i1 : true;
+    const long long tok = bh * prm.S + static_cast<long long>(i0) * 64 + row;
+    const float my_lse2 = valid ? prm.lse2[tok] : 0.f;
+    const float my_delta = valid ? prm.delta[tok] : 0.f;
+    const float sl2 = prm.scale_log2;
+    unsigned char* dsrow = sDS + row * 128;
+    int it = 0;
+    bool ok = true;
+    for (;; ++it) {
+      const int s = it % L::kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (it / L::kStages) & 1, prm.status, kDevTimeoutTmaFull));
+      if (!ok) break;
+      const uint32_t mt = meta[s];
+      if (mt == kEnd) break;
+      const bool keep = upper ? ((mt >> 29) & 1u) : ((mt >> 28) & 1u);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutSFull));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t col = (it & 1) * 128;
+      uint32_t dk[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tmem + lane_base + col + half * 32, sv);
+        tmem_ld32(tmem + lane_base + col + 64 + half * 32, dv);
+        tmem_wait_ld();
+        if (keep) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -my_lse2));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -my_lse2));
+            dk[half * 16 + (c >> 1)] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - my_delta),
+                                                   p1 * (__uint_as_float(dv[c + 1]) - my_delta));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) dk[half * 16 + c] = 0u;
+        }
+      }
+      const int b = it & 1;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(dsrow + b * C::kPBytes + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    bool have = ok && it > 0;
+    if (have) {
+      have = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, prm.status, kDevTimeoutOBar));
+      tc_fence_after();
+    }
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t ov[32];
+      if (have) {
+        tmem_ld32(tmem + lane_base + C::kColAcc0 + c0, ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) ov[c] = 0u;
+      }
+      if (valid) {
+        float4* dst = reinterpret_cast<float4*>(prm.out0 + tok * D + c0);
+        const float mul = prm.scale;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          dst[c] = make_float4(__uint_as_float(ov[4 * c]) * mul, __uint_as_float(ov[4 * c + 1]) * mul,
+                               __uint_as_float(ov[4 * c + 2]) * mul, __uint_as_float(ov[4 * c + 3]) * mul);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* o, int o_f32,
+                       const void* dout, const float* lse, const int32_t* ridx, const int32_t* rcnt,
+                       const int32_t* cidx, const int32_t* ccnt, const Dims& d, float scale,
+                       float* dq, float* dk, float* dv, void* ws, cudaStream_t st, bool* map_ok) {
+  const long long rows = static_cast<long long>(d.BH) * d.S;
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
+  float* lse2 = delta + align_up(static_cast<size_t>(rows), 64);
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      o, o_f32, static_cast<const __nv_bfloat16*>(dout), lse, delta, lse2, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128, mk64, mv64;
+  *map_ok = make_map_bf16(&mq64, q, rows, D, 64) && make_map_bf16(&mdo64, dout, rows, D, 64) &&
+            make_map_bf16(&mk128, k, rows, D, 128) && make_map_bf16(&mv128, v, rows, D, 128) &&
+            make_map_bf16(&mq128, q, rows, D, 128) && make_map_bf16(&mdo128, dout, rows, D, 128) &&
+            make_map_bf16(&mk64, k, rows, D, 64) && make_map_bf16(&mv64, v, rows, D, 64);
+  if (!*map_ok) return cudaErrorInvalidValue;
+
+  BwdParams p;
+  p.delta = delta;
+  p.lse2 = lse2;
+  p.status = status;
+  p.nb = d.nb;
+  p.S = d.S;
+  p.scale_log2 = scale * kLog2e;
+  p.scale = scale;
+  dim3 grid((d.nb + 1) / 2, d.BH);
+
+  p.list_idx = cidx;
+  p.list_cnt = ccnt;
+  p.out0 = dv;
+  p.out1 = dk;
+  e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           DkdvLayout<D>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk128, mv128, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  p.list_idx = ridx;
+  p.list_cnt = rcnt;
+  p.out0 = dq;
+  p.out1 = nullptr;
+  e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           DqLayout<D>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kSmemBytes, st>>>(mq128, mdo128, mk64, mv64, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace nabla
+
+using namespace nabla;
+
+extern "C" size_t nabla_bwd_workspace_bytes(nabla_shape s) {
+  Dims d;
+  if (check_shape(s, &d) != NABLA_OK) return 0;
+  const size_t rows = align_up(static_cast<size_t>(d.BH) * d.S, 64);
+  return kStatusBytes + 2 * rows * sizeof(float);
+}
+
+extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                                       nabla_dtype o_dtype, const void* dout, const float* lse,
+                                       const int32_t* row_idx, const int32_t* row_cnt,
+                                       const int32_t* col_idx, const int32_t* col_cnt,
+                                       nabla_shape s, float scale, float* dq, float* dk, float* dv,
+                                       void* workspace, size_t workspace_bytes,
+                                       nabla_stream_t stream) {
+  Dims d;
+  nabla_status rc = check_shape(s, &d);
+  if (rc != NABLA_OK) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !row_idx || !row_cnt || !col_idx || !col_cnt ||
+      !dq || !dk || !dv)
+    return NABLA_ERR_INVALID_ARG;
+  const void* al16[] = {q, k, v, o, dout, lse, dq, dk, dv};
+  for (const void* p : al16)
+    if (!aligned16(p)) return NABLA_ERR_INVALID_ARG;
+  const void* al4[] = {row_idx, row_cnt, col_idx, col_cnt};
+  for (const void* p : al4)
+    if (reinterpret_cast<uintptr_t>(p) & 3) return NABLA_ERR_INVALID_ARG;
+  if (o_dtype != NABLA_BF16 && o_dtype != NABLA_F32) return NABLA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < nabla_bwd_workspace_bytes(s) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return NABLA_ERR_WORKSPACE;
+  if (static_cast<long long>(d.BH) * d.S >= (1ll << 31)) return NABLA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  bool map_ok = true;
+  e = d.D == 64 ? launch_bwd<64>(q, k, v, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
+                                 col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok)
+                : launch_bwd<128>(q, k, v, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
+                                  col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok);
+  return cuda_status(e);
+}

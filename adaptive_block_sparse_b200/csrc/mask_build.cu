@@ -1,0 +1,411 @@
+// Adaptive block mask: pooled scores, row softmax, CDF threshold, STA union, bitmask and
+// row / column lists.
+//
+// "NABLA: Neighborhood Adaptive Block-Level Attention" (gist.science, Chinese edition),
+// technical summary, Methodology, "adaptive mask construction": Q and K are pooled per
+// block, full attention is computed on the pooled map, and per row the blocks whose
+// cumulative probability exceeds 1 - thr are kept; "hybrid integration with STA": the
+// final mask is the union with a static window mask.  lsdiaocha.cn article, section 4:
+// sort each row and accumulate the probability.
+//
+// Decision precision: the whole decision is taken in fp64 (pooled means, logits,
+// softmax, ranked mass), so it agrees with an fp64 statement of the method except for
+// blocks whose ranked mass lies within rounding (~1e-15) of thr.
+//
+// Selection without a sort: block j is kept iff E_j < thr, where E_j is the mass ranked
+// strictly before j (probability descending, ties by lower index).  The kept set is a
+// prefix of that ranking, so it is found by a most-significant-digit radix select over
+// the fp64 bit patterns of the probabilities (non-negative doubles order like their bit
+// patterns), carrying per-digit counts and masses.  Masses are accumulated as 2^-62
+// fixed-point integers so the result does not depend on the order of the shared-memory
+// atomics (deterministic), with an error below 1e-15 per row.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace nabla {
+
+cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st);
+
+namespace {
+
+constexpr int kThreads = 256;   // 8 warps; one pooled row per warp during selection
+constexpr int kWarps = kThreads / 32;
+constexpr int KC = 32;          // pooled key rows per shared-memory chunk
+constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
+constexpr double kFix = 4611686018427387904.0;  // 2^62
+
+__device__ __forceinline__ unsigned long long to_fix(double p) { return __double2ull_rn(p * kFix); }
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) mask_rows_kernel(
+    const double* __restrict__ qpool, const double* __restrict__ kpool, int nb, int nw, int R,
+    double scale, double thr, int sta_on, int wt2, int wh2, int ww2, int Hb, int Wb,
+    uint32_t* __restrict__ bits, int32_t* __restrict__ row_idx, int32_t* __restrict__ row_cnt) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  unsigned long long* hmass = reinterpret_cast<unsigned long long*>(smem_raw);  // 8 x 256
+  uint32_t* hcnt = reinterpret_cast<uint32_t*>(hmass + kWarps * 256);           // 8 x 256
+  double* qs = reinterpret_cast<double*>(hcnt + kWarps * 256);                  // R x D
+  double* ks = qs + R * D;                                                      // KC x (D+1)
+  double* prow = ks + KC * (D + 1);                                             // R x nb
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const long long bh = blockIdx.y;
+  const int i0 = blockIdx.x * R;
+  const int nrows = min(R, nb - i0);
+
+  for (int e = tid; e < R * D; e += kThreads) {
+    const int r = e / D;
+    qs[e] = (r < nrows) ? qpool[(bh * nb + i0 + r) * D + (e - r * D)] : 0.0;
+  }
+  // ---- pooled logits A = Qp Kp^T * scale (fp64) --------------------------------------
+  for (int j0 = 0; j0 < nb; j0 += KC) {
+    __syncthreads();
+    for (int e = tid; e < KC * D; e += kThreads) {
+      const int jj = e / D;
+      const int dd = e - jj * D;
+      ks[jj * (D + 1) + dd] = (j0 + jj < nb) ? kpool[(bh * nb + j0 + jj) * D + dd] : 0.0;
+    }
+    __syncthreads();
+    for (int e = tid; e < R * KC; e += kThreads) {
+      const int r = e / KC;
+      const int jj = e - r * KC;
+      if (r < nrows && j0 + jj < nb) {
+        const double* qr = qs + r * D;
+        const double* kr = ks + jj * (D + 1);
+        double acc = 0.0;
+#pragma unroll 16
+        for (int dd = 0; dd < D; ++dd) acc = fma(qr[dd], kr[dd], acc);
+        prow[r * nb + j0 + jj] = acc * scale;
+      }
+    }
+  }
+  __syncthreads();
+
+  const unsigned long long T = to_fix(thr);
+  const bool keep_all = thr >= 1.0;
+  const bool keep_none = thr <= 0.0;
+  unsigned long long* mass = hmass + warp * 256;
+  uint32_t* cnt = hcnt + warp * 256;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  for (int r = warp; r < nrows; r += kWarps) {
+    double* row = prow + r * nb;
+    const int i = i0 + r;
+    // ---- row softmax (fp64) -------------------------------------------------------------
+    double m = -INFINITY;
+    for (int j = lane; j < nb; j += 32) m = fmax(m, row[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    double ssum = 0.0;
+    for (int j = lane; j < nb; j += 32) {
+      const double e = exp(row[j] - m);
+      row[j] = e;
+      ssum += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+    for (int j = lane; j < nb; j += 32) row[j] = row[j] / ssum;
+    __syncwarp();
+
+    // ---- radix select of the threshold key ---------------------------------------------
+    // mode 0: keep key >= kstar.  mode 1: keep key > kstar, plus the first `tie_keep`
+    // blocks (by index) whose key == kstar.
+    unsigned long long kstar = 0;
+    int mode = 0;
+    int tie_keep = 0;
+    if (!keep_all && !keep_none) {
+      unsigned long long prefix = 0, pmask = 0, above = 0;
+      int shift = 56;
+      while (true) {
+        for (int k = lane; k < 256; k += 32) { cnt[k] = 0; mass[k] = 0ull; }
+        __syncwarp();
+        for (int j = lane; j < nb; j += 32) {
+          const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(row[j]));
+          if ((key & pmask) == prefix) {
+            const int dg = static_cast<int>((key >> shift) & 255ull);
+            atomicAdd(&cnt[dg], 1u);
+            atomicAdd(&mass[dg], to_fix(row[j]));
+          }
+        }
+        __syncwarp();
+        // lane l owns digits 255-8l .. 248-8l (descending)
+        unsigned long long msum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) msum += mass[255 - 8 * lane - q];
+        unsigned long long incl = msum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        unsigned long long Bq = above + incl - msum;
+        int found = -1;
+        unsigned long long fB = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int dg = 255 - 8 * lane - q;
+          const unsigned long long mm = mass[dg];
+          if (found < 0 && Bq < T && T <= Bq + mm) { found = dg; fB = Bq; }
+          Bq += mm;
+        }
+        const uint32_t fb = __ballot_sync(0xffffffffu, found >= 0);
+        if (fb == 0) {  // the whole prefix range holds < thr: keep all of it
+          kstar = prefix;
+          mode = 0;
+          break;
+        }
+        const int src = __ffs(fb) - 1;
+        const int dg = __shfl_sync(0xffffffffu, found, src);
+        above = __shfl_sync(0xffffffffu, fB, src);
+        const uint32_t c = cnt[dg];
+        prefix |= static_cast<unsigned long long>(dg) << shift;
+        pmask |= 255ull << shift;
+        __syncwarp();
+        if (c == 1) {  // the crossing block is unique: keep every key >= its key
+          unsigned long long mine = 0;
+          for (int j = lane; j < nb; j += 32) {
+            const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(row[j]));
+            if ((key & pmask) == prefix) mine = key;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mine |= __shfl_xor_sync(0xffffffffu, mine, o);
+          kstar = mine;
+          mode = 0;
+          break;
+        }
+        if (shift == 0) {  // c > 1 blocks with identical probability straddle thr
+          kstar = prefix;
+          mode = 1;
+          const unsigned long long f = to_fix(__longlong_as_double(static_cast<long long>(prefix)));
+          const unsigned long long room = T - above;   // > 0
+          unsigned long long need = (f == 0ull) ? c : (room + f - 1ull) / f;
+          tie_keep = static_cast<int>(need < c ? need : c);
+          break;
+        }
+        shift -= 8;
+      }
+    }
+
+    // ---- emit bitmask words and the ascending row list ---------------------------------
+    const int ti = i / (Hb * Wb);
+    const int hi = (i / Wb) % Hb;
+    const int wi = i % Wb;
+    int run = 0;
+    int tie_seen = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int j = w * 32 + lane;
+      bool k = false;
+      bool is_tie = false;
+      if (j < nb) {
+        const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(row[j]));
+        if (keep_all) k = true;
+        else if (keep_none) k = false;
+        else if (mode == 0) k = key >= kstar;
+        else { k = key > kstar; is_tie = key == kstar; }
+      }
+      const uint32_t tb = __ballot_sync(0xffffffffu, is_tie);
+      if (is_tie) k = (tie_seen + __popc(tb & lt_mask)) < tie_keep;
+      tie_seen += __popc(tb);
+      if (sta_on && j < nb) {
+        const int tj = j / (Hb * Wb);
+        const int hj = (j / Wb) % Hb;
+        const int wj = j % Wb;
+        k = k || (abs(ti - tj) <= wt2 && abs(hi - hj) <= wh2 && abs(wi - wj) <= ww2);
+      }
+      const uint32_t kb = __ballot_sync(0xffffffffu, k);
+      if (lane == 0) bits[(bh * nb + i) * nw + w] = kb;
+      if (row_idx != nullptr && k) row_idx[(bh * nb + i) * nb + run + __popc(kb & lt_mask)] = j;
+      run += __popc(kb);
+    }
+    if (row_cnt != nullptr && lane == 0) row_cnt[bh * nb + i] = run;
+    __syncwarp();
+  }
+}
+
+// Column lists (transpose of the bitmask): one warp per 32-column word of one head.
+__global__ void __launch_bounds__(32) col_lists_kernel(const uint32_t* __restrict__ bits, int nb,
+                                                       int nw, int32_t* __restrict__ col_idx,
+                                                       int32_t* __restrict__ col_cnt) {
+  const int w = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const int lane = threadIdx.x;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int mycnt = 0;
+  for (int i0 = 0; i0 < nb; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t word = (i < nb) ? bits[(bh * nb + i) * nw + w] : 0u;
+#pragma unroll 4
+    for (int c = 0; c < 32; ++c) {
+      const bool set = (word >> c) & 1u;
+      const uint32_t b = __ballot_sync(0xffffffffu, set);
+      const int base = __shfl_sync(0xffffffffu, mycnt, c);
+      const int col = 32 * w + c;
+      if (set && col < nb) col_idx[(bh * nb + col) * nb + base + __popc(b & lt_mask)] = i;
+      if (lane == c) mycnt += __popc(b);
+    }
+  }
+  if (32 * w + lane < nb) col_cnt[bh * nb + 32 * w + lane] = mycnt;
+}
+
+// Row lists from a bitmask: one warp per row.
+__global__ void __launch_bounds__(256) row_lists_kernel(const uint32_t* __restrict__ bits, int nb,
+                                                        int nw, long long rows,
+                                                        int32_t* __restrict__ row_idx,
+                                                        int32_t* __restrict__ row_cnt) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  int run = 0;
+  for (int w0 = 0; w0 < nw; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t word = (w < nw) ? bits[row * nw + w] : 0u;
+    if (w == nw - 1 && (nb & 31)) word &= (1u << (nb & 31)) - 1u;
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int pos = run + incl - c;
+    while (word) {
+      const int b = __ffs(word) - 1;
+      row_idx[row * nb + pos++] = 32 * w + b;
+      word &= word - 1u;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) row_cnt[row] = run;
+}
+
+int rows_per_cta(int nb) {
+  int r = kRowBudget / (nb * 8);
+  return r < 1 ? 1 : (r > 8 ? 8 : r);
+}
+
+size_t mask_rows_smem(int nb, int D, int R) {
+  return static_cast<size_t>(kWarps) * 256 * (8 + 4) + static_cast<size_t>(R) * D * 8 +
+         static_cast<size_t>(KC) * (D + 1) * 8 + static_cast<size_t>(R) * nb * 8;
+}
+
+template <int D>
+cudaError_t launch_mask_rows(const double* qp, const double* kp, const Dims& d, double scale,
+                             double thr, const nabla_window& w, uint32_t* bits, int32_t* ridx,
+                             int32_t* rcnt, cudaStream_t st) {
+  const int R = rows_per_cta(d.nb);
+  const size_t smem = mask_rows_smem(d.nb, D, R);
+  cudaError_t e = cudaFuncSetAttribute(mask_rows_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int sta_on = (w.t | w.h | w.w) != 0;
+  dim3 grid((d.nb + R - 1) / R, d.BH);
+  mask_rows_kernel<D><<<grid, kThreads, smem, st>>>(qp, kp, d.nb, d.nw, R, scale, thr, sta_on,
+                                                   w.t / 2, w.h / 2, w.w / 2, d.Hb, d.Wb, bits,
+                                                   ridx, rcnt);
+  return cudaGetLastError();
+}
+
+nabla_status check_lists(const int32_t* idx, const int32_t* cnt) {
+  if ((idx == nullptr) != (cnt == nullptr)) return NABLA_ERR_INVALID_ARG;
+  if (idx && ((reinterpret_cast<uintptr_t>(idx) & 3) || (reinterpret_cast<uintptr_t>(cnt) & 3)))
+    return NABLA_ERR_INVALID_ARG;
+  return NABLA_OK;
+}
+
+cudaError_t launch_col_lists(const uint32_t* bits, const Dims& d, int32_t* cidx, int32_t* ccnt,
+                             cudaStream_t st) {
+  dim3 grid(d.nw, d.BH);
+  col_lists_kernel<<<grid, 32, 0, st>>>(bits, d.nb, d.nw, cidx, ccnt);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace nabla
+
+using namespace nabla;
+
+extern "C" size_t nabla_mask_workspace_bytes(nabla_shape s) {
+  Dims d;
+  if (check_shape(s, &d) != NABLA_OK) return 0;
+  const size_t pool = align_up(static_cast<size_t>(d.BH) * d.nb * d.D * sizeof(double), 256);
+  return kStatusBytes + 2 * pool;
+}
+
+extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const double* q_pool,
+                                         const double* k_pool, nabla_shape s, double thr,
+                                         nabla_window sta, double scale, uint32_t* mask_bits,
+                                         int32_t* row_idx, int32_t* row_cnt, int32_t* col_idx,
+                                         int32_t* col_cnt, void* workspace,
+                                         size_t workspace_bytes, nabla_stream_t stream) {
+  Dims d;
+  nabla_status rc = check_shape(s, &d);
+  if (rc != NABLA_OK) return rc;
+  if (!(thr >= 0.0 && thr <= 1.0)) return NABLA_ERR_INVALID_ARG;   // also rejects NaN
+  if (!(scale > 0.0) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
+  const int sizes[3] = {sta.t, sta.h, sta.w};
+  const bool sta_off = sta.t == 0 && sta.h == 0 && sta.w == 0;
+  if (!sta_off)
+    for (int a = 0; a < 3; ++a)
+      if (sizes[a] < 1 || (sizes[a] % 2) == 0) return NABLA_ERR_INVALID_ARG;
+  if (!mask_bits || (reinterpret_cast<uintptr_t>(mask_bits) & 3)) return NABLA_ERR_INVALID_ARG;
+  if ((rc = check_lists(row_idx, row_cnt)) != NABLA_OK) return rc;
+  if ((rc = check_lists(col_idx, col_cnt)) != NABLA_OK) return rc;
+  if (!q_pool && (!q || !aligned16(q))) return NABLA_ERR_INVALID_ARG;
+  if (!k_pool && (!k || !aligned16(k))) return NABLA_ERR_INVALID_ARG;
+  if ((q_pool && (reinterpret_cast<uintptr_t>(q_pool) & 7)) ||
+      (k_pool && (reinterpret_cast<uintptr_t>(k_pool) & 7)))
+    return NABLA_ERR_INVALID_ARG;
+  const size_t need = nabla_mask_workspace_bytes(s);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return NABLA_ERR_WORKSPACE;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t pool_bytes = align_up(static_cast<size_t>(d.BH) * d.nb * d.D * sizeof(double), 256);
+  double* qp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes);
+  double* kp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes + pool_bytes);
+  cudaError_t e = cudaSuccess;
+  const double* qp = q_pool;
+  const double* kp = k_pool;
+  if (!qp) {
+    if ((e = pool_blocks_device(q, qp_ws, d, st)) != cudaSuccess) return cuda_status(e);
+    qp = qp_ws;
+  }
+  if (!kp) {
+    if ((e = pool_blocks_device(k, kp_ws, d, st)) != cudaSuccess) return cuda_status(e);
+    kp = kp_ws;
+  }
+  e = d.D == 64 ? launch_mask_rows<64>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt, st)
+                : launch_mask_rows<128>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (col_idx) {
+    if ((e = launch_col_lists(mask_bits, d, col_idx, col_cnt, st)) != cudaSuccess) return cuda_status(e);
+  }
+  return NABLA_OK;
+}
+
+extern "C" nabla_status nabla_mask_lists(const uint32_t* mask_bits, nabla_shape s, int32_t* row_idx,
+                                         int32_t* row_cnt, int32_t* col_idx, int32_t* col_cnt,
+                                         nabla_stream_t stream) {
+  Dims d;
+  nabla_status rc = check_shape(s, &d);
+  if (rc != NABLA_OK) return rc;
+  if (!mask_bits || (reinterpret_cast<uintptr_t>(mask_bits) & 3)) return NABLA_ERR_INVALID_ARG;
+  if ((rc = check_lists(row_idx, row_cnt)) != NABLA_OK) return rc;
+  if ((rc = check_lists(col_idx, col_cnt)) != NABLA_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (row_idx) {
+    const long long rows = static_cast<long long>(d.BH) * d.nb;
+    row_lists_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(mask_bits, d.nb, d.nw,
+                                                                          rows, row_idx, row_cnt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+  }
+  if (col_idx) {
+    if ((e = launch_col_lists(mask_bits, d, col_idx, col_cnt, st)) != cudaSuccess) return cuda_status(e);
+  }
+  return NABLA_OK;
+}

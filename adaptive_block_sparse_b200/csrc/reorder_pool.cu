@@ -1,0 +1,126 @@
+// Fractal-flatten token reorder and block mean pooling (HBM-bound).
+//
+// "NABLA: Neighborhood Adaptive Block-Level Attention" (gist.science, Chinese edition),
+// technical summary, Methodology: "token reordering (fractal flatten)" groups the tokens
+// of every P x P spatial patch into one contiguous run with frames kept in order, and
+// "adaptive mask construction / downsampling" average-pools Q and K per block.
+//
+// One CTA moves one block of N = 64 tokens of one (b, h): 64 rows of D bf16.  In
+// natural order a patch row (8 tokens of one image row) is one contiguous run of
+// 8 * D * 2 bytes, so every warp issues 16-byte loads over 512-byte contiguous spans;
+// the reordered block is one contiguous 64 * D * 2-byte run.  The optional pool sums
+// the block's 64 rows column by column in fp64, in token order (exact for bf16), and
+// divides by 64.
+#include "common.cuh"
+
+namespace nabla {
+
+namespace {
+
+constexpr int kThreads = 128;
+
+// GATHER: the source is in natural order (forward reorder); otherwise the source block
+// is contiguous (already reordered).  SCATTER: the destination is natural order
+// (inverse reorder).  WRITE: write a destination at all.  POOL: emit fp64 block means.
+template <int D, bool GATHER, bool SCATTER, bool WRITE, bool POOL>
+__global__ void __launch_bounds__(kThreads) reorder_pool_kernel(
+    const uint4* __restrict__ src, uint4* __restrict__ dst, double* __restrict__ pool_out,
+    int Hg, int W, int Hb, int Wb, int nb) {
+  constexpr int V = D / 8;            // uint4 chunks per token row
+  constexpr int kChunks = 64 * V;     // per block
+  constexpr int kPer = kChunks / kThreads;
+  __shared__ __align__(16) uint4 tile[POOL ? kChunks : 1];
+
+  const int blk = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const long long S = static_cast<long long>(nb) * 64;
+  const int t = blk / (Hb * Wb);
+  const int rem = blk - t * (Hb * Wb);
+  const int hb = rem / Wb;
+  const int wb = rem - hb * Wb;
+  const long long head_base = bh * S;   // in tokens
+
+  uint4 regs[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int e = threadIdx.x + u * kThreads;
+    const int tt = e / V;
+    const int c = e - tt * V;
+    const long long nat =
+        (static_cast<long long>(t) * Hg + hb * 8 + (tt >> 3)) * W + wb * 8 + (tt & 7);
+    const long long frac = static_cast<long long>(blk) * 64 + tt;
+    const long long s_tok = GATHER ? nat : frac;
+    regs[u] = __ldg(src + (head_base + s_tok) * V + c);
+    if constexpr (WRITE) {
+      const long long d_tok = SCATTER ? nat : frac;
+      dst[(head_base + d_tok) * V + c] = regs[u];
+    }
+    if constexpr (POOL) tile[e] = regs[u];
+  }
+  if constexpr (POOL) {
+    __syncthreads();
+    if (threadIdx.x < D) {
+      const __nv_bfloat16* tb = reinterpret_cast<const __nv_bfloat16*>(tile);
+      double acc = 0.0;
+#pragma unroll 8
+      for (int tt = 0; tt < 64; ++tt) acc += static_cast<double>(__bfloat162float(tb[tt * D + threadIdx.x]));
+      pool_out[(bh * nb + blk) * D + threadIdx.x] = acc / 64.0;
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims& d, int inverse,
+                           cudaStream_t st) {
+  dim3 grid(d.nb, d.BH);
+  const uint4* s = static_cast<const uint4*>(src);
+  uint4* o = static_cast<uint4*>(dst);
+  if (inverse) {
+    reorder_pool_kernel<D, false, true, true, false>
+        <<<grid, kThreads, 0, st>>>(s, o, nullptr, d.Hg, d.W, d.Hb, d.Wb, d.nb);
+  } else if (pool) {
+    reorder_pool_kernel<D, true, false, true, true>
+        <<<grid, kThreads, 0, st>>>(s, o, pool, d.Hg, d.W, d.Hb, d.Wb, d.nb);
+  } else {
+    reorder_pool_kernel<D, true, false, true, false>
+        <<<grid, kThreads, 0, st>>>(s, o, nullptr, d.Hg, d.W, d.Hb, d.Wb, d.nb);
+  }
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_pool_only(const void* x, double* pool, const Dims& d, cudaStream_t st) {
+  dim3 grid(d.nb, d.BH);
+  reorder_pool_kernel<D, false, false, false, true><<<grid, kThreads, 0, st>>>(
+      static_cast<const uint4*>(x), nullptr, pool, d.Hg, d.W, d.Hb, d.Wb, d.nb);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Pools a reordered bf16 tensor into fp64 block means (used by the mask build).
+cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st) {
+  return d.D == 64 ? launch_pool_only<64>(x, pool, d, st) : launch_pool_only<128>(x, pool, d, st);
+}
+
+}  // namespace nabla
+
+using namespace nabla;
+
+extern "C" nabla_status nabla_reorder(const void* src, void* dst, double* pool_out,
+                                      nabla_shape s, int32_t inverse, nabla_stream_t stream) {
+  Dims d;
+  nabla_status rc = check_shape(s, &d);
+  if (rc != NABLA_OK) return rc;
+  if (!src || !dst) return NABLA_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return NABLA_ERR_INVALID_ARG;
+  if (pool_out && (inverse || (reinterpret_cast<uintptr_t>(pool_out) & 7))) return NABLA_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(d.BH) * d.S * d.D * 2;
+  const char* a = static_cast<const char*>(src);
+  const char* b = static_cast<const char*>(dst);
+  if (a < b + bytes && b < a + bytes) return NABLA_ERR_INVALID_ARG;   // overlap
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = d.D == 64 ? launch_reorder<64>(src, dst, pool_out, d, inverse, st)
+                            : launch_reorder<128>(src, dst, pool_out, d, inverse, st);
+  return cuda_status(e);
+}

@@ -1,0 +1,487 @@
+"""Benchmark of the NABLA hot path on B200 (one JSON line on stdout, rank 0).
+
+A step is one pass of the whole hot path over one batch of synthetic video-latent input
+already resident in HBM:
+  reorder Q, K, V (fused block pooling of Q and K)  ->  adaptive mask build (pooled
+  scores, softmax, CDF threshold, optional STA union)  ->  block-sparse attention forward
+  [-> backward for the training workload].
+The headline value is the kept-block throughput of the whole step: kept (query block,
+key block) tiles x 4*64*64*D FLOPs (x 3.5 with the backward: 2 + 5 GEMMs) / step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan720p] [--impl ours]
+  python bench.py --impl reference ...     # the CPU oracle arm (host cores)
+
+Multi-GPU: heads are independent, so every rank runs its own copy of the workload
+(weak scaling, no data-path collective); the step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, make_dout, make_qkv  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "NABLA attn fwd ms & TFLOP/s (kept blocks), % bf16 TC peak, vs dense; mask GB/s"
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK}, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+# --------------------------------------------------------------------------------------
+# clocks sampler (nvidia-smi during the timed region)
+# --------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        time.sleep(0.05)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------------------
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------------------
+# the CUDA path
+# --------------------------------------------------------------------------------------
+class Path:
+    """Buffers and the step of the hot path for one workload on one GPU."""
+
+    def __init__(self, wl, dev):
+        import adaptive_block_sparse_b200 as m
+        self.m = m
+        self.wl = wl
+        self.dev = dev
+        self.shape = m.Shape(wl.B, wl.H, wl.T, wl.Hg, wl.W, wl.D, wl.P)
+        sh = self.shape
+        self.thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
+        self.q, self.k, self.v = make_qkv(wl, device=dev)          # natural order
+        self.qf, self.kf, self.vf = (torch.empty_like(self.q) for _ in range(3))
+        self.qp = torch.empty(wl.B, wl.H, sh.nb, wl.D, dtype=torch.float64, device=dev)
+        self.kp = torch.empty_like(self.qp)
+        self.bits, self.ridx, self.rcnt, self.cidx, self.ccnt = m.alloc_mask(
+            sh, dev, cols=wl.backward)
+        self.mask_ws = torch.zeros(m.nabla_mask_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        self.fwd_ws = torch.zeros(m.nabla_fwd_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        self.o_dtype = m.NABLA_F32 if wl.backward else m.NABLA_BF16
+        self.o = torch.empty(self.q.shape, device=dev,
+                             dtype=torch.float32 if wl.backward else torch.bfloat16)
+        self.lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=dev)
+        if wl.backward:
+            self.do = make_dout(wl, device=dev)
+            self.dq, self.dk, self.dv = (torch.empty(self.q.shape, dtype=torch.float32, device=dev)
+                                         for _ in range(3))
+            self.bwd_ws = torch.zeros(m.nabla_bwd_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        self.ev = {}
+
+    def launches_per_step(self):
+        return 3 + 1 + (1 if self.wl.backward else 0) + 1 + (3 if self.wl.backward else 0)
+
+    def _mark(self, name, timing):
+        if timing:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            self.ev.setdefault(name, []).append(e)
+
+    def step(self, timing=False):
+        m, sh, wl = self.m, self.shape, self.wl
+        self._mark("t0", timing)
+        m.nabla_reorder(self.q, self.qf, sh, pool_out=self.qp)
+        m.nabla_reorder(self.k, self.kf, sh, pool_out=self.kp)
+        m.nabla_reorder(self.v, self.vf, sh)
+        self._mark("t_reorder", timing)
+        m.nabla_build_mask(None, None, sh, self.thr, wl.window, mask_bits=self.bits,
+                           row_idx=self.ridx, row_cnt=self.rcnt, col_idx=self.cidx,
+                           col_cnt=self.ccnt, q_pool=self.qp, k_pool=self.kp,
+                           workspace=self.mask_ws)
+        self._mark("t_mask", timing)
+        m.nabla_attn_fwd(self.qf, self.kf, self.vf, self.ridx, self.rcnt, sh, o=self.o,
+                         o_dtype=self.o_dtype, lse=self.lse, workspace=self.fwd_ws)
+        self._mark("t_fwd", timing)
+        if wl.backward:
+            m.nabla_attn_bwd(self.qf, self.kf, self.vf, self.o, self.do, self.lse, self.ridx,
+                             self.rcnt, self.cidx, self.ccnt, sh, dq=self.dq, dk=self.dk,
+                             dv=self.dv, workspace=self.bwd_ws)
+            self._mark("t_bwd", timing)
+
+    def segment_ms(self, a, b):
+        return [x.elapsed_time(y) for x, y in zip(self.ev[a], self.ev[b])]
+
+    def kept_pairs(self):
+        return int(self.rcnt.to(torch.int64).sum().item())
+
+    def check_status(self):
+        for ws in [self.fwd_ws] + ([self.bwd_ws] if self.wl.backward else []):
+            code = self.m.nabla_read_device_status(ws)
+            if code:
+                raise RuntimeError(f"device status 0x{code:x}")
+
+
+def time_call(fn, iters, warm=2):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(iters):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+# --------------------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+# --------------------------------------------------------------------------------------
+def oracle_sample(wl, q_nat, k_nat, v_nat, rcnt, budget_s=20.0):
+    """Times the CPU oracle on a bounded sample and extrapolates the whole step.
+
+    Sample: the oracle mask of ``n_mask`` heads (pool -> pooled softmax -> CDF -> STA) and
+    the oracle attention forward of query blocks drawn from several heads.  Full-step time
+    = mask time per head x B*H + kept FLOPs / (oracle attention FLOP rate).
+    """
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    BH = wl.B * wl.H
+    thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
+    scale = 1 / math.sqrt(wl.D)
+    t0 = time.perf_counter()
+    n_mask = 0
+    masks = {}
+    for bh in range(BH):
+        b, h = divmod(bh, wl.H)
+        qf = oracle.reorder(q_nat[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
+        kf = oracle.reorder(k_nat[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
+        mk, _, _ = oracle.nabla_mask(qf, kf, wl.T, wl.Hg, wl.W, wl.P, thr, wl.window)
+        masks[bh] = (qf, kf, mk[0, 0])
+        n_mask += 1
+        if time.perf_counter() - t0 > budget_s * 0.3 or n_mask >= 4:
+            break
+    t_mask = (time.perf_counter() - t0) / n_mask
+    t1 = time.perf_counter()
+    flops = 0.0
+    blocks = 0
+    rng = np.random.default_rng(0)
+    for bh, (qf, kf, mk) in masks.items():
+        b, h = divmod(bh, wl.H)
+        vf = oracle.reorder(v_nat[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
+        for i in rng.choice(wl.nb, size=min(4, wl.nb), replace=False):
+            rows = np.arange(i * wl.N, (i + 1) * wl.N)
+            oracle.block_sparse_attention_rows(qf[0, 0], kf[0, 0], vf[0, 0], mk, wl.N, scale, rows)
+            flops += 4.0 * wl.N * wl.N * wl.D * mk[i].sum()
+            blocks += 1
+        if time.perf_counter() - t1 > budget_s * 0.7:
+            break
+    t_attn = time.perf_counter() - t1
+    rate = flops / max(t_attn, 1e-9)
+    kept_flops = 4.0 * wl.N * wl.N * wl.D * float(rcnt)
+    est = t_mask * BH + kept_flops / rate
+    return {
+        "value": kept_flops / est / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        "threads_blas": os.environ.get("OMP_NUM_THREADS", "default"),
+        "sample": (f"oracle mask of {n_mask} head(s) ({t_mask:.2f} s/head) + oracle forward of "
+                   f"{blocks} query blocks ({flops / 1e9:.2f} GFLOP in {t_attn:.2f} s); full "
+                   f"step extrapolated to {BH} heads and {rcnt} kept tiles: {est:.1f} s"),
+        "est_step_s": est,
+    }
+
+
+# --------------------------------------------------------------------------------------
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    torch.manual_seed(0)
+    q, k, v = make_qkv(wl, device="cpu", heads=list(range(min(4, wl.B * wl.H))))
+    import oracle
+    thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
+    # kept tiles of the sampled heads, scaled to all heads
+    kept = 0
+    nh = min(4, wl.B * wl.H)
+    for bh in range(nh):
+        b, h = divmod(bh, wl.H)
+        qf = oracle.reorder(q[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
+        kf = oracle.reorder(k[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
+        mk, _, _ = oracle.nabla_mask(qf, kf, wl.T, wl.Hg, wl.W, wl.P, thr, wl.window)
+        kept += int(mk.sum())
+    kept_all = kept * (wl.B * wl.H) / nh
+    times = []
+    cb = None
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        cb = oracle_sample(wl, q, k, v, kept_all, budget_s=min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+        if s >= args.warmup:
+            times.append(cb["est_step_s"])
+        del t0
+    est = statistics.median(times)
+    flops = 4.0 * 64 * 64 * wl.D * kept_all
+    val = flops / est / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "H": wl.H,
+                                             "grid": [wl.T, wl.Hg, wl.W], "D": wl.D,
+                                             "thr": thr, "sta": list(wl.window)},
+            "cpu_baseline": {k2: cb[k2] for k2 in ("kind", "cores", "sample")} | {"value": val, "unit": "TFLOP/s"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="wan720p", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+    wl = WORKLOADS[args.config]
+    world, rank, local = init_dist() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk, pk_kind = peaks()
+    path = Path(wl, dev)
+
+    for _ in range(max(3, args.warmup)):
+        path.step()
+    torch.cuda.synchronize()
+    path.check_status()
+    kept = path.kept_pairs()
+    nb = path.shape.nb
+    BH = wl.B * wl.H
+
+    # ---- timed region ---------------------------------------------------------------------
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    path.ev = {}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        path.step(timing=True)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms_local = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms_local, world, dev)
+    path.check_status()
+    fwd_ms = statistics.mean(path.segment_ms("t_mask", "t_fwd"))
+    mask_ms_fused = statistics.mean(path.segment_ms("t_reorder", "t_mask"))
+    reorder_ms = statistics.mean(path.segment_ms("t0", "t_reorder"))
+    bwd_ms = statistics.mean(path.segment_ms("t_fwd", "t_bwd")) if wl.backward else None
+
+    fl_fwd = 4.0 * 64 * 64 * wl.D
+    step_flops = kept * fl_fwd * (3.5 if wl.backward else 1.0)
+    total_flops = sum_over_ranks(step_flops, world, dev)
+    value = total_flops / (ms * 1e-3) / 1e12
+    fwd_tflops = kept * fl_fwd / (fwd_ms * 1e-3) / 1e12
+    bwd_tflops = kept * fl_fwd * 2.5 / (bwd_ms * 1e-3) / 1e12 if wl.backward else None
+
+    # ---- side measurements (outside the timed region) ----------------------------------------
+    m, sh = path.m, path.shape
+    mask_ms = time_call(lambda: m.nabla_build_mask(path.qf, path.kf, sh, path.thr, wl.window,
+                                                   mask_bits=path.bits, row_idx=path.ridx,
+                                                   row_cnt=path.rcnt, workspace=path.mask_ws), 5)
+    mask_bytes = 2 * BH * wl.S * wl.D * 2 + BH * nb * sh.nw * 4
+    reorder_bytes = 3 * 2 * BH * wl.S * wl.D * 2 + 2 * BH * nb * wl.D * 8
+    ones = torch.full((wl.B, wl.H, nb, nb), True)
+    import oracle
+    dense_bits = torch.from_numpy(oracle.pack_mask_bits(ones.numpy()[:1, :1]).view(np.int32)).to(dev)
+    dense_bits = dense_bits.expand(wl.B, wl.H, nb, sh.nw).contiguous()
+    d_ridx = torch.empty(wl.B, wl.H, nb, nb, dtype=torch.int32, device=dev)
+    d_rcnt = torch.empty(wl.B, wl.H, nb, dtype=torch.int32, device=dev)
+    m.nabla_mask_lists(dense_bits, sh, d_ridx, d_rcnt)
+    dense_iters = 2 if nb > 1000 else 5
+    dense_ms = time_call(lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, d_ridx, d_rcnt, sh,
+                                                  o=path.o, o_dtype=path.o_dtype, lse=path.lse,
+                                                  workspace=path.fwd_ws), dense_iters, warm=1)
+    dense_tflops = BH * nb * nb * fl_fwd / (dense_ms * 1e-3) / 1e12
+    path.check_status()
+    # restore the NABLA lists (the dense run reused the output buffers only)
+    del d_ridx, d_rcnt, dense_bits
+
+    # ---- end to end through the public API with host buffers --------------------------------
+    hq, hk, hv = (t.cpu().pin_memory() for t in (path.q, path.k, path.v))
+    ho = torch.empty(path.o.shape, dtype=path.o.dtype).pin_memory()
+    hdo = path.do.cpu().pin_memory() if wl.backward else None
+    hgrads = [torch.empty(path.q.shape, dtype=torch.float32).pin_memory() for _ in range(3)] if wl.backward else []
+    barrier(world)
+    torch.cuda.synchronize()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_s.record()
+    for _ in range(args.e2e_steps):
+        path.q.copy_(hq, non_blocking=True)
+        path.k.copy_(hk, non_blocking=True)
+        path.v.copy_(hv, non_blocking=True)
+        if wl.backward:
+            path.do.copy_(hdo, non_blocking=True)
+        path.step()
+        ho.copy_(path.o, non_blocking=True)
+        for hg, g in zip(hgrads, (path.dq, path.dk, path.dv) if wl.backward else ()):
+            hg.copy_(g, non_blocking=True)
+    e_e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / args.e2e_steps, world, dev)
+    h2d = 3 * path.q.numel() * 2 + (path.do.numel() * 2 if wl.backward else 0)
+    d2h = path.o.numel() * path.o.element_size() + (3 * path.q.numel() * 4 if wl.backward else 0)
+    e2e_value = total_flops / (e2e_ms * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(wl, path.q.cpu(), path.k.cpu(), path.v.cpu(), kept, budget_s=20.0)
+        cpu = {k2: cb[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
+
+    peak_burst = pk["bf16_tflops"]
+    roof = {"bound": "tensor", "kernel": "attn_fwd_kernel<128>" if wl.D == 128 else "attn_fwd_kernel<64>",
+            "achieved": fwd_tflops, "peak": peak_burst, "unit": "TFLOP/s",
+            "frac": fwd_tflops / peak_burst, "peak_kind": f"{pk_kind} burst bf16 dense",
+            "frac_of_sustained": fwd_tflops / pk["bf16_tflops_sustained"],
+            "traffic": None,
+            "algorithmic_per_launch": f"{kept} kept 64x64 tiles x {int(fl_fwd)} FLOP"}
+    sparsity = 1.0 - kept / (BH * nb * nb)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.T, wl.Hg, wl.W],
+                   "D": wl.D, "P": wl.P, "thr": path.thr, "sta": list(wl.window),
+                   "step": "reorder+pool, mask, attn fwd" + (", attn bwd" if wl.backward else ""),
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"heads-replicated x{world}"},
+        "fwd_ms": fwd_ms, "fwd_tflops_kept": fwd_tflops,
+        "dense_fwd_ms": dense_ms, "dense_tflops": dense_tflops, "speedup_vs_dense": dense_ms / fwd_ms,
+        "mask_ms": mask_ms, "mask_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
+        "mask_frac_hbm": mask_bytes / (mask_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+        "mask_ms_from_pools": mask_ms_fused, "reorder_ms": reorder_ms,
+        "reorder_gbs": reorder_bytes / (reorder_ms * 1e-3) / 1e9,
+        "bwd_ms": bwd_ms, "bwd_tflops_kept": bwd_tflops,
+        "kept_tiles": kept, "sparsity": sparsity,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": path.launches_per_step() * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

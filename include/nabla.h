@@ -1,0 +1,179 @@
+/*
+ * nabla.h -- C ABI of the NABLA (Neighborhood Adaptive Block-Level Attention) hot path
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method (arXiv 2507.13546) as described by:
+ *   [ZH-TS]  "NABLA: Neighborhood Adaptive Block-Level Attention", gist.science (Chinese
+ *            edition), technical summary, section "Methodology".
+ *   [LSD-2]  lsdiaocha.cn article on NABLA, section 2 ("core innovation": pooled
+ *            scouting, CDF filtering, exact mapping back to N x N tiles, OR with STA).
+ *   [LSD-4]  same article, section 4 ("technical principles").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are dense, contiguous, row-major [B, H, S, D] with S = T * Hg * W tokens.
+ *    Every call except nabla_reorder's source works in the reordered ("fractal") token
+ *    order: block i = tokens [i*N, (i+1)*N), N = P*P, nb = S / N blocks.
+ *  - bf16 tensors are IEEE bfloat16 stored as uint16.  All pointers are DEVICE pointers
+ *    of the current CUDA device unless stated otherwise.
+ *  - Ownership: the caller allocates and frees every buffer, workspaces included.  The
+ *    library allocates no device memory and keeps no state between calls.
+ *  - Asynchrony: every call only enqueues work on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and returns.  All arguments are validated on the host
+ *    first; when a call returns anything but NABLA_OK nothing has been enqueued.
+ *  - Supported: P = 8 (N = 64), D in {64, 128}, Hg and W multiples of P, B*H >= 1,
+ *    nb <= 16384.  Pointers to bf16/f32 tensors must be 16-byte aligned.
+ *  - Device-side status: kernels that wait on hardware barriers bound every wait; on
+ *    a timeout they record a code in the first 16 bytes of the call's workspace and
+ *    return early.  nabla_read_device_status() reads it.
+ */
+#ifndef NABLA_H_
+#define NABLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nabla_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  NABLA_OK = 0,
+  NABLA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad shape, thr out of range */
+  NABLA_ERR_UNSUPPORTED = 2,  /* valid request outside the supported set (D, P, nb) */
+  NABLA_ERR_WORKSPACE = 3,    /* workspace pointer null or smaller than required */
+  NABLA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (launch, encode) */
+  NABLA_ERR_DEVICE_CHECK = 5  /* a kernel recorded a device-side failure (bounded wait) */
+} nabla_status;
+
+typedef enum { NABLA_BF16 = 0, NABLA_F32 = 1 } nabla_dtype;
+
+/* Problem shape.  S = T*Hg*W, N = P*P, nb = S/N.  Hg is the (padded) latent height. */
+typedef struct {
+  int32_t B, H, T, Hg, W, D, P;
+} nabla_shape;
+
+/* Static STA window in blocks on the (T, Hg/P, W/P) block grid; odd sizes, centred on
+ * the query block and truncated at the grid edges.  {0,0,0} = no STA part. */
+typedef struct {
+  int32_t t, h, w;
+} nabla_window;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *nabla_status_string(nabla_status s);
+
+/* ---------------------------------------------------------------------------------
+ * Token reordering ("fractal flatten")                                       [ZH-TS]
+ * [ZH-TS] Methodology, "token reordering": the tokens of each P x P spatial patch are
+ * grouped into one contiguous run; frames stay in order.  Natural index
+ * n = (t*Hg + h)*W + w maps to r = ((t*Hb + h/P)*Wb + w/P)*N + (h%P)*P + (w%P) with
+ * Hb = Hg/P, Wb = W/P (row-major patches, row-major inside a patch).
+ *
+ * inverse == 0: dst[b,h,r,:] = src[b,h,n(r),:] (natural -> reordered).
+ * inverse != 0: dst[b,h,n(r),:] = src[b,h,r,:] (reordered -> natural).
+ * src, dst: bf16 [B,H,S,D]; must not overlap.
+ * pool_out (nullable, only with inverse == 0): fp64 [B,H,nb,D], the mean of each
+ *   block's N reordered token vectors (sum in token order in fp64, then / N), i.e.
+ *   the pooled Q or K of [ZH-TS] "downsampling", ready for nabla_build_mask.
+ * Errors: INVALID_ARG (nulls, overlap, shape), UNSUPPORTED (D, P), CUDA (launch).
+ * --------------------------------------------------------------------------------- */
+nabla_status nabla_reorder(const void *src, void *dst, double *pool_out, nabla_shape s,
+                           int32_t inverse, nabla_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Adaptive mask construction                                         [ZH-TS, LSD-2]
+ * [ZH-TS] Methodology, "adaptive mask construction": Q and K are average-pooled per
+ * block of N tokens; full attention is computed on the pooled map (logits scaled by
+ * `scale`); each row is softmax-normalised; per row the CDF is taken and the blocks
+ * whose cumulative probability exceeds 1 - thr are kept; the binary mask defines which
+ * N x N tiles are computed.  "Hybrid integration": M = M_nabla OR M_STA.
+ * Ranking inside a row: probability descending, ties by lower block index.  Block j is
+ * kept iff the probability mass ranked strictly before it is < thr (equivalently the
+ * ascending CDF at j is > 1 - thr).  thr >= 1 keeps every block; thr == 0 keeps none,
+ * so the result is the pure STA mask.  The decision is taken in fp64.
+ *
+ * q, k       : bf16 [B,H,S,D] reordered (read only when the matching pool is NULL).
+ * q_pool,
+ * k_pool     : nullable fp64 [B,H,nb,D] block means from nabla_reorder; when given, the
+ *              call reads them instead of q / k (q / k may then be NULL).
+ * thr        : in [0, 1]; scale > 0 (usually 1/sqrt(D)).
+ * sta        : window, {0,0,0} = off; each size must be 0 (all off) or odd >= 1.
+ * mask_bits  : out uint32 [B,H,nb,ceil(nb/32)]; bit (j%32) of word j/32 of row i is 1
+ *              iff query block i attends to key block j.  Padding bits are 0.
+ * row_idx    : out, nullable, int32 [B,H,nb,nb]: kept key blocks of row i ascending in
+ *              row_idx[..,i,0:row_cnt[..,i]]; the rest is not written.
+ * row_cnt    : out int32 [B,H,nb] (required iff row_idx is given).
+ * col_idx,
+ * col_cnt    : out, nullable: the transpose (query blocks that keep key block j,
+ *              ascending), same shapes; used by the backward pass.
+ * workspace  : >= nabla_mask_workspace_bytes(s) bytes, 256-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * --------------------------------------------------------------------------------- */
+size_t nabla_mask_workspace_bytes(nabla_shape s);
+nabla_status nabla_build_mask(const void *q, const void *k, const double *q_pool,
+                              const double *k_pool, nabla_shape s, double thr,
+                              nabla_window sta, double scale, uint32_t *mask_bits,
+                              int32_t *row_idx, int32_t *row_cnt, int32_t *col_idx,
+                              int32_t *col_cnt, void *workspace, size_t workspace_bytes,
+                              nabla_stream_t stream);
+
+/* Row and column lists of an arbitrary block mask (e.g. a dense all-ones mask for the
+ * dense comparator, or a caller-made mask).  Same layouts as nabla_build_mask; any of
+ * the two list pairs may be NULL.  Padding bits of mask_bits are ignored. */
+nabla_status nabla_mask_lists(const uint32_t *mask_bits, nabla_shape s, int32_t *row_idx,
+                              int32_t *row_cnt, int32_t *col_idx, int32_t *col_cnt,
+                              nabla_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Block-sparse attention forward                                    [ZH-TS, LSD-2]
+ * [ZH-TS] Methodology, "expansion" + FlexAttention: exact softmax attention restricted
+ * to the kept N x N tiles.  For token row r of query block i:
+ *   O_r = sum_c softmax_c(scale * Q_r . K_c) V_c over tokens c of the kept key blocks
+ *   of row i;  LSE_r = ln sum_c exp(scale * Q_r . K_c).
+ * A row with no kept block gives O = 0 and LSE = -inf.
+ *
+ * q, k, v    : bf16 [B,H,S,D] reordered.  row_idx / row_cnt as from nabla_build_mask.
+ * o          : out [B,H,S,D], bf16 or f32 per o_dtype.   lse: out f32 [B,H,S] (natural
+ *              log; nullable when not needed).
+ * workspace  : >= nabla_fwd_workspace_bytes(s) bytes (tile schedule + status word).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * --------------------------------------------------------------------------------- */
+size_t nabla_fwd_workspace_bytes(nabla_shape s);
+nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v,
+                            const int32_t *row_idx, const int32_t *row_cnt, nabla_shape s,
+                            float scale, void *o, nabla_dtype o_dtype, float *lse,
+                            void *workspace, size_t workspace_bytes, nabla_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Block-sparse attention backward (mask constant)                   [ZH-TS, LSD-2]
+ * The pages credit NABLA with faster training as well as inference; the binary mask
+ * has no gradient, so gradients flow through attention on the kept tiles only:
+ *   P = exp(scale*Q K^T - LSE), Dr = rowsum(dO * O), dS = P * (dO V^T - Dr),
+ *   dV = P^T dO, dK = scale * dS^T Q, dQ = scale * dS K   (kept tiles only).
+ * q, k, v, dout: bf16 [B,H,S,D]; o: forward output (o_dtype); lse: forward LSE.
+ * row_* and col_* lists from nabla_build_mask / nabla_mask_lists.
+ * dq, dk, dv : out f32 [B,H,S,D] (fully overwritten; deterministic, no atomics).
+ * workspace  : >= nabla_bwd_workspace_bytes(s) bytes.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * --------------------------------------------------------------------------------- */
+size_t nabla_bwd_workspace_bytes(nabla_shape s);
+nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                            nabla_dtype o_dtype, const void *dout, const float *lse,
+                            const int32_t *row_idx, const int32_t *row_cnt,
+                            const int32_t *col_idx, const int32_t *col_cnt, nabla_shape s,
+                            float scale, float *dq, float *dk, float *dv, void *workspace,
+                            size_t workspace_bytes, nabla_stream_t stream);
+
+/* Reads (synchronously on `stream`) the device status word that the kernels of the
+ * last call on `workspace` recorded: 0 = fine, otherwise a code naming the barrier
+ * wait that gave up.  Returns NABLA_ERR_DEVICE_CHECK when the word is non-zero, and
+ * clears it.  `code` (nullable) receives the raw word. */
+nabla_status nabla_read_device_status(void *workspace, uint32_t *code,
+                                      nabla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NABLA_H_ */

@@ -1,0 +1,100 @@
+"""C-ABI library: loads, exports every declared symbol, rejects bad arguments on the host.
+
+No GPU is needed: every call below fails validation before any CUDA call is made.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from adaptive_block_sparse_b200 import build as b
+    b.build()
+    import adaptive_block_sparse_b200 as nb
+    return nb.load_library()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "nabla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nabla_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("nabla_reorder", "nabla_build_mask", "nabla_attn_fwd", "nabla_attn_bwd"):
+        assert n in names
+    assert len(names) >= 10
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import adaptive_block_sparse_b200 as nb
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert set(nb.EXPORTED) == set(_declared_functions())
+
+
+def test_library_is_built_for_sm100a():
+    from adaptive_block_sparse_b200 import build as b
+    assert "arch=compute_100a,code=sm_100a" in " ".join(b.ARCH)
+
+
+def _shape(nb, **kw):
+    base = dict(B=1, H=2, T=2, Hg=16, W=16, D=64, P=8)
+    base.update(kw)
+    return nb._Shape(*[base[k] for k in ("B", "H", "T", "Hg", "W", "D", "P")])
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    import adaptive_block_sparse_b200 as nb
+    A = ctypes.c_void_p(0x10000)       # fake, aligned, never dereferenced
+    Bp = ctypes.c_void_p(0x20000000)
+    mis = ctypes.c_void_p(0x10008)     # not 16-byte aligned
+    st = ctypes.c_void_p(0)
+    good = _shape(nb)
+    INV, UNS, WS = nb.NABLA_ERR_INVALID_ARG, nb.NABLA_ERR_UNSUPPORTED, nb.NABLA_ERR_WORKSPACE
+    # shapes
+    assert lib.nabla_reorder(A, Bp, None, _shape(nb, Hg=12), 0, st) == INV
+    assert lib.nabla_reorder(A, Bp, None, _shape(nb, D=96), 0, st) == UNS
+    assert lib.nabla_reorder(A, Bp, None, _shape(nb, P=4), 0, st) == UNS
+    assert lib.nabla_reorder(A, Bp, None, _shape(nb, B=0), 0, st) == INV
+    # pointers
+    assert lib.nabla_reorder(None, Bp, None, good, 0, st) == INV
+    assert lib.nabla_reorder(mis, Bp, None, good, 0, st) == INV
+    assert lib.nabla_reorder(A, A, None, good, 0, st) == INV              # overlap
+    assert lib.nabla_reorder(A, Bp, A, good, 1, st) == INV                # pool with inverse
+    win = nb._Window(0, 0, 0)
+    ws_need = lib.nabla_mask_workspace_bytes(good)
+    assert ws_need > 256
+
+    def bm(thr=0.5, window=win, scale=0.125, bits=A, ridx=None, rcnt=None, ws=Bp, wsb=ws_need):
+        return lib.nabla_build_mask(A, A, None, None, good, thr, window, scale, bits, ridx, rcnt,
+                                    None, None, ws, wsb, st)
+    assert bm(thr=1.5) == INV
+    assert bm(thr=-0.1) == INV
+    assert bm(thr=float("nan")) == INV
+    assert bm(window=nb._Window(2, 3, 3)) == INV                          # even window
+    assert bm(window=nb._Window(3, 0, 3)) == INV
+    assert bm(scale=0.0) == INV
+    assert bm(bits=None) == INV
+    assert bm(ridx=A, rcnt=None) == INV                                   # list without count
+    assert bm(wsb=ws_need - 1) == WS
+    assert bm(ws=None) == WS
+    assert bm(ws=ctypes.c_void_p(0x20000010)) == WS                       # misaligned workspace
+    fws = lib.nabla_fwd_workspace_bytes(good)
+
+    def fwd(q=A, o=Bp, scale=0.125, odt=0, ws=Bp, wsb=fws, ridx=A):
+        return lib.nabla_attn_fwd(q, A, A, ridx, A, good, scale, o, odt, None, ws, wsb, st)
+    assert fwd(q=None) == INV
+    assert fwd(q=mis) == INV
+    assert fwd(ridx=None) == INV
+    assert fwd(scale=-1.0) == INV
+    assert fwd(odt=7) == INV
+    assert fwd(wsb=fws - 1) == WS
+    assert lib.nabla_fwd_workspace_bytes(_shape(nb, D=96)) == 0
+    assert lib.nabla_status_string(3) == b"NABLA_ERR_WORKSPACE"

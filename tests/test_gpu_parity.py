@@ -1,0 +1,174 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Reorder and pooling: bit-exact.  Masks: bit-exact except blocks whose ranked mass lies
+within 1e-6 of thr (counted).  Attention: max-abs 2e-2 and mean-abs 2e-3 against fp64;
+a bf16 output additionally allows half an ulp of bf16 storage of the reference.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import WORKLOADS, Workload, make_qkv, random_bf16
+from parity_lib import (bits_to_mask, check_close, check_lists, check_lse, check_mask,
+                        gpu_mask, gpu_reorder, nbl, oracle_mask_per_head, shape_of, to64)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+ODD = Workload("odd", B=1, H=3, T=1, Hg=24, W=8, D=128, thrs=(0.8,), sigma=(1.5, 1.5), seed=77)
+ODD64 = Workload("odd64", B=2, H=1, T=3, Hg=8, W=8, D=64, thrs=(0.6,), sigma=(1.0, 1.0), seed=78)
+
+
+@pytest.fixture(scope="module")
+def data():
+    cache = {}
+
+    def get(wl):
+        if wl.name not in cache:
+            q, k, v = make_qkv(wl, device=DEV)
+            cache[wl.name] = (q, k, v)
+        return cache[wl.name]
+    return get
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_reorder_and_pool_bit_exact(data, name):
+    wl = WORKLOADS[name]
+    shape = shape_of(wl)
+    q, _, _ = data(wl)
+    qf, pool = gpu_reorder(q, shape, pool=True)
+    ref = oracle.reorder(q.cpu().view(torch.int16).numpy(), wl.T, wl.Hg, wl.W, wl.P)
+    assert np.array_equal(qf.cpu().view(torch.int16).numpy(), ref)
+    back = torch.empty_like(qf)
+    nbl().nabla_reorder(qf, back, shape, inverse=True)
+    assert torch.equal(back.view(torch.int16), q.view(torch.int16))
+    ref_pool = oracle.pool_blocks(oracle.reorder(to64(q), wl.T, wl.Hg, wl.W, wl.P), wl.N)
+    assert np.array_equal(pool.cpu().numpy(), ref_pool)
+
+
+MASK_CASES = [("tiny", 0.8, (0, 0, 0)), ("small", 0.5, (0, 0, 0)), ("small", 0.8, (0, 0, 0)),
+              ("small", 0.95, (0, 0, 0)), ("small", 0.7, (1, 3, 3)), ("tiny", 1.0, (0, 0, 0)),
+              ("small", 0.0, (3, 1, 3)), ("odd", 0.8, (1, 1, 1)), ("odd64", 0.6, (0, 0, 0))]
+
+
+def _wl(name):
+    return {"odd": ODD, "odd64": ODD64}.get(name) or WORKLOADS[name]
+
+
+@pytest.mark.parametrize("name,thr,window", MASK_CASES)
+def test_mask_parity(data, name, thr, window):
+    wl = _wl(name)
+    shape = shape_of(wl)
+    q, k, _ = data(wl)
+    qf, qp = gpu_reorder(q, shape, pool=True)
+    kf, kp = gpu_reorder(k, shape, pool=True)
+    bits, ridx, rcnt, cidx, ccnt = gpu_mask(qf, kf, shape, thr, window)
+    gm = bits_to_mask(bits, wl.nb)
+    om, E = oracle_mask_per_head(q.cpu(), k.cpu(), wl, thr, window)
+    mism, amb = check_mask(gm, om, E, thr)
+    print(f"{name} thr={thr} sta={window}: sparsity {1 - gm.mean():.4f}, "
+          f"near-threshold {amb}, differing {mism}")
+    check_lists(ridx, rcnt, gm)
+    check_lists(cidx, ccnt, np.swapaxes(gm, -1, -2))
+    # padding bits are zero
+    nw = bits.shape[-1]
+    if wl.nb % 32:
+        last = bits[..., nw - 1].cpu().numpy().view(np.uint32)
+        assert not np.any(last >> np.uint32(wl.nb % 32))
+    # the pooled means from the fused reorder give the identical mask
+    bits2, *_ = gpu_mask(None, None, shape, thr, window, cols=False, q_pool=qp, k_pool=kp)
+    assert torch.equal(bits2, bits)
+
+
+def _fwd_case(data, wl, thr, window, o_dtype):
+    m = nbl()
+    shape = shape_of(wl)
+    q, k, v = data(wl)
+    qf, _ = gpu_reorder(q, shape)
+    kf, _ = gpu_reorder(k, shape)
+    vf, _ = gpu_reorder(v, shape)
+    bits, ridx, rcnt, _, _ = gpu_mask(qf, kf, shape, thr, window, cols=False)
+    lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
+    o, _ = m.nabla_attn_fwd(qf, kf, vf, ridx, rcnt, shape, o_dtype=o_dtype, lse=lse)
+    torch.cuda.synchronize()
+    gm = bits_to_mask(bits, wl.nb)
+    O, L = oracle.block_sparse_attention(to64(qf), to64(kf), to64(vf), gm, wl.N, 1 / math.sqrt(wl.D))
+    return o, lse, O, L, gm
+
+
+@pytest.mark.parametrize("name,thr,window", [("tiny", 0.8, (0, 0, 0)), ("small", 0.8, (0, 0, 0)),
+                                             ("small", 0.95, (0, 0, 0)), ("small", 0.5, (1, 3, 3)),
+                                             ("odd", 0.8, (0, 0, 0)), ("odd64", 0.6, (0, 0, 0))])
+@pytest.mark.parametrize("o_dtype", ["f32", "bf16"])
+def test_fwd_parity(data, name, thr, window, o_dtype):
+    m = nbl()
+    wl = _wl(name)
+    odt = m.NABLA_F32 if o_dtype == "f32" else m.NABLA_BF16
+    o, lse, O, L, gm = _fwd_case(data, wl, thr, window, odt)
+    mx, mean = check_close(to64(o), O, f"O {name}", storage_bf16=(o_dtype == "bf16"))
+    check_lse(lse.cpu().numpy().astype(np.float64), L)
+    print(f"{name} thr={thr}: density {gm.mean():.4f} max|O| {np.abs(O).max():.2f} "
+          f"max err {mx:.2e} mean err {mean:.2e}")
+
+
+def test_fwd_dense_and_empty_rows(data):
+    """All-ones mask = dense attention; rows with no kept block give O = 0, LSE = -inf."""
+    m = nbl()
+    wl = WORKLOADS["small"]
+    shape = shape_of(wl)
+    q, k, v = data(wl)
+    qf, _ = gpu_reorder(q, shape)
+    kf, _ = gpu_reorder(k, shape)
+    vf, _ = gpu_reorder(v, shape)
+    nb, nw = wl.nb, shape.nw
+    rng = np.random.default_rng(5)
+    cases = {"dense": np.ones((wl.B, wl.H, nb, nb), dtype=bool),
+             "holes": rng.random((wl.B, wl.H, nb, nb)) < 0.1}
+    cases["holes"][:, :, 3] = False       # an empty row whose partner row is not empty
+    cases["holes"][:, :, 10:12] = False   # an empty pair of rows
+    for name, mask in cases.items():
+        bits = torch.from_numpy(oracle.pack_mask_bits(mask).view(np.int32)).to(DEV)
+        ridx = torch.empty(wl.B, wl.H, nb, nb, dtype=torch.int32, device=DEV)
+        rcnt = torch.empty(wl.B, wl.H, nb, dtype=torch.int32, device=DEV)
+        m.nabla_mask_lists(bits, shape, ridx, rcnt)
+        lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
+        o, _ = m.nabla_attn_fwd(qf, kf, vf, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse)
+        torch.cuda.synchronize()
+        check_lists(ridx, rcnt, mask)
+        O, L = oracle.block_sparse_attention(to64(qf), to64(kf), to64(vf), mask, wl.N,
+                                             1 / math.sqrt(wl.D))
+        check_close(to64(o), O, f"O {name}")
+        check_lse(lse.cpu().numpy().astype(np.float64), L)
+        if name == "holes":
+            assert torch.all(o[:, :, 3 * 64:4 * 64] == 0)
+            assert torch.all(torch.isneginf(lse[:, :, 10 * 64:12 * 64]))
+
+
+@pytest.mark.parametrize("name,thr,window", [("tiny", 0.8, (0, 0, 0)), ("small", 0.8, (3, 3, 3)),
+                                             ("small", 0.95, (0, 0, 0)), ("odd", 0.8, (1, 1, 1)),
+                                             ("odd64", 0.6, (0, 0, 0))])
+def test_bwd_parity(data, name, thr, window):
+    """dQ, dK, dV (fp32) against the fp64 oracle on the GPU's mask (held constant)."""
+    from synth import make_dout
+    m = nbl()
+    wl = _wl(name)
+    shape = shape_of(wl)
+    q, k, v = data(wl)
+    qf, _ = gpu_reorder(q, shape)
+    kf, _ = gpu_reorder(k, shape)
+    vf, _ = gpu_reorder(v, shape)
+    bits, ridx, rcnt, cidx, ccnt = gpu_mask(qf, kf, shape, thr, window)
+    lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
+    o, _ = m.nabla_attn_fwd(qf, kf, vf, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse)
+    do = make_dout(wl, device=DEV)
+    dq, dk, dv = m.nabla_attn_bwd(qf, kf, vf, o, do, lse, ridx, rcnt, cidx, ccnt, shape)
+    torch.cuda.synchronize()
+    gm = bits_to_mask(bits, wl.nb)
+    rq, rk, rv = oracle.block_sparse_attention_bwd(to64(qf), to64(kf), to64(vf), to64(do), gm, wl.N,
+                                                   1 / math.sqrt(wl.D))
+    for got, ref, what in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+        mx, mean = check_close(to64(got), ref, f"{what} {name}")
+        print(f"{name} {what}: max|ref| {np.abs(ref).max():.2f} max err {mx:.2e} mean err {mean:.2e}")
