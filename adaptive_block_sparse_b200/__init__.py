@@ -34,6 +34,7 @@ NABLA_ERR_CUDA = 4
 NABLA_ERR_DEVICE_CHECK = 5
 NABLA_BF16 = 0
 NABLA_F32 = 1
+NABLA_F16 = 2
 
 EXPORTED = (
     "nabla_status_string", "nabla_reorder", "nabla_mask_workspace_bytes", "nabla_build_mask",
@@ -56,17 +57,18 @@ _i32 = ctypes.c_int32
 
 _sigs = {
     "nabla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
-    "nabla_reorder": (ctypes.c_int, [_vp, _vp, _vp, _Shape, _i32, _vp]),
+    "nabla_reorder": (ctypes.c_int, [_vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _Shape, _i32, _vp]),
     "nabla_mask_workspace_bytes": (_sz, [_Shape]),
     "nabla_build_mask": (ctypes.c_int, [_vp, _vp, _vp, _vp, _Shape, ctypes.c_double, _Window,
                                         ctypes.c_double, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "nabla_mask_lists": (ctypes.c_int, [_vp, _Shape, _vp, _vp, _vp, _vp, _vp]),
     "nabla_fwd_workspace_bytes": (_sz, [_Shape]),
-    "nabla_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _Shape, ctypes.c_float, _vp,
-                                      ctypes.c_int, _vp, _vp, _sz, _vp]),
+    "nabla_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _Shape, ctypes.c_float,
+                                      _vp, ctypes.c_int, _vp, _vp, _sz, _vp]),
     "nabla_bwd_workspace_bytes": (_sz, [_Shape]),
-    "nabla_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
-                                      _vp, _Shape, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nabla_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp,
+                                      _vp, _vp, _vp, _Shape, ctypes.c_float, _vp, _vp, _vp, _vp,
+                                      _sz, _vp]),
     "nabla_read_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
 }
 
@@ -125,6 +127,14 @@ class Shape:
         return _Shape(self.B, self.H, self.T, self.Hg, self.W, self.D, self.P)
 
 
+def dtype_code(t) -> int:
+    """nabla_dtype of a tensor (bf16, f32 or f16)."""
+    codes = {torch.bfloat16: NABLA_BF16, torch.float32: NABLA_F32, torch.float16: NABLA_F16}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -145,9 +155,13 @@ def nabla_status_string(status: int) -> str:
 
 
 def nabla_reorder(src, dst, shape: Shape, inverse=False, pool_out=None, stream=None):
-    """Natural <-> reordered token order (bf16 [B,H,S,D]); optional fp64 block means."""
-    _check(load_library().nabla_reorder(_ptr(src), _ptr(dst), _ptr(pool_out), shape.c(), int(bool(inverse)),
-                              _stream(stream)), "nabla_reorder")
+    """Natural <-> reordered token order ([B,H,S,D]); optional fp64 block means.
+
+    Forward: bf16 ``src`` into a bf16 or fp16 ``dst``.  Inverse: same dtype both sides.
+    """
+    _check(load_library().nabla_reorder(_ptr(src), dtype_code(src), _ptr(dst), dtype_code(dst),
+                                        _ptr(pool_out), shape.c(), int(bool(inverse)),
+                                        _stream(stream)), "nabla_reorder")
     return dst
 
 
@@ -201,7 +215,8 @@ def nabla_attn_fwd(q, k, v, row_idx, row_cnt, shape: Shape, scale=None, o=None,
                         device=q.device)
     if workspace is None:
         workspace = torch.zeros(nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=q.device)
-    _check(load_library().nabla_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(row_idx), _ptr(row_cnt), shape.c(),
+    _check(load_library().nabla_attn_fwd(_ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(row_idx),
+                               _ptr(row_cnt), shape.c(),
                                float(scale), _ptr(o), int(o_dtype), _ptr(lse), _ptr(workspace),
                                workspace.numel(), _stream(stream)), "nabla_attn_fwd")
     return o, lse
@@ -218,7 +233,8 @@ def nabla_attn_bwd(q, k, v, o, dout, lse, row_idx, row_cnt, col_idx, col_cnt, sh
     dv = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dv is None else dv
     if workspace is None:
         workspace = torch.zeros(nabla_bwd_workspace_bytes(shape), dtype=torch.uint8, device=q.device)
-    _check(load_library().nabla_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), o_dtype, _ptr(dout), _ptr(lse),
+    _check(load_library().nabla_attn_bwd(_ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(o), o_dtype,
+                               _ptr(dout), _ptr(lse),
                                _ptr(row_idx), _ptr(row_cnt), _ptr(col_idx), _ptr(col_cnt),
                                shape.c(), float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
                                _ptr(workspace), workspace.numel(), _stream(stream)),

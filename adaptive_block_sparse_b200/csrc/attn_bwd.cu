@@ -25,11 +25,14 @@
 
 #include <cudaTypedefs.h>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace nabla {
 
-bool make_map_bf16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows);
+bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows,
+                 bool fp16);
 
 namespace {
 
@@ -50,29 +53,46 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
 // -------------------------------------------------------------------------------------
 // 1. preprocess: delta = rowsum(dO * O), lse2 = LSE * log2(e)
 // -------------------------------------------------------------------------------------
+// Also writes fp16 copies of Q, K, V and dO for the MMAs of the backward pass: P and dS
+// are then rounded to fp16 (11-bit significand) instead of bf16 (8-bit), which keeps the
+// gradients within 2e-2 of fp64 where bf16 P / dS would not (|dS| reaches ~30).  bf16 ->
+// fp16 is exact for 2^-14 <= |x| <= 65504; smaller magnitudes lose low bits (absolute error
+// below 6e-8); larger ones cannot be represented and are reported as a device status.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const void* __restrict__ o, int o_f32,
-                                                             const __nv_bfloat16* __restrict__ dout,
-                                                             const float* __restrict__ lse,
-                                                             float* __restrict__ delta,
-                                                             float* __restrict__ lse2, long long rows) {
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(
+    const void* __restrict__ o, int o_f32, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const void* __restrict__ v, int v_f16,
+    __half* __restrict__ q16, __half* __restrict__ k16, __half* __restrict__ v16,
+    __half* __restrict__ do16, float* __restrict__ delta, float* __restrict__ lse2,
+    long long rows, uint32_t* status) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   constexpr int E = D / 32;  // elements per lane (contiguous)
+  const long long base = row * D + lane * E;
   float acc = 0.f;
-  const __nv_bfloat16* g = dout + row * D + lane * E;
-  if (o_f32) {
-    const float* f = static_cast<const float*>(o) + row * D + lane * E;
+  bool range_ok = true;
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(g[e]), f[e], acc);
-  } else {
-    const __nv_bfloat16* f = static_cast<const __nv_bfloat16*>(o) + row * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(g[e]), __bfloat162float(f[e]), acc);
+  for (int e = 0; e < E; ++e) {
+    const float g = __bfloat162float(dout[base + e]);
+    const float of = o_f32 ? static_cast<const float*>(o)[base + e]
+                           : __bfloat162float(static_cast<const __nv_bfloat16*>(o)[base + e]);
+    acc = fmaf(g, of, acc);
+    const float qv = __bfloat162float(q[base + e]);
+    const float kv = __bfloat162float(k[base + e]);
+    const float vv = v_f16 ? __half2float(static_cast<const __half*>(v)[base + e])
+                           : __bfloat162float(static_cast<const __nv_bfloat16*>(v)[base + e]);
+    range_ok = range_ok && fabsf(g) <= 65504.f && fabsf(qv) <= 65504.f && fabsf(kv) <= 65504.f &&
+               fabsf(vv) <= 65504.f;
+    do16[base + e] = __float2half_rn(g);
+    q16[base + e] = __float2half_rn(qv);
+    k16[base + e] = __float2half_rn(kv);
+    v16[base + e] = __float2half_rn(vv);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (!__all_sync(0xffffffffu, range_ok) && lane == 0) record_status(status, kDevFp16Range);
   if (lane == 0) {
     delta[row] = acc;
     lse2[row] = lse[row] * kLog2e;
@@ -80,6 +100,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const void* __restr
 }
 
 struct BwdParams {
+  const int32_t* order;      // work items (head * npairs + pair), longest first
+  int npairs;
   const int32_t* list_idx;   // column lists (dK/dV pass) or row lists (dQ pass)
   const int32_t* list_cnt;
   const float* delta;
@@ -170,9 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long bh = blockIdx.y;
+  const int item = prm.order[blockIdx.x];
+  const long long bh = item / prm.npairs;
   const int nb = prm.nb;
-  const int j0 = 2 * blockIdx.x;
+  const int j0 = 2 * (item - static_cast<int>(bh) * prm.npairs);
   const bool has_j1 = (j0 + 1) < nb;
 
   if (threadIdx.x == 0) {
@@ -218,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       wk.c1 = has_j1 ? min(max(prm.list_cnt[bh * nb + j0 + 1], 0), nb) : 0;
       wk.a = wk.b = 0;
       int it = 0;
+      bool ended = false;
       while (true) {
         uint32_t f = 0;
         const int i = wk.next(&f);
@@ -227,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i < 0 || i >= nb) {
           meta[s] = kEnd;
           mbar_arrive(&full[s]);
+          ended = true;
           break;
         }
         meta[s] = static_cast<uint32_t>(i) | (f << 28);
@@ -242,7 +267,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(st + 2 * C::kTileBytes + 256, prm.delta + qrow, 256, &full[s]);
         ++it;
       }
-      const int first = it > L::kStages ? it - L::kStages : 0;
+      // Copies still in flight: the last kStages iterations, except that placing the end
+      // marker waited for the oldest of them to be consumed (its stage was reused), and a
+      // parity wait on that stage would now look two phases back.
+      const int keep = ended ? L::kStages - 1 : L::kStages;
+      const int first = it > keep ? it - keep : 0;
       for (int x = first; x < it; ++x)
         mbar_wait(&full[x % L::kStages], (x / L::kStages) & 1, prm.status, kDevTimeoutDrain);
       mbar_wait(kv_full, 0, prm.status, kDevTimeoutDrain);
@@ -250,8 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_s = idesc_f16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_acc = idesc_f16_f32(128, D, false, true);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       const uint32_t st_addr = smem_u32(sStage);
       const uint32_t pt_addr = smem_u32(sPT), dst_addr = smem_u32(sDST);
@@ -347,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -s_lse[q0 + 1]));
             const float d0 = p0 * (__uint_as_float(dv[c]) - s_del[q0]);
             const float d1 = p1 * (__uint_as_float(dv[c + 1]) - s_del[q0 + 1]);
-            pk[half * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
-            dk[half * 16 + (c >> 1)] = pack_bf16x2(d0, d1);
+            pk[half * 16 + (c >> 1)] = pack_f16x2(p0, p1);
+            dk[half * 16 + (c >> 1)] = pack_f16x2(d0, d1);
           }
         } else {
 #pragma unroll
@@ -451,9 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long bh = blockIdx.y;
+  const int item = prm.order[blockIdx.x];
+  const long long bh = item / prm.npairs;
   const int nb = prm.nb;
-  const int i0 = 2 * blockIdx.x;
+  const int i0 = 2 * (item - static_cast<int>(bh) * prm.npairs);
   const bool has_i1 = (i0 + 1) < nb;
 
   if (threadIdx.x == 0) {
@@ -499,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       wk.c1 = has_i1 ? min(max(prm.list_cnt[bh * nb + i0 + 1], 0), nb) : 0;
       wk.a = wk.b = 0;
       int it = 0;
+      bool ended = false;
       while (true) {
         uint32_t f = 0;
         const int j = wk.next(&f);
@@ -508,6 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j < 0 || j >= nb) {
           meta[s] = kEnd;
           mbar_arrive(&full[s]);
+          ended = true;
           break;
         }
         meta[s] = static_cast<uint32_t>(j) | (f << 28);
@@ -521,7 +553,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++it;
       }
-      const int first = it > L::kStages ? it - L::kStages : 0;
+      // Copies still in flight: the last kStages iterations, except that placing the end
+      // marker waited for the oldest of them to be consumed (its stage was reused), and a
+      // parity wait on that stage would now look two phases back.
+      const int keep = ended ? L::kStages - 1 : L::kStages;
+      const int first = it > keep ? it - keep : 0;
       for (int x = first; x < it; ++x)
         mbar_wait(&full[x % L::kStages], (x / L::kStages) & 1, prm.status, kDevTimeoutDrain);
       mbar_wait(q_full, 0, prm.status, kDevTimeoutDrain);
@@ -529,8 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_s = idesc_f16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_acc = idesc_f16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
       const uint32_t st_addr = smem_u32(sStage), ds_addr = smem_u32(sDS);
       auto issue_sd = [&](int x) {
@@ -619,8 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 32; c += 2) {
             const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -my_lse2));
             const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -my_lse2));
-            dk[half * 16 + (c >> 1)] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - my_delta),
-                                                   p1 * (__uint_as_float(dv[c + 1]) - my_delta));
+            dk[half * 16 + (c >> 1)] = pack_f16x2(p0 * (__uint_as_float(dv[c]) - my_delta),
+                                                  p1 * (__uint_as_float(dv[c + 1]) - my_delta));
           }
         } else {
 #pragma unroll
@@ -670,24 +706,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* o, int o_f32,
+cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, const void* o, int o_f32,
                        const void* dout, const float* lse, const int32_t* ridx, const int32_t* rcnt,
                        const int32_t* cidx, const int32_t* ccnt, const Dims& d, float scale,
                        float* dq, float* dk, float* dv, void* ws, cudaStream_t st, bool* map_ok) {
   const long long rows = static_cast<long long>(d.BH) * d.S;
   float* delta = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
   float* lse2 = delta + align_up(static_cast<size_t>(rows), 64);
+  char* sched = reinterpret_cast<char*>(lse2 + align_up(static_cast<size_t>(rows), 64));
+  __half* h16 = reinterpret_cast<__half*>(sched + 2 * schedule_scratch_bytes(d));
+  const size_t tensor_elems = static_cast<size_t>(rows) * D;
+  __half *q16 = h16, *k16 = h16 + tensor_elems, *v16 = h16 + 2 * tensor_elems,
+         *do16 = h16 + 3 * tensor_elems;
   uint32_t* status = static_cast<uint32_t*>(ws);
-  bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-      o, o_f32, static_cast<const __nv_bfloat16*>(dout), lse, delta, lse2, rows);
-  cudaError_t e = cudaGetLastError();
+  int32_t* order_cols = nullptr;
+  int32_t* order_rows = nullptr;
+  cudaError_t e = build_schedule(ccnt, d, sched, &order_cols, st);
+  if (e == cudaSuccess) e = build_schedule(rcnt, d, sched + schedule_scratch_bytes(d), &order_rows, st);
   if (e != cudaSuccess) return e;
+  bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      o, o_f32, static_cast<const __nv_bfloat16*>(dout), lse, static_cast<const __nv_bfloat16*>(q),
+      static_cast<const __nv_bfloat16*>(k), v, v_f16, q16, k16, v16,
+      do16, delta, lse2, rows, status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128, mk64, mv64;
-  *map_ok = make_map_bf16(&mq64, q, rows, D, 64) && make_map_bf16(&mdo64, dout, rows, D, 64) &&
-            make_map_bf16(&mk128, k, rows, D, 128) && make_map_bf16(&mv128, v, rows, D, 128) &&
-            make_map_bf16(&mq128, q, rows, D, 128) && make_map_bf16(&mdo128, dout, rows, D, 128) &&
-            make_map_bf16(&mk64, k, rows, D, 64) && make_map_bf16(&mv64, v, rows, D, 64);
+  *map_ok = make_map_16(&mq64, q16, rows, D, 64, true) && make_map_16(&mdo64, do16, rows, D, 64, true) &&
+            make_map_16(&mk128, k16, rows, D, 128, true) && make_map_16(&mv128, v16, rows, D, 128, true) &&
+            make_map_16(&mq128, q16, rows, D, 128, true) && make_map_16(&mdo128, do16, rows, D, 128, true) &&
+            make_map_16(&mk64, k16, rows, D, 64, true) && make_map_16(&mv64, v16, rows, D, 64, true);
   if (!*map_ok) return cudaErrorInvalidValue;
 
   BwdParams p;
@@ -698,8 +745,10 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
   p.S = d.S;
   p.scale_log2 = scale * kLog2e;
   p.scale = scale;
-  dim3 grid((d.nb + 1) / 2, d.BH);
+  const unsigned grid = static_cast<unsigned>(d.BH) * static_cast<unsigned>((d.nb + 1) / 2);
+  p.npairs = (d.nb + 1) / 2;
 
+  p.order = order_cols;
   p.list_idx = cidx;
   p.list_cnt = ccnt;
   p.out0 = dv;
@@ -710,6 +759,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
   attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk128, mv128, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
+  p.order = order_rows;
   p.list_idx = ridx;
   p.list_cnt = rcnt;
   p.out0 = dq;
@@ -730,10 +780,12 @@ extern "C" size_t nabla_bwd_workspace_bytes(nabla_shape s) {
   Dims d;
   if (check_shape(s, &d) != NABLA_OK) return 0;
   const size_t rows = align_up(static_cast<size_t>(d.BH) * d.S, 64);
-  return kStatusBytes + 2 * rows * sizeof(float);
+  return kStatusBytes + 2 * rows * sizeof(float) + 2 * schedule_scratch_bytes(d) +
+         4 * static_cast<size_t>(d.BH) * d.S * d.D * 2;
 }
 
-extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void* v,
+                                       nabla_dtype v_dtype, const void* o,
                                        nabla_dtype o_dtype, const void* dout, const float* lse,
                                        const int32_t* row_idx, const int32_t* row_cnt,
                                        const int32_t* col_idx, const int32_t* col_cnt,
@@ -753,6 +805,7 @@ extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void*
   for (const void* p : al4)
     if (reinterpret_cast<uintptr_t>(p) & 3) return NABLA_ERR_INVALID_ARG;
   if (o_dtype != NABLA_BF16 && o_dtype != NABLA_F32) return NABLA_ERR_INVALID_ARG;
+  if (v_dtype != NABLA_BF16 && v_dtype != NABLA_F16) return NABLA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < nabla_bwd_workspace_bytes(s) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -762,9 +815,9 @@ extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void*
   cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
   if (e != cudaSuccess) return cuda_status(e);
   bool map_ok = true;
-  e = d.D == 64 ? launch_bwd<64>(q, k, v, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
+  e = d.D == 64 ? launch_bwd<64>(q, k, v, v_dtype == NABLA_F16, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
                                  col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok)
-                : launch_bwd<128>(q, k, v, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
+                : launch_bwd<128>(q, k, v, v_dtype == NABLA_F16, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
                                   col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok);
   return cuda_status(e);
 }

@@ -34,21 +34,21 @@ constexpr uint32_t kEnd = 0xFFFFFFFFu;    // end-of-list marker in the stage met
 template <int D>
 struct FwdCfg {
   static constexpr int kPanels = D / 64;                  // 128-byte swizzle panels
-  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kStages = (D == 128) ? 2 : 4;   // two CTAs per SM
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVTileBytes = 64 * D * 2;         // one K or one V tile
-  static constexpr int kPBytes = 128 * 64 * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVTileBytes;
-  static constexpr int kOffP = kOffV + kStages * kKVTileBytes;
-  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kOffBar = kOffV + kStages * kKVTileBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 256;              // S0 | S1 | O
   static constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;
 };
 
 struct FwdParams {
+  const int32_t* order;      // work items (head * npairs + pair), longest first
+  int npairs;
   const int32_t* row_idx;
   const int32_t* row_cnt;
   void* o;
@@ -60,8 +60,8 @@ struct FwdParams {
   int o_f32;
 };
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool VF16>
+__global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const FwdParams prm) {
@@ -72,22 +72,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sK = smem + C::kOffK;
   unsigned char* sV = smem + C::kOffV;
-  unsigned char* sP = smem + C::kOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;                       // [kStages]
   uint64_t* empty = bars + C::kStages;         // [kStages]
   uint64_t* q_full = bars + 2 * C::kStages;
   uint64_t* s_full = q_full + 1;               // [2]
   uint64_t* p_full = s_full + 2;               // [2]
-  uint64_t* o_bar = p_full + 2;
-  uint64_t* drain = o_bar + 1;
+  uint64_t* o_bar = p_full + 2;                // one phase per PV (rescale waits)
+  uint64_t* o_final = o_bar + 1;               // single phase: every PV has landed
+  uint64_t* drain = o_final + 1;
   uint32_t* meta = reinterpret_cast<uint32_t*>(drain + 1);   // [kStages]
   uint32_t* tmem_slot = meta + C::kStages;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int pair = blockIdx.x;
-  const long long bh = blockIdx.y;
+  const int item = prm.order[blockIdx.x];
+  const long long bh = item / prm.npairs;
+  const int pair = item - static_cast<int>(bh) * prm.npairs;
   const int nb = prm.nb;
   const int i0 = 2 * pair;
   const bool has_i1 = (i0 + 1) < nb;
@@ -103,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&p_full[0], 128);
     mbar_init(&p_full[1], 128);
     mbar_init(o_bar, 1);
+    mbar_init(o_final, 1);
     mbar_init(drain, 1);
     fence_mbarrier_init();
   }
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c0 = min(max(prm.row_cnt[bh * nb + i0], 0), nb);
       const int c1 = has_i1 ? min(max(prm.row_cnt[bh * nb + i0 + 1], 0), nb) : 0;
       int a = 0, b = 0, it = 0;
-      bool ok = true;
+      bool ok = true, ended = false;
       while (true) {
         int j = -1;
         uint32_t f = 0;
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j < 0) {
           meta[s] = kEnd;
           mbar_arrive(&full[s]);
+          ended = true;
           break;
         }
         meta[s] = static_cast<uint32_t>(j) | (f << 28);
@@ -162,7 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every issued copy must have landed before the CTA may exit.
       (void)ok;
-      const int first = it > C::kStages ? it - C::kStages : 0;
+      // Copies still in flight: the last kStages iterations, except that placing the end
+      // marker waited for the oldest of them to be consumed (its stage was reused), and a
+      // parity wait on that stage would now look two phases back.
+      const int keep = ended ? C::kStages - 1 : C::kStages;
+      const int first = it > keep ? it - keep : 0;
       for (int x = first; x < it; ++x)
         mbar_wait(&full[x % C::kStages], (x / C::kStages) & 1, prm.status, kDevTimeoutDrain);
       mbar_wait(q_full, 0, prm.status, kDevTimeoutDrain);
@@ -172,11 +179,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_o = VF16 ? idesc_f16_f32(128, D, false, true)
+                                        : idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
-      const uint32_t p_addr = smem_u32(sP);
       auto issue_s = [&](int x) {
         const int st = x % C::kStages;
         const uint32_t d_tmem = tmem + ((x & 1) ? C::kColS1 : C::kColS0);
@@ -189,13 +196,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&s_full[x & 1]);
       };
+      // O += P V with P (bf16) read from TMEM where the softmax warps stored it, over the
+      // first 32 columns of the score buffer it came from.
       auto issue_pv = [&](int x) {
         const int st = x % C::kStages;
+        const uint32_t p_tmem = tmem + ((x & 1) ? C::kColS1 : C::kColS0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = sdesc_sw128(p_addr + (x & 1) * C::kPBytes + kk * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(v_addr + st * C::kKVTileBytes + kk * 2048, 8192, 1024);
-          mma_bf16_ss(tmem + C::kColO, ad, bd, idesc_o, (x > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::kColO, p_tmem + kk * 8, bd, idesc_o, (x > 0 || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(q_full, 0, prm.status, kDevTimeoutQFull);
@@ -218,6 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (end1) break;
         }
       }
+      // o_final completes once when every MMA issued above has finished; the epilogue
+      // waits on it (a per-PV parity wait could be satisfied two phases early).
+      mma_commit(o_final);
       // Drain: all MMAs of this CTA complete before TMEM is released.
       mma_commit(drain);
       mbar_wait(drain, 0, prm.status, kDevTimeoutDrain);
@@ -233,7 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l = 0.f;
     int it = 0;
     bool ok = true;
-    unsigned char* prow = sP + row * 128;
     for (;; ++it) {
       const int s = it % C::kStages;
       ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (it / C::kStages) & 1, prm.status, kDevTimeoutTmaFull));
@@ -285,32 +296,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       }
-      uint32_t packed[32];
-      if (keep) {
-        float sum = 0.f;
+      // P = 2^(s*scale*log2e - m) as bf16 pairs, written over the score buffer in TMEM.
+      // Every fourth element uses the FMA-pipe exponential to offload the MUFU unit.
+      const uint32_t pcol = tmem + lane_base + ((it & 1) ? C::kColS1 : C::kColS0);
+      float sum = 0.f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sa[2 * c]), sl2, -m_ref));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sa[2 * c + 1]), sl2, -m_ref));
-          const float p2 = fast_exp2(fmaf(__uint_as_float(sb[2 * c]), sl2, -m_ref));
-          const float p3 = fast_exp2(fmaf(__uint_as_float(sb[2 * c + 1]), sl2, -m_ref));
-          sum += (p0 + p1) + (p2 + p3);
-          packed[c] = pack_bf16x2(p0, p1);
-          packed[16 + c] = pack_bf16x2(p2, p3);
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t (&sv)[32] = half ? sb : sa;
+        uint32_t packed[16];
+        if (keep) {
+#pragma unroll
+          for (int c = 0; c < 16; c += 2) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl2, -m_ref));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -m_ref));
+            const float p2 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 2]), sl2, -m_ref));
+            const float p3 = poly_exp2(fmaf(__uint_as_float(sv[2 * c + 3]), sl2, -m_ref));
+            // The row sum takes the rounded weights that enter the PV product, so the
+            // output is an exact convex combination of those weights.
+            if constexpr (VF16) {
+              packed[c] = pack_f16x2(p0, p1);
+              packed[c + 1] = pack_f16x2(p2, p3);
+              sum += (f16lo(packed[c]) + f16hi(packed[c])) + (f16lo(packed[c + 1]) + f16hi(packed[c + 1]));
+            } else {
+              packed[c] = pack_bf16x2(p0, p1);
+              packed[c + 1] = pack_bf16x2(p2, p3);
+              sum += (bf16lo(packed[c]) + bf16hi(packed[c])) + (bf16lo(packed[c + 1]) + bf16hi(packed[c + 1]));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) packed[c] = 0u;
         }
-        l += sum;
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) packed[c] = 0u;
+        tmem_st16(pcol + half * 16, packed);
       }
-      // P row -> shared memory, K-major 128-byte-swizzled (16-byte chunk ^= row % 8).
-      unsigned char* pdst = prow + (it & 1) * C::kPBytes;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint4 v = make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(pdst + ((ch ^ (row & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
+      l += sum;
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[it & 1]);
     }
@@ -320,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long tok = bh * prm.S + static_cast<long long>(i0) * 64 + row;
     bool have_o = ok && nit > 0;
     if (have_o) {
-      have_o = __all_sync(0xffffffffu, mbar_wait(o_bar, (nit - 1) & 1, prm.status, kDevTimeoutOBar));
+      have_o = __all_sync(0xffffffffu, mbar_wait(o_final, 0, prm.status, kDevTimeoutOBar));
       tc_fence_after();
     }
     const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
@@ -382,36 +402,37 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over [rows, D] (row stride D*2 bytes), box = 64 columns x box_rows rows,
-// 128-byte swizzle, zero fill out of bounds.
-bool make_map_bf16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows) {
+// 2-D map of 16-bit elements (bf16, or fp16 when `fp16`) over [rows, D] (row stride
+// D*2 bytes), box = 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows,
+                 bool fp16) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
   cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = enc(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 namespace {
-template <int D>
+template <int D, bool VF16>
 cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& d,
                        const FwdParams& prm, cudaStream_t st, bool* map_ok) {
   CUtensorMap mq, mk, mv;
   const long long rows = static_cast<long long>(d.BH) * d.S;
-  *map_ok = make_map_bf16(&mq, q, rows, D, 128) && make_map_bf16(&mk, k, rows, D, 64) &&
-            make_map_bf16(&mv, v, rows, D, 64);
+  *map_ok = make_map_16(&mq, q, rows, D, 128, false) && make_map_16(&mk, k, rows, D, 64, false) &&
+            make_map_16(&mv, v, rows, D, 64, VF16);
   if (!*map_ok) return cudaErrorInvalidValue;
   using C = FwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, VF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((d.nb + 1) / 2, d.BH);
-  attn_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, prm);
+  const unsigned items = static_cast<unsigned>(d.BH) * static_cast<unsigned>((d.nb + 1) / 2);
+  attn_fwd_kernel<D, VF16><<<items, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 }  // namespace
@@ -423,11 +444,11 @@ using namespace nabla;
 extern "C" size_t nabla_fwd_workspace_bytes(nabla_shape s) {
   Dims d;
   if (check_shape(s, &d) != NABLA_OK) return 0;
-  return kStatusBytes;
+  return kStatusBytes + schedule_scratch_bytes(d);
 }
 
 extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void* v,
-                                       const int32_t* row_idx, const int32_t* row_cnt,
+                                       nabla_dtype v_dtype, const int32_t* row_idx, const int32_t* row_cnt,
                                        nabla_shape s, float scale, void* o, nabla_dtype o_dtype,
                                        float* lse, void* workspace, size_t workspace_bytes,
                                        nabla_stream_t stream) {
@@ -440,6 +461,7 @@ extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void*
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
     return NABLA_ERR_INVALID_ARG;
   if (o_dtype != NABLA_BF16 && o_dtype != NABLA_F32) return NABLA_ERR_INVALID_ARG;
+  if (v_dtype != NABLA_BF16 && v_dtype != NABLA_F16) return NABLA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < nabla_fwd_workspace_bytes(s) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -458,8 +480,16 @@ extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void*
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t ce = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
   if (ce != cudaSuccess) return cuda_status(ce);
+  int32_t* order = nullptr;
+  ce = build_schedule(row_cnt, d, static_cast<char*>(workspace) + kStatusBytes, &order, st);
+  if (ce != cudaSuccess) return cuda_status(ce);
+  prm.order = order;
+  prm.npairs = (d.nb + 1) / 2;
   bool map_ok = true;
-  cudaError_t e = d.D == 64 ? launch_fwd<64>(q, k, v, d, prm, st, &map_ok)
-                            : launch_fwd<128>(q, k, v, d, prm, st, &map_ok);
+  const bool vf16 = v_dtype == NABLA_F16;
+  cudaError_t e = d.D == 64 ? (vf16 ? launch_fwd<64, true>(q, k, v, d, prm, st, &map_ok)
+                                    : launch_fwd<64, false>(q, k, v, d, prm, st, &map_ok))
+                            : (vf16 ? launch_fwd<128, true>(q, k, v, d, prm, st, &map_ok)
+                                    : launch_fwd<128, false>(q, k, v, d, prm, st, &map_ok));
   return cuda_status(e);
 }

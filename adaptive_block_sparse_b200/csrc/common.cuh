@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -30,6 +31,11 @@ nabla_status check_shape(const nabla_shape& s, Dims* d);
 bool aligned16(const void* p);
 nabla_status cuda_status(cudaError_t e);
 
+// Longest-first tile order (schedule.cu): scratch size and builder.
+size_t schedule_scratch_bytes(const Dims& d);
+cudaError_t build_schedule(const int32_t* cnt, const Dims& d, void* scratch, int32_t** order_out,
+                           cudaStream_t st);
+
 // Device status codes (recorded in workspace word 0; first error wins).
 enum : uint32_t {
   kDevOk = 0,
@@ -41,6 +47,7 @@ enum : uint32_t {
   kDevTimeoutQFull = 0x106,
   kDevTimeoutDrain = 0x107,
   kDevTimeoutBwd = 0x108,
+  kDevFp16Range = 0x201,   // backward: an input exceeds the fp16 range (|x| > 65504)
 };
 
 #if defined(__CUDACC__)
@@ -200,6 +207,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// D(tmem) (+)= A(tmem) * B(smem desc); A is M x K bf16 in TMEM (lane = row, two K
+// elements per 32-bit column), bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when all previously issued tcgen05 MMAs of this thread are done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -221,6 +240,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
         "=r"(r[31])
       : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -254,6 +283,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// Instruction descriptor of kind::f16 with fp16 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major,
+                                                     bool b_mn_major) {
+  return (1u << 4)                                   // D format: f32 (A, B format 0: f16)
+         | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                       bool b_mn_major) {
@@ -274,10 +311,42 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The two fp16 halves of a packed pair, widened to f32 (exact).
+__device__ __forceinline__ float f16lo(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16hi(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+}
+
+// The two bf16 halves of a packed pair, widened to f32 (exact).
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe (relieves the special-function unit): Cody-Waite style range
+// reduction x = j + f, j = floor(x), f in [0, 1), then a degree-3 minimax polynomial for
+// 2^f (coefficients from a Remez fit of the relative error on [0, 1]; max relative error
+// 7.5e-5, far below the 2^-8 rounding of the bf16 probabilities it feeds), and j added to
+// the exponent field.  Valid for x <= 127; inputs below -126 are clamped (result ~1e-38).
+__device__ __forceinline__ float poly_exp2(float x) {
+  x = fmaxf(x, -126.0f);
+  const float j = floorf(x);
+  const float f = x - j;
+  float p = fmaf(0.07802452147006989f, f, 0.22606715559959412f);
+  p = fmaf(p, f, 0.6958335638046265f);
+  p = fmaf(p, f, 0.9999251961708069f);
+  return __int_as_float(__float_as_int(p) + (static_cast<int>(j) << 23));
 }
 
 #endif  // __CUDACC__

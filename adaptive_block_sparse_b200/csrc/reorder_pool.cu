@@ -19,14 +19,20 @@ namespace {
 
 constexpr int kThreads = 128;
 
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // GATHER: the source is in natural order (forward reorder); otherwise the source block
 // is contiguous (already reordered).  SCATTER: the destination is natural order
-// (inverse reorder).  WRITE: write a destination at all.  POOL: emit fp64 block means.
-template <int D, bool GATHER, bool SCATTER, bool WRITE, bool POOL>
+// (inverse reorder).  WRITE: write a destination at all.  POOL: emit fp64 block means of
+// the (bf16) source.  TO_F16: convert bf16 -> fp16 on the way.  ESZ: element bytes.
+template <int D, int ESZ, bool GATHER, bool SCATTER, bool WRITE, bool POOL, bool TO_F16>
 __global__ void __launch_bounds__(kThreads) reorder_pool_kernel(
     const uint4* __restrict__ src, uint4* __restrict__ dst, double* __restrict__ pool_out,
     int Hg, int W, int Hb, int Wb, int nb) {
-  constexpr int V = D / 8;            // uint4 chunks per token row
+  constexpr int V = D * ESZ / 16;     // uint4 chunks per token row
   constexpr int kChunks = 64 * V;     // per block
   constexpr int kPer = kChunks / kThreads;
   __shared__ __align__(16) uint4 tile[POOL ? kChunks : 1];
@@ -40,7 +46,6 @@ __global__ void __launch_bounds__(kThreads) reorder_pool_kernel(
   const int wb = rem - hb * Wb;
   const long long head_base = bh * S;   // in tokens
 
-  uint4 regs[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
     const int e = threadIdx.x + u * kThreads;
@@ -50,12 +55,19 @@ __global__ void __launch_bounds__(kThreads) reorder_pool_kernel(
         (static_cast<long long>(t) * Hg + hb * 8 + (tt >> 3)) * W + wb * 8 + (tt & 7);
     const long long frac = static_cast<long long>(blk) * 64 + tt;
     const long long s_tok = GATHER ? nat : frac;
-    regs[u] = __ldg(src + (head_base + s_tok) * V + c);
+    const uint4 val = __ldg(src + (head_base + s_tok) * V + c);
     if constexpr (WRITE) {
       const long long d_tok = SCATTER ? nat : frac;
-      dst[(head_base + d_tok) * V + c] = regs[u];
+      uint4 out = val;
+      if constexpr (TO_F16) {
+        out.x = bf16x2_to_f16x2(val.x);
+        out.y = bf16x2_to_f16x2(val.y);
+        out.z = bf16x2_to_f16x2(val.z);
+        out.w = bf16x2_to_f16x2(val.w);
+      }
+      dst[(head_base + d_tok) * V + c] = out;
     }
-    if constexpr (POOL) tile[e] = regs[u];
+    if constexpr (POOL) tile[e] = val;
   }
   if constexpr (POOL) {
     __syncthreads();
@@ -69,58 +81,62 @@ __global__ void __launch_bounds__(kThreads) reorder_pool_kernel(
   }
 }
 
-template <int D>
-cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims& d, int inverse,
-                           cudaStream_t st) {
+template <int D, int ESZ, bool GATHER, bool SCATTER, bool WRITE, bool POOL, bool TO_F16>
+cudaError_t go(const void* src, void* dst, double* pool, const Dims& d, cudaStream_t st) {
   dim3 grid(d.nb, d.BH);
-  const uint4* s = static_cast<const uint4*>(src);
-  uint4* o = static_cast<uint4*>(dst);
-  if (inverse) {
-    reorder_pool_kernel<D, false, true, true, false>
-        <<<grid, kThreads, 0, st>>>(s, o, nullptr, d.Hg, d.W, d.Hb, d.Wb, d.nb);
-  } else if (pool) {
-    reorder_pool_kernel<D, true, false, true, true>
-        <<<grid, kThreads, 0, st>>>(s, o, pool, d.Hg, d.W, d.Hb, d.Wb, d.nb);
-  } else {
-    reorder_pool_kernel<D, true, false, true, false>
-        <<<grid, kThreads, 0, st>>>(s, o, nullptr, d.Hg, d.W, d.Hb, d.Wb, d.nb);
-  }
+  reorder_pool_kernel<D, ESZ, GATHER, SCATTER, WRITE, POOL, TO_F16><<<grid, kThreads, 0, st>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), pool, d.Hg, d.W, d.Hb, d.Wb, d.nb);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_pool_only(const void* x, double* pool, const Dims& d, cudaStream_t st) {
-  dim3 grid(d.nb, d.BH);
-  reorder_pool_kernel<D, false, false, false, true><<<grid, kThreads, 0, st>>>(
-      static_cast<const uint4*>(x), nullptr, pool, d.Hg, d.W, d.Hb, d.Wb, d.nb);
-  return cudaGetLastError();
+cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims& d, int inverse,
+                           int esz, bool to_f16, cudaStream_t st) {
+  if (inverse) {
+    return esz == 4 ? go<D, 4, false, true, true, false, false>(src, dst, nullptr, d, st)
+                    : go<D, 2, false, true, true, false, false>(src, dst, nullptr, d, st);
+  }
+  if (to_f16) {
+    return pool ? go<D, 2, true, false, true, true, true>(src, dst, pool, d, st)
+                : go<D, 2, true, false, true, false, true>(src, dst, nullptr, d, st);
+  }
+  return pool ? go<D, 2, true, false, true, true, false>(src, dst, pool, d, st)
+              : go<D, 2, true, false, true, false, false>(src, dst, nullptr, d, st);
 }
 
 }  // namespace
 
 // Pools a reordered bf16 tensor into fp64 block means (used by the mask build).
 cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st) {
-  return d.D == 64 ? launch_pool_only<64>(x, pool, d, st) : launch_pool_only<128>(x, pool, d, st);
+  return d.D == 64 ? go<64, 2, false, false, false, true, false>(x, nullptr, pool, d, st)
+                   : go<128, 2, false, false, false, true, false>(x, nullptr, pool, d, st);
 }
 
 }  // namespace nabla
 
 using namespace nabla;
 
-extern "C" nabla_status nabla_reorder(const void* src, void* dst, double* pool_out,
-                                      nabla_shape s, int32_t inverse, nabla_stream_t stream) {
+extern "C" nabla_status nabla_reorder(const void* src, nabla_dtype src_dtype, void* dst,
+                                      nabla_dtype dst_dtype, double* pool_out, nabla_shape s,
+                                      int32_t inverse, nabla_stream_t stream) {
   Dims d;
   nabla_status rc = check_shape(s, &d);
   if (rc != NABLA_OK) return rc;
   if (!src || !dst) return NABLA_ERR_INVALID_ARG;
   if (!aligned16(src) || !aligned16(dst)) return NABLA_ERR_INVALID_ARG;
+  const bool dt_ok = inverse ? (src_dtype == dst_dtype &&
+                                (src_dtype == NABLA_BF16 || src_dtype == NABLA_F16 || src_dtype == NABLA_F32))
+                             : (src_dtype == NABLA_BF16 && (dst_dtype == NABLA_BF16 || dst_dtype == NABLA_F16));
+  if (!dt_ok) return NABLA_ERR_INVALID_ARG;
   if (pool_out && (inverse || (reinterpret_cast<uintptr_t>(pool_out) & 7))) return NABLA_ERR_INVALID_ARG;
-  const size_t bytes = static_cast<size_t>(d.BH) * d.S * d.D * 2;
+  const int esz = src_dtype == NABLA_F32 ? 4 : 2;
+  const size_t bytes = static_cast<size_t>(d.BH) * d.S * d.D * esz;
   const char* a = static_cast<const char*>(src);
   const char* b = static_cast<const char*>(dst);
   if (a < b + bytes && b < a + bytes) return NABLA_ERR_INVALID_ARG;   // overlap
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = d.D == 64 ? launch_reorder<64>(src, dst, pool_out, d, inverse, st)
-                            : launch_reorder<128>(src, dst, pool_out, d, inverse, st);
+  const bool to_f16 = !inverse && dst_dtype == NABLA_F16;
+  cudaError_t e = d.D == 64 ? launch_reorder<64>(src, dst, pool_out, d, inverse, esz, to_f16, st)
+                            : launch_reorder<128>(src, dst, pool_out, d, inverse, esz, to_f16, st);
   return cuda_status(e);
 }

@@ -159,7 +159,8 @@ class Path:
         sh = self.shape
         self.thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
         self.q, self.k, self.v = make_qkv(wl, device=dev)          # natural order
-        self.qf, self.kf, self.vf = (torch.empty_like(self.q) for _ in range(3))
+        self.qf, self.kf = (torch.empty_like(self.q) for _ in range(2))
+        self.vf = torch.empty(self.q.shape, dtype=torch.float16, device=dev)   # fp16 V operand
         self.qp = torch.empty(wl.B, wl.H, sh.nb, wl.D, dtype=torch.float64, device=dev)
         self.kp = torch.empty_like(self.qp)
         self.bits, self.ridx, self.rcnt, self.cidx, self.ccnt = m.alloc_mask(
@@ -178,7 +179,14 @@ class Path:
         self.ev = {}
 
     def launches_per_step(self):
-        return 3 + 1 + (1 if self.wl.backward else 0) + 1 + (3 if self.wl.backward else 0)
+        """Kernels of this library launched by one step (memsets not counted).
+
+        reorder x3; mask rows (+ column lists for the backward); forward: 3 schedule
+        kernels + attention; backward: 2 x 3 schedule kernels + preprocess + dK/dV + dQ.
+        """
+        fwd = 3 + 1 + 4
+        bwd = 1 + 9 if self.wl.backward else 0
+        return fwd + bwd
 
     def _mark(self, name, timing):
         if timing:
@@ -333,7 +341,7 @@ def run_reference(args, wl, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="wan720p", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -48,7 +48,7 @@ typedef enum {
   NABLA_ERR_DEVICE_CHECK = 5  /* a kernel recorded a device-side failure (bounded wait) */
 } nabla_status;
 
-typedef enum { NABLA_BF16 = 0, NABLA_F32 = 1 } nabla_dtype;
+typedef enum { NABLA_BF16 = 0, NABLA_F32 = 1, NABLA_F16 = 2 } nabla_dtype;
 
 /* Problem shape.  S = T*Hg*W, N = P*P, nb = S/N.  Hg is the (padded) latent height. */
 typedef struct {
@@ -71,15 +71,20 @@ const char *nabla_status_string(nabla_status s);
  * n = (t*Hg + h)*W + w maps to r = ((t*Hb + h/P)*Wb + w/P)*N + (h%P)*P + (w%P) with
  * Hb = Hg/P, Wb = W/P (row-major patches, row-major inside a patch).
  *
- * inverse == 0: dst[b,h,r,:] = src[b,h,n(r),:] (natural -> reordered).
- * inverse != 0: dst[b,h,n(r),:] = src[b,h,r,:] (reordered -> natural).
- * src, dst: bf16 [B,H,S,D]; must not overlap.
+ * inverse == 0: dst[b,h,r,:] = src[b,h,n(r),:] (natural -> reordered).  src_dtype must be
+ *   NABLA_BF16; dst_dtype NABLA_BF16 (copy) or NABLA_F16 (converted on the way, for the
+ *   V operand of the attention kernels; exact for 2^-14 <= |x| <= 65504, larger
+ *   magnitudes become +-inf).
+ * inverse != 0: dst[b,h,n(r),:] = src[b,h,r,:] (reordered -> natural), src_dtype ==
+ *   dst_dtype in {NABLA_BF16, NABLA_F16, NABLA_F32} (e.g. to restore an output O).
+ * src, dst: [B,H,S,D] of those dtypes; must not overlap.
  * pool_out (nullable, only with inverse == 0): fp64 [B,H,nb,D], the mean of each
  *   block's N reordered token vectors (sum in token order in fp64, then / N), i.e.
  *   the pooled Q or K of [ZH-TS] "downsampling", ready for nabla_build_mask.
  * Errors: INVALID_ARG (nulls, overlap, shape), UNSUPPORTED (D, P), CUDA (launch).
  * --------------------------------------------------------------------------------- */
-nabla_status nabla_reorder(const void *src, void *dst, double *pool_out, nabla_shape s,
+nabla_status nabla_reorder(const void *src, nabla_dtype src_dtype, void *dst,
+                           nabla_dtype dst_dtype, double *pool_out, nabla_shape s,
                            int32_t inverse, nabla_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
@@ -134,14 +139,17 @@ nabla_status nabla_mask_lists(const uint32_t *mask_bits, nabla_shape s, int32_t 
  *   of row i;  LSE_r = ln sum_c exp(scale * Q_r . K_c).
  * A row with no kept block gives O = 0 and LSE = -inf.
  *
- * q, k, v    : bf16 [B,H,S,D] reordered.  row_idx / row_cnt as from nabla_build_mask.
+ * q, k       : bf16 [B,H,S,D] reordered.  row_idx / row_cnt as from nabla_build_mask.
+ * v, v_dtype : [B,H,S,D] reordered, NABLA_BF16 or NABLA_F16.  With fp16 V the
+ *              probabilities P enter the PV product as fp16 (11-bit significand)
+ *              instead of bf16 (8-bit): about 8x smaller output error.
  * o          : out [B,H,S,D], bf16 or f32 per o_dtype.   lse: out f32 [B,H,S] (natural
  *              log; nullable when not needed).
  * workspace  : >= nabla_fwd_workspace_bytes(s) bytes (tile schedule + status word).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  * --------------------------------------------------------------------------------- */
 size_t nabla_fwd_workspace_bytes(nabla_shape s);
-nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v,
+nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v, nabla_dtype v_dtype,
                             const int32_t *row_idx, const int32_t *row_cnt, nabla_shape s,
                             float scale, void *o, nabla_dtype o_dtype, float *lse,
                             void *workspace, size_t workspace_bytes, nabla_stream_t stream);
@@ -152,14 +160,18 @@ nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v,
  * has no gradient, so gradients flow through attention on the kept tiles only:
  *   P = exp(scale*Q K^T - LSE), Dr = rowsum(dO * O), dS = P * (dO V^T - Dr),
  *   dV = P^T dO, dK = scale * dS^T Q, dQ = scale * dS K   (kept tiles only).
- * q, k, v, dout: bf16 [B,H,S,D]; o: forward output (o_dtype); lse: forward LSE.
+ * q, k, dout: bf16 [B,H,S,D]; v: bf16 or fp16 (v_dtype); o: forward output (o_dtype);
+ * lse: forward LSE.  The MMAs run on fp16 copies of Q, K, V and dO made in the
+ * workspace (P and dS rounded to fp16): inputs must satisfy |x| <= 65504, otherwise the
+ * device status word reports it (0x201).
  * row_* and col_* lists from nabla_build_mask / nabla_mask_lists.
  * dq, dk, dv : out f32 [B,H,S,D] (fully overwritten; deterministic, no atomics).
  * workspace  : >= nabla_bwd_workspace_bytes(s) bytes.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  * --------------------------------------------------------------------------------- */
 size_t nabla_bwd_workspace_bytes(nabla_shape s);
-nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, nabla_dtype v_dtype,
+                            const void *o,
                             nabla_dtype o_dtype, const void *dout, const float *lse,
                             const int32_t *row_idx, const int32_t *row_cnt,
                             const int32_t *col_idx, const int32_t *col_cnt, nabla_shape s,

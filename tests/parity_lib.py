@@ -23,9 +23,9 @@ def shape_of(wl):
     return nbl().Shape(wl.B, wl.H, wl.T, wl.Hg, wl.W, wl.D, wl.P)
 
 
-def gpu_reorder(x_nat, shape, pool=False):
+def gpu_reorder(x_nat, shape, pool=False, dtype=torch.bfloat16):
     m = nbl()
-    dst = torch.empty_like(x_nat)
+    dst = torch.empty(x_nat.shape, dtype=dtype, device=x_nat.device)
     pool_out = (torch.empty(shape.B, shape.H, shape.nb, shape.D, dtype=torch.float64,
                             device=x_nat.device) if pool else None)
     m.nabla_reorder(x_nat, dst, shape, pool_out=pool_out)

@@ -59,15 +59,22 @@ def test_host_validation_rejects_bad_arguments(lib):
     good = _shape(nb)
     INV, UNS, WS = nb.NABLA_ERR_INVALID_ARG, nb.NABLA_ERR_UNSUPPORTED, nb.NABLA_ERR_WORKSPACE
     # shapes
-    assert lib.nabla_reorder(A, Bp, None, _shape(nb, Hg=12), 0, st) == INV
-    assert lib.nabla_reorder(A, Bp, None, _shape(nb, D=96), 0, st) == UNS
-    assert lib.nabla_reorder(A, Bp, None, _shape(nb, P=4), 0, st) == UNS
-    assert lib.nabla_reorder(A, Bp, None, _shape(nb, B=0), 0, st) == INV
-    # pointers
-    assert lib.nabla_reorder(None, Bp, None, good, 0, st) == INV
-    assert lib.nabla_reorder(mis, Bp, None, good, 0, st) == INV
-    assert lib.nabla_reorder(A, A, None, good, 0, st) == INV              # overlap
-    assert lib.nabla_reorder(A, Bp, A, good, 1, st) == INV                # pool with inverse
+    BF, F32, F16 = nb.NABLA_BF16, nb.NABLA_F32, nb.NABLA_F16
+
+    def ro(src=A, sd=BF, dst=Bp, dd=BF, pool=None, shape=good, inv=0):
+        return lib.nabla_reorder(src, sd, dst, dd, pool, shape, inv, st)
+    assert ro(shape=_shape(nb, Hg=12)) == INV
+    assert ro(shape=_shape(nb, D=96)) == UNS
+    assert ro(shape=_shape(nb, P=4)) == UNS
+    assert ro(shape=_shape(nb, B=0)) == INV
+    # pointers and dtypes
+    assert ro(src=None) == INV
+    assert ro(src=mis) == INV
+    assert ro(dst=A) == INV                                               # overlap
+    assert ro(pool=A, inv=1) == INV                                       # pool with inverse
+    assert ro(sd=F16) == INV                                              # forward needs bf16 source
+    assert ro(dd=F32) == INV                                              # no f32 forward output
+    assert ro(sd=F32, dd=BF, inv=1) == INV                                # inverse keeps the dtype
     win = nb._Window(0, 0, 0)
     ws_need = lib.nabla_mask_workspace_bytes(good)
     assert ws_need > 256
@@ -88,13 +95,15 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert bm(ws=ctypes.c_void_p(0x20000010)) == WS                       # misaligned workspace
     fws = lib.nabla_fwd_workspace_bytes(good)
 
-    def fwd(q=A, o=Bp, scale=0.125, odt=0, ws=Bp, wsb=fws, ridx=A):
-        return lib.nabla_attn_fwd(q, A, A, ridx, A, good, scale, o, odt, None, ws, wsb, st)
+    def fwd(q=A, o=Bp, scale=0.125, odt=0, ws=Bp, wsb=fws, ridx=A, vdt=0):
+        return lib.nabla_attn_fwd(q, A, A, vdt, ridx, A, good, scale, o, odt, None, ws, wsb, st)
     assert fwd(q=None) == INV
     assert fwd(q=mis) == INV
     assert fwd(ridx=None) == INV
     assert fwd(scale=-1.0) == INV
     assert fwd(odt=7) == INV
+    assert fwd(odt=2) == INV
+    assert fwd(vdt=1) == INV
     assert fwd(wsb=fws - 1) == WS
     assert lib.nabla_fwd_workspace_bytes(_shape(nb, D=96)) == 0
     assert lib.nabla_status_string(3) == b"NABLA_ERR_WORKSPACE"

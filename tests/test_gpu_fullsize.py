@@ -1,0 +1,81 @@
+"""Parity at the benchmark's full sizes, in the launch configuration bench.py times.
+
+Masks: every head against the oracle (bit-exact outside the 1e-6 band).  Forward:
+sampled heads x sampled query blocks, computed row by row by the oracle on the GPU's
+mask.  Backward (training workload): two sampled heads in full.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_lib import bits_to_mask, check_close, check_lists, check_lse, check_mask, to64
+from synth import WORKLOADS
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(name):
+    import bench
+    wl = WORKLOADS[name]
+    path = bench.Path(wl, torch.device("cuda", 0))
+    path.step()
+    torch.cuda.synchronize()
+    path.check_status()
+    return wl, path
+
+
+def _head(t, b, h, wl, reorder=False):
+    x = t[b, h].detach().cpu().double().numpy()
+    return oracle.reorder(x[None, None], wl.T, wl.Hg, wl.W, wl.P)[0, 0] if reorder else x
+
+
+@pytest.mark.parametrize("name", ["wan720p", "wan720p_sta", "train_mid"])
+def test_fullsize_mask_and_forward(name):
+    wl, path = _run(name)
+    thr = path.thr
+    gm = bits_to_mask(path.bits, wl.nb)
+    check_lists(path.ridx, path.rcnt, gm)
+    mism = amb = 0
+    qn, kn = path.q.cpu(), path.k.cpu()
+    for b in range(wl.B):
+        for h in range(wl.H):
+            qf = oracle.reorder(qn[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
+            kf = oracle.reorder(kn[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
+            om, E, _ = oracle.nabla_mask(qf, kf, wl.T, wl.Hg, wl.W, wl.P, thr, wl.window)
+            m1, a1 = check_mask(gm[b, h][None, None], om, E, thr)
+            mism += m1
+            amb += a1
+    print(f"{name}: sparsity {1 - gm.mean():.4f}, near-threshold blocks {amb}, differing {mism}")
+    # forward on sampled heads / query blocks (rows of whole blocks)
+    rng = np.random.default_rng(7)
+    bf16_out = path.o.dtype == torch.bfloat16
+    scale = 1 / math.sqrt(wl.D)
+    heads = [(int(b), int(h)) for b, h in zip(rng.integers(0, wl.B, 4), rng.integers(0, wl.H, 4))]
+    for b, h in heads:
+        q, k = (_head(t, b, h, wl) for t in (path.qf, path.kf))
+        v = _head(path.v, b, h, wl, reorder=True)        # bf16 values (the kernel reads fp16 V)
+        blocks = rng.choice(wl.nb, size=6, replace=False)
+        rows = (blocks[:, None] * wl.N + np.arange(wl.N)[None, :]).reshape(-1)
+        O, L = oracle.block_sparse_attention_rows(q, k, v, gm[b, h], wl.N, scale, rows)
+        got = path.o[b, h, torch.from_numpy(rows).cuda()].detach().cpu().double().numpy()
+        check_close(got, O, f"O {name} head {b},{h}", storage_bf16=bf16_out)
+        lse = path.lse[b, h, torch.from_numpy(rows).cuda()].cpu().double().numpy()
+        check_lse(lse, L)
+
+
+def test_fullsize_backward():
+    wl, path = _run("train_mid")
+    gm = bits_to_mask(path.bits, wl.nb)
+    check_lists(path.cidx, path.ccnt, np.swapaxes(gm, -1, -2))
+    scale = 1 / math.sqrt(wl.D)
+    for b, h in ((0, 3), (1, 17)):
+        q, k, do = (_head(t, b, h, wl) for t in (path.qf, path.kf, path.do))
+        v = _head(path.v, b, h, wl, reorder=True)
+        ref = oracle.block_sparse_attention_bwd(q[None, None], k[None, None], v[None, None],
+                                                do[None, None], gm[b:b + 1, h:h + 1], wl.N, scale)
+        for got, r, what in zip((path.dq, path.dk, path.dv), ref, ("dQ", "dK", "dV")):
+            mx, mean = check_close(to64(got[b, h]), r[0, 0], f"{what} train_mid head {b},{h}")
+            print(f"train_mid {what} head {b},{h}: max err {mx:.2e} mean {mean:.2e}")

@@ -47,6 +47,16 @@ def test_reorder_and_pool_bit_exact(data, name):
     assert torch.equal(back.view(torch.int16), q.view(torch.int16))
     ref_pool = oracle.pool_blocks(oracle.reorder(to64(q), wl.T, wl.Hg, wl.W, wl.P), wl.N)
     assert np.array_equal(pool.cpu().numpy(), ref_pool)
+    # fp16 destination: the same permutation, values converted with round-to-nearest-even
+    q16, _ = gpu_reorder(q, shape, dtype=torch.float16)
+    ref16 = oracle.reorder(q.cpu().to(torch.float16).view(torch.int16).numpy(), wl.T, wl.Hg, wl.W, wl.P)
+    assert np.array_equal(q16.cpu().view(torch.int16).numpy(), ref16)
+    # inverse of a float32 tensor
+    x32 = torch.randn(q.shape, device=DEV)
+    back32 = torch.empty_like(x32)
+    nbl().nabla_reorder(x32, back32, shape, inverse=True)
+    ref32 = oracle.inverse_reorder(x32.cpu().numpy(), wl.T, wl.Hg, wl.W, wl.P)
+    assert np.array_equal(back32.cpu().numpy(), ref32)
 
 
 MASK_CASES = [("tiny", 0.8, (0, 0, 0)), ("small", 0.5, (0, 0, 0)), ("small", 0.8, (0, 0, 0)),
@@ -83,17 +93,20 @@ def test_mask_parity(data, name, thr, window):
     assert torch.equal(bits2, bits)
 
 
-def _fwd_case(data, wl, thr, window, o_dtype):
+def _fwd_case(data, wl, thr, window, o_dtype, v_dtype=torch.float16):
     m = nbl()
     shape = shape_of(wl)
     q, k, v = data(wl)
     qf, _ = gpu_reorder(q, shape)
     kf, _ = gpu_reorder(k, shape)
-    vf, _ = gpu_reorder(v, shape)
+    vf, _ = gpu_reorder(v, shape)                     # bf16 values for the oracle
+    vk, _ = gpu_reorder(v, shape, dtype=v_dtype)      # the kernel's V operand
     bits, ridx, rcnt, _, _ = gpu_mask(qf, kf, shape, thr, window, cols=False)
     lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
-    o, _ = m.nabla_attn_fwd(qf, kf, vf, ridx, rcnt, shape, o_dtype=o_dtype, lse=lse)
+    ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    o, _ = m.nabla_attn_fwd(qf, kf, vk, ridx, rcnt, shape, o_dtype=o_dtype, lse=lse, workspace=ws)
     torch.cuda.synchronize()
+    assert m.nabla_read_device_status(ws) == 0
     gm = bits_to_mask(bits, wl.nb)
     O, L = oracle.block_sparse_attention(to64(qf), to64(kf), to64(vf), gm, wl.N, 1 / math.sqrt(wl.D))
     return o, lse, O, L, gm
@@ -102,12 +115,13 @@ def _fwd_case(data, wl, thr, window, o_dtype):
 @pytest.mark.parametrize("name,thr,window", [("tiny", 0.8, (0, 0, 0)), ("small", 0.8, (0, 0, 0)),
                                              ("small", 0.95, (0, 0, 0)), ("small", 0.5, (1, 3, 3)),
                                              ("odd", 0.8, (0, 0, 0)), ("odd64", 0.6, (0, 0, 0))])
-@pytest.mark.parametrize("o_dtype", ["f32", "bf16"])
-def test_fwd_parity(data, name, thr, window, o_dtype):
+@pytest.mark.parametrize("o_dtype,v_dtype", [("f32", "f16"), ("bf16", "f16"), ("f32", "bf16")])
+def test_fwd_parity(data, name, thr, window, o_dtype, v_dtype):
     m = nbl()
     wl = _wl(name)
     odt = m.NABLA_F32 if o_dtype == "f32" else m.NABLA_BF16
-    o, lse, O, L, gm = _fwd_case(data, wl, thr, window, odt)
+    vdt = torch.float16 if v_dtype == "f16" else torch.bfloat16
+    o, lse, O, L, gm = _fwd_case(data, wl, thr, window, odt, vdt)
     mx, mean = check_close(to64(o), O, f"O {name}", storage_bf16=(o_dtype == "bf16"))
     check_lse(lse.cpu().numpy().astype(np.float64), L)
     print(f"{name} thr={thr}: density {gm.mean():.4f} max|O| {np.abs(O).max():.2f} "
@@ -123,6 +137,7 @@ def test_fwd_dense_and_empty_rows(data):
     qf, _ = gpu_reorder(q, shape)
     kf, _ = gpu_reorder(k, shape)
     vf, _ = gpu_reorder(v, shape)
+    vk, _ = gpu_reorder(v, shape, dtype=torch.float16)
     nb, nw = wl.nb, shape.nw
     rng = np.random.default_rng(5)
     cases = {"dense": np.ones((wl.B, wl.H, nb, nb), dtype=bool),
@@ -135,8 +150,11 @@ def test_fwd_dense_and_empty_rows(data):
         rcnt = torch.empty(wl.B, wl.H, nb, dtype=torch.int32, device=DEV)
         m.nabla_mask_lists(bits, shape, ridx, rcnt)
         lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
-        o, _ = m.nabla_attn_fwd(qf, kf, vf, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse)
+        ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+        o, _ = m.nabla_attn_fwd(qf, kf, vk, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse,
+                                workspace=ws)
         torch.cuda.synchronize()
+        assert m.nabla_read_device_status(ws) == 0
         check_lists(ridx, rcnt, mask)
         O, L = oracle.block_sparse_attention(to64(qf), to64(kf), to64(vf), mask, wl.N,
                                              1 / math.sqrt(wl.D))
@@ -160,12 +178,17 @@ def test_bwd_parity(data, name, thr, window):
     qf, _ = gpu_reorder(q, shape)
     kf, _ = gpu_reorder(k, shape)
     vf, _ = gpu_reorder(v, shape)
+    vk, _ = gpu_reorder(v, shape, dtype=torch.float16)
     bits, ridx, rcnt, cidx, ccnt = gpu_mask(qf, kf, shape, thr, window)
     lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
-    o, _ = m.nabla_attn_fwd(qf, kf, vf, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse)
+    fws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    o, _ = m.nabla_attn_fwd(qf, kf, vk, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse, workspace=fws)
     do = make_dout(wl, device=DEV)
-    dq, dk, dv = m.nabla_attn_bwd(qf, kf, vf, o, do, lse, ridx, rcnt, cidx, ccnt, shape)
+    bws = torch.zeros(m.nabla_bwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    dq, dk, dv = m.nabla_attn_bwd(qf, kf, vk, o, do, lse, ridx, rcnt, cidx, ccnt, shape, workspace=bws)
     torch.cuda.synchronize()
+    assert m.nabla_read_device_status(fws) == 0
+    assert m.nabla_read_device_status(bws) == 0
     gm = bits_to_mask(bits, wl.nb)
     rq, rk, rv = oracle.block_sparse_attention_bwd(to64(qf), to64(kf), to64(vf), to64(do), gm, wl.N,
                                                    1 / math.sqrt(wl.D))
