@@ -40,6 +40,7 @@ EXPORTED = (
     "nabla_status_string", "nabla_reorder", "nabla_mask_workspace_bytes", "nabla_build_mask",
     "nabla_mask_lists", "nabla_fwd_workspace_bytes", "nabla_attn_fwd",
     "nabla_bwd_workspace_bytes", "nabla_attn_bwd", "nabla_read_device_status",
+    "nabla_attn_fwd_noalloc",
 )
 
 
@@ -70,6 +71,8 @@ _sigs = {
                                       _vp, _vp, _vp, _Shape, ctypes.c_float, _vp, _vp, _vp, _vp,
                                       _sz, _vp]),
     "nabla_read_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
+    "nabla_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _Shape,
+                                              ctypes.c_float, _vp, ctypes.c_int, _vp, _vp]),
 }
 
 
@@ -240,6 +243,23 @@ def nabla_attn_bwd(q, k, v, o, dout, lse, row_idx, row_cnt, col_idx, col_cnt, sh
                                _ptr(workspace), workspace.numel(), _stream(stream)),
            "nabla_attn_bwd")
     return dq, dk, dv
+
+
+def nabla_attn_fwd_noalloc(q, k, v, row_idx, row_cnt, shape: Shape, o, lse=None, scale=None,
+                           stream=None):
+    """Forward without a caller workspace, for callers that cannot allocate device memory.
+
+    Same results as :func:`nabla_attn_fwd`; the workspace is a fixed 1 MiB array inside
+    the library (looked up on the first call on a device, so make that call before any
+    stream capture).  ``o`` (and ``lse``) must be given: this path allocates nothing.
+    Calls that may overlap on the GPU share that array and must be serialised.
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(shape.D)
+    _check(load_library().nabla_attn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(row_idx), _ptr(row_cnt), shape.c(),
+        float(scale), _ptr(o), dtype_code(o), _ptr(lse), _stream(stream)), "nabla_attn_fwd_noalloc")
+    return o, lse
 
 
 def nabla_read_device_status(workspace, stream=None) -> int:

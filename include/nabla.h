@@ -178,6 +178,29 @@ nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, nabla_d
                             float scale, float *dq, float *dk, float *dv, void *workspace,
                             size_t workspace_bytes, nabla_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Allocation-free forward (no counterpart in the NABLA pages; a library convenience).
+ * For callers that cannot call cudaMalloc where they run attention -- e.g. a host
+ * framework that owns all device memory through its own pool and forbids driver
+ * allocations on its hot path, or a latency-critical loop that must not pay for an
+ * allocation -- and so cannot provide nabla_attn_fwd's workspace.  Same arguments and
+ * results as nabla_attn_fwd without the workspace: the workspace is a fixed 1 MiB
+ * array in the library's own device memory (every GPU that loads the library holds it
+ * until the process exits).  Problems whose workspace (nabla_fwd_workspace_bytes)
+ * exceeds 1 MiB are rejected with NABLA_ERR_UNSUPPORTED before anything is enqueued
+ * (the 720p-like 40-head problem needs about 210 KB).  The first call on a device looks
+ * up that array's device address (cudaGetSymbolAddress, with the device current); make
+ * that first call before any stream capture.  The call allocates nothing.  All calls
+ * share the one array, which keeps the last call's contents (each call clears what
+ * must start at zero): calls that can overlap on the GPU (different streams, or several
+ * host threads on one device) race on it and must be serialised by the caller.  The
+ * device status word of the last call is not readable through this entry point.
+ * --------------------------------------------------------------------------------- */
+nabla_status nabla_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                    nabla_dtype v_dtype, const int32_t *row_idx,
+                                    const int32_t *row_cnt, nabla_shape s, float scale, void *o,
+                                    nabla_dtype o_dtype, float *lse, nabla_stream_t stream);
+
 /* Reads (synchronously on `stream`) the device status word that the kernels of the
  * last call on `workspace` recorded: 0 = fine, otherwise a code naming the barrier
  * wait that gave up.  Returns NABLA_ERR_DEVICE_CHECK when the word is non-zero, and
