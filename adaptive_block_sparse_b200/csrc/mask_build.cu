@@ -26,6 +26,12 @@
 namespace nabla {
 
 cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st);
+size_t mask_fast_scratch_bytes(const Dims& d);
+bool mask_fast_supported(const Dims& d);
+cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, double scale, double thr,
+                          const nabla_window& w, uint32_t* bits, int32_t* ridx, int32_t* rcnt,
+                          void* scratch, uint32_t* status, int32_t** rescue_list,
+                          int32_t** rescue_cnt, cudaStream_t st);
 
 namespace {
 
@@ -34,6 +40,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int KC = 32;          // pooled key rows per shared-memory chunk
 constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
 constexpr double kFix = 4611686018427387904.0;  // 2^62
+constexpr int kRescueCtasPerHead = 16;
 
 __device__ __forceinline__ unsigned long long to_fix(double p) { return __double2ull_rn(p * kFix); }
 
@@ -41,8 +48,12 @@ template <int D>
 __global__ void __launch_bounds__(kThreads) mask_rows_kernel(
     const double* __restrict__ qpool, const double* __restrict__ kpool, int nb, int nw, int R,
     double scale, double thr, int sta_on, int wt2, int wh2, int ww2, int Hb, int Wb,
-    uint32_t* __restrict__ bits, int32_t* __restrict__ row_idx, int32_t* __restrict__ row_cnt) {
+    uint32_t* __restrict__ bits, int32_t* __restrict__ row_idx, int32_t* __restrict__ row_cnt,
+    const int32_t* __restrict__ rlist, const int32_t* __restrict__ rlist_cnt) {
+  // Rows: R consecutive rows from blockIdx.x * R, or (rlist != nullptr) the head's listed
+  // rows rlist[bh*nb + ...], taken R at a time by the CTAs of the head in turn.
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ int rows_s[8];
   unsigned long long* hmass = reinterpret_cast<unsigned long long*>(smem_raw);  // 8 x 256
   uint32_t* hcnt = reinterpret_cast<uint32_t*>(hmass + kWarps * 256);           // 8 x 256
   double* qs = reinterpret_cast<double*>(hcnt + kWarps * 256);                  // R x D
@@ -53,12 +64,26 @@ __global__ void __launch_bounds__(kThreads) mask_rows_kernel(
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const long long bh = blockIdx.y;
-  const int i0 = blockIdx.x * R;
-  const int nrows = min(R, nb - i0);
+  const int listed = rlist != nullptr ? min(max(rlist_cnt[bh], 0), nb) : 0;
+  for (int g = rlist != nullptr ? blockIdx.x : 0;; g += gridDim.x) {
+  int nrows;
+  if (rlist != nullptr) {
+    if (g * R >= listed) break;
+    nrows = min(R, listed - g * R);
+  } else {
+    if (g > 0) break;
+    nrows = min(R, nb - static_cast<int>(blockIdx.x) * R);
+  }
+  __syncthreads();
+  if (tid < R)
+    rows_s[tid] = tid < nrows ? (rlist != nullptr ? rlist[bh * nb + g * R + tid]
+                                                  : static_cast<int>(blockIdx.x) * R + tid)
+                              : 0;
+  __syncthreads();
 
   for (int e = tid; e < R * D; e += kThreads) {
     const int r = e / D;
-    qs[e] = (r < nrows) ? qpool[(bh * nb + i0 + r) * D + (e - r * D)] : 0.0;
+    qs[e] = (r < nrows) ? qpool[(bh * nb + rows_s[r]) * D + (e - r * D)] : 0.0;
   }
   // ---- pooled logits A = Qp Kp^T * scale (fp64) --------------------------------------
   for (int j0 = 0; j0 < nb; j0 += KC) {
@@ -93,7 +118,7 @@ __global__ void __launch_bounds__(kThreads) mask_rows_kernel(
 
   for (int r = warp; r < nrows; r += kWarps) {
     double* row = prow + r * nb;
-    const int i = i0 + r;
+    const int i = rows_s[r];
     // ---- row softmax (fp64) -------------------------------------------------------------
     double m = -INFINITY;
     for (int j = lane; j < nb; j += 32) m = fmax(m, row[j]);
@@ -223,6 +248,7 @@ __global__ void __launch_bounds__(kThreads) mask_rows_kernel(
     if (row_cnt != nullptr && lane == 0) row_cnt[bh * nb + i] = run;
     __syncwarp();
   }
+  }  // row groups
 }
 
 // Column lists (transpose of the bitmask): one warp per 32-column word of one head.
@@ -294,7 +320,8 @@ size_t mask_rows_smem(int nb, int D, int R) {
 template <int D>
 cudaError_t launch_mask_rows(const double* qp, const double* kp, const Dims& d, double scale,
                              double thr, const nabla_window& w, uint32_t* bits, int32_t* ridx,
-                             int32_t* rcnt, cudaStream_t st) {
+                             int32_t* rcnt, const int32_t* rlist, const int32_t* rlist_cnt,
+                             cudaStream_t st) {
   const int R = rows_per_cta(d.nb);
   const size_t smem = mask_rows_smem(d.nb, D, R);
   cudaError_t e = cudaFuncSetAttribute(mask_rows_kernel<D>,
@@ -302,10 +329,11 @@ cudaError_t launch_mask_rows(const double* qp, const double* kp, const Dims& d, 
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int sta_on = (w.t | w.h | w.w) != 0;
-  dim3 grid((d.nb + R - 1) / R, d.BH);
+  // Listed rows: a few CTAs per head take the head's rows R at a time.
+  dim3 grid(rlist != nullptr ? kRescueCtasPerHead : (d.nb + R - 1) / R, d.BH);
   mask_rows_kernel<D><<<grid, kThreads, smem, st>>>(qp, kp, d.nb, d.nw, R, scale, thr, sta_on,
                                                    w.t / 2, w.h / 2, w.w / 2, d.Hb, d.Wb, bits,
-                                                   ridx, rcnt);
+                                                   ridx, rcnt, rlist, rlist_cnt);
   return cudaGetLastError();
 }
 
@@ -332,7 +360,7 @@ extern "C" size_t nabla_mask_workspace_bytes(nabla_shape s) {
   Dims d;
   if (check_shape(s, &d) != NABLA_OK) return 0;
   const size_t pool = align_up(static_cast<size_t>(d.BH) * d.nb * d.D * sizeof(double), 256);
-  return kStatusBytes + 2 * pool;
+  return kStatusBytes + 2 * pool + (mask_fast_supported(d) ? mask_fast_scratch_bytes(d) : 0);
 }
 
 extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const double* q_pool,
@@ -365,6 +393,7 @@ extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const dou
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t pool_bytes = align_up(static_cast<size_t>(d.BH) * d.nb * d.D * sizeof(double), 256);
+  if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return NABLA_ERR_CUDA;
   double* qp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes);
   double* kp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes + pool_bytes);
   cudaError_t e = cudaSuccess;
@@ -378,8 +407,24 @@ extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const dou
     if ((e = pool_blocks_device(k, kp_ws, d, st)) != cudaSuccess) return cuda_status(e);
     kp = kp_ws;
   }
-  e = d.D == 64 ? launch_mask_rows<64>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt, st)
-                : launch_mask_rows<128>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt, st);
+  // Fast tier (tensor-core logits, certified fp32 cut) for every row, then the fp64
+  // kernel for the rows it could not certify.  Without the fast tier: fp64 for all rows.
+  const int32_t* rlist = nullptr;
+  const int32_t* rlist_cnt = nullptr;
+  if (mask_fast_supported(d)) {
+    int32_t* rl = nullptr;
+    int32_t* rc = nullptr;
+    e = mask_fast_run(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt,
+                      static_cast<char*>(workspace) + kStatusBytes + 2 * pool_bytes,
+                      static_cast<uint32_t*>(workspace), &rl, &rc, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    rlist = rl;
+    rlist_cnt = rc;
+  }
+  e = d.D == 64 ? launch_mask_rows<64>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt,
+                                       rlist, rlist_cnt, st)
+                : launch_mask_rows<128>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt,
+                                        rlist, rlist_cnt, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (col_idx) {
     if ((e = launch_col_lists(mask_bits, d, col_idx, col_cnt, st)) != cudaSuccess) return cuda_status(e);
