@@ -64,14 +64,14 @@ _sigs = {
                                         ctypes.c_double, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "nabla_mask_lists": (ctypes.c_int, [_vp, _Shape, _vp, _vp, _vp, _vp, _vp]),
     "nabla_fwd_workspace_bytes": (_sz, [_Shape]),
-    "nabla_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _Shape, ctypes.c_float,
+    "nabla_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape, ctypes.c_float,
                                       _vp, ctypes.c_int, _vp, _vp, _sz, _vp]),
     "nabla_bwd_workspace_bytes": (_sz, [_Shape]),
     "nabla_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp,
                                       _vp, _vp, _vp, _Shape, ctypes.c_float, _vp, _vp, _vp, _vp,
                                       _sz, _vp]),
     "nabla_read_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
-    "nabla_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _vp, _Shape,
+    "nabla_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape,
                                               ctypes.c_float, _vp, ctypes.c_int, _vp, _vp]),
 }
 
@@ -208,7 +208,7 @@ def nabla_mask_lists(mask_bits, shape: Shape, row_idx=None, row_cnt=None, col_id
     return row_idx, row_cnt, col_idx, col_cnt
 
 
-def nabla_attn_fwd(q, k, v, row_idx, row_cnt, shape: Shape, scale=None, o=None,
+def nabla_attn_fwd(q, k, v, mask_bits, shape: Shape, scale=None, o=None,
                    o_dtype=NABLA_BF16, lse=None, workspace=None, stream=None):
     """Block-sparse attention forward.  Returns (o, lse)."""
     if scale is None:
@@ -218,8 +218,8 @@ def nabla_attn_fwd(q, k, v, row_idx, row_cnt, shape: Shape, scale=None, o=None,
                         device=q.device)
     if workspace is None:
         workspace = torch.zeros(nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=q.device)
-    _check(load_library().nabla_attn_fwd(_ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(row_idx),
-                               _ptr(row_cnt), shape.c(),
+    _check(load_library().nabla_attn_fwd(_ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(mask_bits),
+                               shape.c(),
                                float(scale), _ptr(o), int(o_dtype), _ptr(lse), _ptr(workspace),
                                workspace.numel(), _stream(stream)), "nabla_attn_fwd")
     return o, lse
@@ -245,7 +245,7 @@ def nabla_attn_bwd(q, k, v, o, dout, lse, row_idx, row_cnt, col_idx, col_cnt, sh
     return dq, dk, dv
 
 
-def nabla_attn_fwd_noalloc(q, k, v, row_idx, row_cnt, shape: Shape, o, lse=None, scale=None,
+def nabla_attn_fwd_noalloc(q, k, v, mask_bits, shape: Shape, o, lse=None, scale=None,
                            stream=None):
     """Forward without a caller workspace, for callers that cannot allocate device memory.
 
@@ -257,7 +257,7 @@ def nabla_attn_fwd_noalloc(q, k, v, row_idx, row_cnt, shape: Shape, o, lse=None,
     if scale is None:
         scale = 1.0 / math.sqrt(shape.D)
     _check(load_library().nabla_attn_fwd_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(row_idx), _ptr(row_cnt), shape.c(),
+        _ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(mask_bits), shape.c(),
         float(scale), _ptr(o), dtype_code(o), _ptr(lse), _stream(stream)), "nabla_attn_fwd_noalloc")
     return o, lse
 

@@ -721,8 +721,8 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   uint32_t* status = static_cast<uint32_t*>(ws);
   int32_t* order_cols = nullptr;
   int32_t* order_rows = nullptr;
-  cudaError_t e = build_schedule(ccnt, d, sched, &order_cols, st);
-  if (e == cudaSuccess) e = build_schedule(rcnt, d, sched + schedule_scratch_bytes(d), &order_rows, st);
+  cudaError_t e = build_schedule(ccnt, nullptr, d, sched, &order_cols, st);
+  if (e == cudaSuccess) e = build_schedule(rcnt, nullptr, d, sched + schedule_scratch_bytes(d), &order_rows, st);
   if (e != cudaSuccess) return e;
   bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
       o, o_f32, static_cast<const __nv_bfloat16*>(dout), lse, static_cast<const __nv_bfloat16*>(q),

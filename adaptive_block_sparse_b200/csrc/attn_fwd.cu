@@ -5,19 +5,25 @@
 // block mask is one full N x N tile of the token attention matrix, computed exactly;
 // the pages run this through FlexAttention.  Here it is a hand-written kernel:
 //
-//  * one CTA = one tile of 128 query rows = two consecutive query blocks (2p, 2p+1) of
-//    one head, so the tensor core runs M = 128 MMAs; the CTA walks the ascending union
-//    of the two blocks' kept-key lists and masks (-inf) the half of the rows whose block
-//    does not keep the current key block;
-//  * warp 0 (one lane) streams K and V tiles with TMA (128-byte swizzle) into a ring of
-//    shared-memory stages; warp 1 (one lane) issues tcgen05.mma: S = Q K^T into one of two
-//    TMEM score buffers, and O += P V into a TMEM accumulator; warps 4-7 run the online
-//    softmax, one query row per thread (TMEM lane = row), write P (bf16) into shared
-//    memory for the second MMA, and rescale O only when a row maximum grows by more
-//    than 2^8 (conditional rescaling);
-//  * the epilogue divides by the row sum and writes O (bf16 or f32) and the natural-log
-//    LSE.  Every barrier wait is bounded; a timeout records a status code and the CTA
-//    drains its own copies / MMAs and frees TMEM before returning.
+//  * work tile = 128 query rows = two consecutive query blocks (2p, 2p+1) of one head
+//    (M = 128 MMAs).  The tile walks the ascending union of the two blocks' kept key
+//    blocks, read from the mask bitmask, two key blocks per step (N = 128 keys per
+//    MMA); a half of the rows whose block does not keep a key block is masked (-inf);
+//  * persistent: one CTA per SM takes tiles in a head-major, longest-first order through
+//    an atomic counter; Q is double-buffered so the next tile's Q and first K/V tiles
+//    load while the current tile finishes;
+//  * warp 0 streams K and V with TMA (128-byte swizzle) through a ring of stages of two
+//    key blocks each; warp 1 (one lane) issues tcgen05.mma: S = Q K^T (128 x 128) into
+//    one of two TMEM score buffers, one step of look-ahead, and O += P V with P read
+//    from TMEM;
+//  * two softmax warpgroups (warps 4-7, 8-11) take alternate steps of the same tile, each
+//    with its own score buffer, running max / sum and TMEM accumulator, one query row per
+//    thread (TMEM lane = row).  Exponentials run on the MUFU unit with a quarter on the
+//    FMA pipe (polynomial); P is rounded to the V operand's 16-bit type and the row sum
+//    takes the rounded weights; O is rescaled only when a row maximum grows by more than
+//    2^8.  The epilogue merges the two partial results (m, l, O);
+//  * every barrier wait is bounded; on a timeout a kernel records a status code, stops,
+//    drains its own copies and MMAs and frees TMEM.
 #include <math.h>
 
 #include <cudaTypedefs.h>
@@ -27,84 +33,115 @@
 namespace nabla {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kSoftmaxWarp0 = 4;          // warps 4..7
-constexpr uint32_t kEnd = 0xFFFFFFFFu;    // end-of-list marker in the stage metadata
+constexpr int kThreads = 384;             // 12 warps
+constexpr int kSoftmaxWarp0 = 4;          // warps 4..7 = group 0, 8..11 = group 1
+constexpr int kMaxWords = 512;            // bitmask words per row (nb <= 16384)
 
 template <int D>
 struct FwdCfg {
   static constexpr int kPanels = D / 64;                  // 128-byte swizzle panels
-  static constexpr int kStages = (D == 128) ? 2 : 4;   // two CTAs per SM
-  static constexpr int kQBytes = 128 * D * 2;
-  static constexpr int kKVTileBytes = 64 * D * 2;         // one K or one V tile
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKVTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kKVTileBytes;
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
-  static constexpr uint32_t kTmemCols = 256;              // S0 | S1 | O
-  static constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;
+  static constexpr int kQBytes = 128 * D * 2;             // 128 rows
+  static constexpr int kPairBytes = 128 * D * 2;          // two K (or V) blocks, 128 rows
+  static constexpr int kStageBytes = 2 * kPairBytes;      // K pair + V pair
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kOffQ = 0;                         // two Q buffers
+  static constexpr int kOffStage = kOffQ + 2 * kQBytes;
+  static constexpr int kOffWords = kOffStage + kStages * kStageBytes;   // [2 tiles][2 rows][kMaxWords]
+  static constexpr int kOffML = kOffWords + 2 * 2 * kMaxWords * 4;     // m, l: [2 tiles][2 groups][128]
+  static constexpr int kOffBar = kOffML + 2 * 2 * 2 * 128 * 4;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
 };
 
 struct FwdParams {
-  const int32_t* order;      // work items (head * npairs + pair), longest first
+  const int32_t* order;      // work items (head * npairs + pair)
+  int items;
   int npairs;
-  const int32_t* row_idx;
-  const int32_t* row_cnt;
+  const uint32_t* bits;      // [B*H, nb, nw]
+  int nw;
   void* o;
   float* lse;
-  uint32_t* status;
+  uint32_t* status;          // word 0: status, word 1: work counter
   int nb;
   long long S;
   float scale_log2;
   int o_f32;
 };
 
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Walks the set bits of w0 | w1 (two rows' bitmask words in shared memory) in ascending
+// order; f = bit0: kept by the first row, bit1: kept by the second.
+struct BitWalk {
+  const uint32_t* w0;
+  const uint32_t* w1;
+  int nw, w;
+  uint32_t cur;
+  __device__ void init(const uint32_t* a, const uint32_t* b, int n) {
+    w0 = a; w1 = b; nw = n; w = 0; cur = n > 0 ? (a[0] | b[0]) : 0u;
+  }
+  __device__ int next(uint32_t* f) {
+    while (cur == 0u) {
+      if (++w >= nw) return -1;
+      cur = w0[w] | w1[w];
+    }
+    const int bit = __ffs(cur) - 1;
+    cur &= cur - 1u;
+    *f = ((w0[w] >> bit) & 1u) | (((w1[w] >> bit) & 1u) << 1);
+    return 32 * w + bit;
+  }
+};
+
 template <int D, bool VF16>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const FwdParams prm) {
   using C = FwdCfg<D>;
+  constexpr int NST = C::kStages;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sQ = smem + C::kOffQ;
-  unsigned char* sK = smem + C::kOffK;
-  unsigned char* sV = smem + C::kOffV;
+  unsigned char* sStage = smem + C::kOffStage;
+  uint32_t* sWords = reinterpret_cast<uint32_t*>(smem + C::kOffWords);
+  float* ml = reinterpret_cast<float*>(smem + C::kOffML);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* full = bars;                       // [kStages]
-  uint64_t* empty = bars + C::kStages;         // [kStages]
-  uint64_t* q_full = bars + 2 * C::kStages;
-  uint64_t* s_full = q_full + 1;               // [2]
-  uint64_t* p_full = s_full + 2;               // [2]
-  uint64_t* o_bar = p_full + 2;                // one phase per PV (rescale waits)
-  uint64_t* o_final = o_bar + 1;               // single phase: every PV has landed
-  uint64_t* drain = o_final + 1;
-  uint32_t* meta = reinterpret_cast<uint32_t*>(drain + 1);   // [kStages]
-  uint32_t* tmem_slot = meta + C::kStages;
+  uint64_t* full = bars;                 // [NST]
+  uint64_t* empty = full + NST;          // [NST]
+  uint64_t* q_full = empty + NST;        // [2]
+  uint64_t* q_empty = q_full + 2;        // [2]
+  uint64_t* s_full = q_empty + 2;        // [2]
+  uint64_t* p_full = s_full + 2;         // [2]
+  uint64_t* tile_done = p_full + 2;
+  uint64_t* o_free = tile_done + 1;
+  uint64_t* drain = o_free + 1;
+  uint32_t* meta = reinterpret_cast<uint32_t*>(drain + 1);   // [NST]
+  int32_t* qmeta = reinterpret_cast<int32_t*>(meta + NST);   // [2][2]: item, blocks
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qmeta + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int item = prm.order[blockIdx.x];
-  const long long bh = item / prm.npairs;
-  const int pair = item - static_cast<int>(bh) * prm.npairs;
   const int nb = prm.nb;
-  const int i0 = 2 * pair;
-  const bool has_i1 = (i0 + 1) < nb;
+  const int nw = prm.nw;
+  uint32_t* status = prm.status;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(&p_full[0], 128);
-    mbar_init(&p_full[1], 128);
-    mbar_init(o_bar, 1);
-    mbar_init(o_final, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+    }
+    mbar_init(tile_done, 1);
+    mbar_init(o_free, 256);
     mbar_init(drain, 1);
     fence_mbarrier_init();
   }
@@ -123,257 +160,337 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_prefetch_desc(&map_q);
       tma_prefetch_desc(&map_k);
       tma_prefetch_desc(&map_v);
-      const int qrow = static_cast<int>(bh * prm.S + static_cast<long long>(i0) * 64);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
-#pragma unroll
-      for (int pn = 0; pn < C::kPanels; ++pn)
-        tma_load_2d(sQ + pn * (128 * 128), &map_q, q_full, pn * 64, qrow);
-      const int32_t* l0 = prm.row_idx + (bh * nb + i0) * static_cast<long long>(nb);
-      const int32_t* l1 = l0 + nb;
-      const int c0 = min(max(prm.row_cnt[bh * nb + i0], 0), nb);
-      const int c1 = has_i1 ? min(max(prm.row_cnt[bh * nb + i0 + 1], 0), nb) : 0;
-      int a = 0, b = 0, it = 0;
-      bool ok = true, ended = false;
-      while (true) {
-        int j = -1;
-        uint32_t f = 0;
-        if (a < c0 && b < c1) {
-          const int ja = l0[a], jb = l1[b];
-          if (ja < jb) { j = ja; f = 1; ++a; }
-          else if (jb < ja) { j = jb; f = 2; ++b; }
-          else { j = ja; f = 3; ++a; ++b; }
-        } else if (a < c0) { j = l0[a++]; f = 1; }
-        else if (b < c1) { j = l1[b++]; f = 2; }
-        const int s = it % C::kStages;
-        const int n = it / C::kStages;
-        if (n > 0 && !mbar_wait(&empty[s], (n - 1) & 1, prm.status, kDevTimeoutKvEmpty)) { ok = false; break; }
-        if (j < 0) {
-          meta[s] = kEnd;
-          mbar_arrive(&full[s]);
-          ended = true;
-          break;
-        }
-        meta[s] = static_cast<uint32_t>(j) | (f << 28);
-        mbar_arrive_expect_tx(&full[s], 2 * C::kKVTileBytes);
-        const int krow = static_cast<int>(bh * prm.S + static_cast<long long>(j) * 64);
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_2d(sK + s * C::kKVTileBytes + pn * 8192, &map_k, &full[s], pn * 64, krow);
-          tma_load_2d(sV + s * C::kKVTileBytes + pn * 8192, &map_v, &full[s], pn * 64, krow);
-        }
-        ++it;
+    }
+    long long g = 0;   // global stage counter
+    for (int tc = 0;; ++tc) {
+      const int qb = tc & 1;
+      int slot = 0;
+      bool ok = true;
+      if (lane == 0) {
+        if (tc >= 2) ok = mbar_wait(&q_empty[qb], ((tc - 2) >> 1) & 1, status, kDevTimeoutQFull);
+        slot = ok ? atomicAdd(status + 1, 1) : prm.items;
       }
-      // Drain: every issued copy must have landed before the CTA may exit.
-      (void)ok;
-      // Copies still in flight: the last kStages iterations, except that placing the end
-      // marker waited for the oldest of them to be consumed (its stage was reused), and a
-      // parity wait on that stage would now look two phases back.
-      const int keep = ended ? C::kStages - 1 : C::kStages;
-      const int first = it > keep ? it - keep : 0;
-      for (int x = first; x < it; ++x)
-        mbar_wait(&full[x % C::kStages], (x / C::kStages) & 1, prm.status, kDevTimeoutDrain);
-      mbar_wait(q_full, 0, prm.status, kDevTimeoutDrain);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      if (!ok) break;
+      if (slot >= prm.items) {
+        if (lane == 0) {
+          qmeta[2 * qb] = -1;
+          qmeta[2 * qb + 1] = 0;
+          mbar_arrive(&q_full[qb]);
+        }
+        break;
+      }
+      const int item = prm.order[slot];
+      const long long bh = item / prm.npairs;
+      const int i0 = 2 * (item - static_cast<int>(bh) * prm.npairs);
+      const bool has_i1 = i0 + 1 < nb;
+      // The two rows' bitmask words -> shared memory; count the union.
+      uint32_t* u0 = sWords + (qb * 2) * kMaxWords;
+      uint32_t* u1 = u0 + kMaxWords;
+      const uint32_t* r0 = prm.bits + (bh * nb + i0) * static_cast<long long>(nw);
+      int cnt = 0;
+      for (int w = lane; w < nw; w += 32) {
+        uint32_t a = r0[w];
+        uint32_t b = has_i1 ? r0[nw + w] : 0u;
+        if (w == nw - 1 && (nb & 31)) {
+          a &= (1u << (nb & 31)) - 1u;
+          b &= (1u << (nb & 31)) - 1u;
+        }
+        u0[w] = a;
+        u1[w] = b;
+        cnt += __popc(a | b);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      __syncwarp();
+      if (lane == 0) {
+        const int steps = (cnt + 1) >> 1;
+        qmeta[2 * qb] = item;
+        qmeta[2 * qb + 1] = steps;
+        mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+        const int qrow = static_cast<int>(bh * prm.S + static_cast<long long>(i0) * 64);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_2d(sQ + qb * C::kQBytes + pn * 16384, &map_q, &q_full[qb], pn * 64, qrow);
+        BitWalk wk;
+        wk.init(u0, u1, nw);
+        for (int k = 0; k < steps; ++k, ++g) {
+          uint32_t fa = 0, fb = 0;
+          const int ja = wk.next(&fa);
+          int jb = wk.next(&fb);
+          if (jb < 0) { jb = ja; fb = 0; }          // odd tail: a masked duplicate
+          const int s = static_cast<int>(g % NST);
+          const long long r = g / NST;
+          if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, status, kDevTimeoutKvEmpty)) { ok = false; break; }
+          meta[s] = static_cast<uint32_t>(ja) | (fa << 14) | (static_cast<uint32_t>(jb) << 16) | (fb << 30);
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          unsigned char* kp = sStage + s * C::kStageBytes;
+          unsigned char* vp = kp + C::kPairBytes;
+          const int ra = static_cast<int>(bh * prm.S + static_cast<long long>(ja) * 64);
+          const int rb = static_cast<int>(bh * prm.S + static_cast<long long>(jb) * 64);
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn) {
+            tma_load_2d(kp + pn * 16384, &map_k, &full[s], pn * 64, ra);
+            tma_load_2d(kp + pn * 16384 + 8192, &map_k, &full[s], pn * 64, rb);
+            tma_load_2d(vp + pn * 16384, &map_v, &full[s], pn * 64, ra);
+            tma_load_2d(vp + pn * 16384 + 8192, &map_v, &full[s], pn * 64, rb);
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      g = __shfl_sync(0xffffffffu, g, 0);
+      if (!ok) break;
+    }
+    if (lane == 0) {
+      // Drain: copies still in flight must land before the CTA exits.
+      for (long long x = g > NST ? g - NST : 0; x < g; ++x)
+        mbar_wait(&full[x % NST], (x / NST) & 1, status, kDevTimeoutDrain);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = VF16 ? idesc_f16_f32(128, D, false, true)
                                         : idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t k_addr = smem_u32(sK);
-      const uint32_t v_addr = smem_u32(sV);
-      auto issue_s = [&](int x) {
-        const int st = x % C::kStages;
-        const uint32_t d_tmem = tmem + ((x & 1) ? C::kColS1 : C::kColS0);
+      const uint32_t st_addr = smem_u32(sStage);
+      long long g = 0;
+      int pcount[2] = {0, 0};
+      bool ok = true;
+      auto issue_s = [&](int qb, long long gs, int b) {
+        const uint32_t kp = st_addr + static_cast<uint32_t>(gs % NST) * C::kStageBytes;
+        const uint32_t d_tmem = tmem + (b ? C::kColS1 : C::kColS0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int pn = kk >> 2, w = kk & 3;
-          const uint64_t ad = sdesc_sw128(q_addr + pn * (128 * 128) + w * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(k_addr + st * C::kKVTileBytes + pn * 8192 + w * 32, 16, 1024);
+          const uint64_t ad = sdesc_sw128(q_addr + qb * C::kQBytes + pn * 16384 + w * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kp + pn * 16384 + w * 32, 16, 1024);
           mma_bf16_ss(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[x & 1]);
+        mma_commit(&s_full[b]);
       };
-      // O += P V with P (bf16) read from TMEM where the softmax warps stored it, over the
-      // first 32 columns of the score buffer it came from.
-      auto issue_pv = [&](int x) {
-        const int st = x % C::kStages;
-        const uint32_t p_tmem = tmem + ((x & 1) ? C::kColS1 : C::kColS0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = sdesc_sw128(v_addr + st * C::kKVTileBytes + kk * 2048, 8192, 1024);
-          mma_bf16_ts(tmem + C::kColO, p_tmem + kk * 8, bd, idesc_o, (x > 0 || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(q_full, 0, prm.status, kDevTimeoutQFull);
-      if (ok) ok = mbar_wait(&full[0], 0, prm.status, kDevTimeoutTmaFull);
-      if (ok && meta[0] != kEnd) {
+      for (int tc = 0; ok; ++tc) {
+        const int qb = tc & 1;
+        if (!mbar_wait(&q_full[qb], (tc >> 1) & 1, status, kDevTimeoutQFull)) break;
+        const int item = qmeta[2 * qb];
+        const int n = qmeta[2 * qb + 1];
+        if (item < 0) break;
         tc_fence_after();
-        issue_s(0);
-        for (int it = 0;; ++it) {
-          const int s1 = (it + 1) % C::kStages;
-          const int n1 = (it + 1) / C::kStages;
-          if (!mbar_wait(&full[s1], n1 & 1, prm.status, kDevTimeoutTmaFull)) break;
-          const bool end1 = meta[s1] == kEnd;
+        if (n > 0) {
+          if (!mbar_wait(&full[g % NST], (g / NST) & 1, status, kDevTimeoutTmaFull)) break;
           tc_fence_after();
-          if (!end1) issue_s(it + 1);
-          if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutPFull)) break;
-          tc_fence_after();
-          issue_pv(it);
-          mma_commit(&empty[it % C::kStages]);
-          mma_commit(o_bar);
-          if (end1) break;
+          issue_s(qb, g, 0);
+          for (int k = 0; k < n; ++k) {
+            if (k + 1 < n) {
+              const long long g1 = g + k + 1;
+              if (!mbar_wait(&full[g1 % NST], (g1 / NST) & 1, status, kDevTimeoutTmaFull)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(qb, g1, (k + 1) & 1);
+            }
+            if (k == 0 && tc > 0 &&
+                !mbar_wait(o_free, (tc - 1) & 1, status, kDevTimeoutOBar)) { ok = false; break; }
+            const int b = k & 1;
+            if (!mbar_wait(&p_full[b], pcount[b] & 1, status, kDevTimeoutPFull)) { ok = false; break; }
+            ++pcount[b];
+            tc_fence_after();
+            // O_b += P V: P (16-bit, 128 keys) in the first 64 columns of score buffer b,
+            // V pair MN-major (panel stride 16 KB along D, 8-row groups 1 KB apart).
+            const long long gk = g + k;
+            const int st = static_cast<int>(gk % NST);
+            const uint32_t vp = st_addr + static_cast<uint32_t>(st) * C::kStageBytes + C::kPairBytes;
+            const uint32_t p_tmem = tmem + (b ? C::kColS1 : C::kColS0);
+            const uint32_t o_tmem = tmem + (b ? C::kColO1 : C::kColO0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t bd = sdesc_sw128(vp + kk * 2048, 16384, 1024);
+              mma_bf16_ts(o_tmem, p_tmem + kk * 8, bd, idesc_o, (k >= 2 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[st]);
+          }
+          if (!ok) break;
+          g += n;
+        } else if (tc > 0) {
+          if (!mbar_wait(o_free, (tc - 1) & 1, status, kDevTimeoutOBar)) break;
         }
+        mma_commit(&q_empty[qb]);
+        mma_commit(tile_done);
       }
-      // o_final completes once when every MMA issued above has finished; the epilogue
-      // waits on it (a per-PV parity wait could be satisfied two phases early).
-      mma_commit(o_final);
-      // Drain: all MMAs of this CTA complete before TMEM is released.
       mma_commit(drain);
-      mbar_wait(drain, 0, prm.status, kDevTimeoutDrain);
+      mbar_wait(drain, 0, status, kDevTimeoutDrain);
     }
     __syncwarp();
   } else if (warp >= kSoftmaxWarp0) {
-    // ------------------------------------------------------------------ softmax + epilogue
-    const int row = threadIdx.x - kSoftmaxWarp0 * 32;            // 0..127 = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp - kSoftmaxWarp0) * 32) << 16;
+    // ------------------------------------------------------------------ softmax groups
+    const int grp = (warp - kSoftmaxWarp0) >> 2;                  // 0 or 1
+    const int row = ((warp - kSoftmaxWarp0) & 3) * 32 + lane;      // 0..127 = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(((warp - kSoftmaxWarp0) & 3) * 32) << 16;
     const bool upper = row >= 64;
     const float sl2 = prm.scale_log2;
-    float m_ref = -INFINITY;
-    float l = 0.f;
-    int it = 0;
+    const uint32_t s_col = tmem + lane_base + (grp ? C::kColS1 : C::kColS0);
+    long long g = 0;
+    int my_iter = 0;
     bool ok = true;
-    for (;; ++it) {
-      const int s = it % C::kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (it / C::kStages) & 1, prm.status, kDevTimeoutTmaFull));
+    for (int tc = 0; ok; ++tc) {
+      const int qb = tc & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qb], (tc >> 1) & 1, status, kDevTimeoutQFull));
       if (!ok) break;
-      const uint32_t mt = meta[s];
-      if (mt == kEnd) break;
-      const bool keep = upper ? ((mt >> 29) & 1u) : ((mt >> 28) & 1u);
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutSFull));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sa[32], sb[32];
-      {
-        const uint32_t col = (it & 1) ? C::kColS1 : C::kColS0;
-        tmem_ld32(tmem + lane_base + col, sa);
-        tmem_ld32(tmem + lane_base + col + 32, sb);
-        tmem_wait_ld();
-      }
-      float factor = 1.f;
-      bool rescale = false;
-      if (keep) {
+      const int item = qmeta[2 * qb];
+      const int n = qmeta[2 * qb + 1];
+      if (item < 0) break;
+      float m_ref = -INFINITY;
+      float l = 0.f;
+      for (int k = grp; k < n; k += 2) {
+        const long long gk = g + k;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[gk % NST], (gk / NST) & 1, status, kDevTimeoutTmaFull));
+        if (!ok) break;
+        const uint32_t mt = meta[gk % NST];
+        const uint32_t fa = (mt >> 14) & 3u, fb = (mt >> 30) & 3u;
+        const bool keep_a = upper ? (fa >> 1) : (fa & 1u);
+        const bool keep_b = upper ? (fb >> 1) : (fb & 1u);
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[grp], my_iter & 1, status, kDevTimeoutSFull));
+        if (!ok) break;
+        ++my_iter;
+        tc_fence_after();
+        // pass 1: row maximum over the kept half-rows
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(__uint_as_float(sa[c]), __uint_as_float(sb[c])));
+        for (int h = 0; h < 2; ++h) {
+          if (h == 0 ? keep_a : keep_b) {
+            uint32_t x[32], y[32];
+            tmem_ld32(s_col + h * 64, x);
+            tmem_ld32(s_col + h * 64 + 32, y);
+            tmem_wait_ld();
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              m4[c & 3] = fmaxf(m4[c & 3], fmaxf(__uint_as_float(x[c]), __uint_as_float(y[c])));
+            mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+          }
+        }
         const float rm = mx * sl2;
-        if (rm > m_ref + 8.0f) {
+        float factor = 1.f;
+        bool rescale = false;
+        if ((keep_a || keep_b) && rm > m_ref + 8.0f) {
           if (m_ref != -INFINITY) {
             factor = fast_exp2(m_ref - rm);
             rescale = true;
           }
           m_ref = rm;
         }
-      }
-      // Warp-uniform O correction (tcgen05.ld/st are warp-collective); lanes that do not
-      // rescale multiply by 1.
-      if (__any_sync(0xffffffffu, rescale)) {
-        l *= factor;
-        // O holds the sum of the previous iterations; wait for the last PV to land.
-        ok = __all_sync(0xffffffffu, mbar_wait(o_bar, (it - 1) & 1, prm.status, kDevTimeoutOBar));
-        if (!ok) break;
-        tc_fence_after();
+        // The group's previous PV has completed (it was issued before this step's S), so
+        // O can be rescaled in place; warp-uniform (tcgen05.ld/st are warp-collective).
+        if (__any_sync(0xffffffffu, rescale)) {
+          l *= factor;
+          const uint32_t o_col = tmem + lane_base + (grp ? C::kColO1 : C::kColO0);
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t ov[32];
-          tmem_ld32(tmem + lane_base + C::kColO + c0, ov);
-          tmem_wait_ld();
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(o_col + c0, ov);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * factor);
-          tmem_st32(tmem + lane_base + C::kColO + c0, ov);
-        }
-        tmem_wait_st();
-      }
-      // P = 2^(s*scale*log2e - m) as bf16 pairs, written over the score buffer in TMEM.
-      // Every fourth element uses the FMA-pipe exponential to offload the MUFU unit.
-      const uint32_t pcol = tmem + lane_base + ((it & 1) ? C::kColS1 : C::kColS0);
-      float sum = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint32_t (&sv)[32] = half ? sb : sa;
-        uint32_t packed[16];
-        if (keep) {
-#pragma unroll
-          for (int c = 0; c < 16; c += 2) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl2, -m_ref));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -m_ref));
-            const float p2 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 2]), sl2, -m_ref));
-            const float p3 = poly_exp2(fmaf(__uint_as_float(sv[2 * c + 3]), sl2, -m_ref));
-            // The row sum takes the rounded weights that enter the PV product, so the
-            // output is an exact convex combination of those weights.
-            if constexpr (VF16) {
-              packed[c] = pack_f16x2(p0, p1);
-              packed[c + 1] = pack_f16x2(p2, p3);
-              sum += (f16lo(packed[c]) + f16hi(packed[c])) + (f16lo(packed[c + 1]) + f16hi(packed[c + 1]));
-            } else {
-              packed[c] = pack_bf16x2(p0, p1);
-              packed[c + 1] = pack_bf16x2(p2, p3);
-              sum += (bf16lo(packed[c]) + bf16hi(packed[c])) + (bf16lo(packed[c + 1]) + bf16hi(packed[c + 1]));
-            }
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * factor);
+            tmem_st32(o_col + c0, ov);
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) packed[c] = 0u;
+          tmem_wait_st();
         }
-        tmem_st16(pcol + half * 16, packed);
+        // pass 2: P = 2^(s*scale*log2e - m) as 16-bit pairs into the first 64 columns of the
+        // score buffer (chunk c of 32 scores -> columns 16c..16c+15, already read).
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const bool kp = c < 2 ? keep_a : keep_b;
+          uint32_t packed[16];
+          if (kp) {
+            uint32_t sv[32];
+            tmem_ld32(s_col + c * 32, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * e]), sl2, -m_ref));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -m_ref));
+              const float p2 = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 2]), sl2, -m_ref));
+              const float p3 = poly_exp2(fmaf(__uint_as_float(sv[2 * e + 3]), sl2, -m_ref));
+              // The row sum takes the rounded weights that enter the PV product, so the
+              // output is an exact convex combination of those weights.
+              if constexpr (VF16) {
+                packed[e] = pack_f16x2(p0, p1);
+                packed[e + 1] = pack_f16x2(p2, p3);
+                sum0 += f16lo(packed[e]) + f16hi(packed[e]);
+                sum1 += f16lo(packed[e + 1]) + f16hi(packed[e + 1]);
+              } else {
+                packed[e] = pack_bf16x2(p0, p1);
+                packed[e + 1] = pack_bf16x2(p2, p3);
+                sum0 += bf16lo(packed[e]) + bf16hi(packed[e]);
+                sum1 += bf16lo(packed[e + 1]) + bf16hi(packed[e + 1]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) packed[e] = 0u;
+          }
+          tmem_st16(s_col + c * 16, packed);
+        }
+        l += sum0 + sum1;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[grp]);
       }
-      l += sum;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[it & 1]);
-    }
-    // ---- epilogue -----------------------------------------------------------------------
-    const int nit = it;
-    const bool valid_row = upper ? has_i1 : true;
-    const long long tok = bh * prm.S + static_cast<long long>(i0) * 64 + row;
-    bool have_o = ok && nit > 0;
-    if (have_o) {
-      have_o = __all_sync(0xffffffffu, mbar_wait(o_final, 0, prm.status, kDevTimeoutOBar));
+      if (!ok) break;
+      // ---- tile epilogue: merge the two groups' partial results ---------------------------
+      ok = __all_sync(0xffffffffu, mbar_wait(tile_done, tc & 1, status, kDevTimeoutOBar));
+      if (!ok) break;
       tc_fence_after();
-    }
-    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      float* m_sh = ml + (qb * 2) * 128;           // [group][row] for this tile parity
+      float* l_sh = ml + 512 + (qb * 2) * 128;
+      m_sh[grp * 128 + row] = m_ref;
+      l_sh[grp * 128 + row] = l;
+      named_barrier_sync(1, 256);
+      const float m0 = m_sh[row], m1 = m_sh[128 + row];
+      const float l0 = l_sh[row], l1 = l_sh[128 + row];
+      const float M = fmaxf(m0, m1);
+      const float f0 = l0 > 0.f ? fast_exp2(m0 - M) : 0.f;
+      const float f1 = l1 > 0.f ? fast_exp2(m1 - M) : 0.f;
+      const float L = l0 * f0 + l1 * f1;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float w0 = f0 * inv, w1 = f1 * inv;
+      const bool has0 = n > 0, has1 = n > 1;       // whether each group wrote O in this tile
+      const long long bh = item / prm.npairs;
+      const int i0 = 2 * (item - static_cast<int>(bh) * prm.npairs);
+      const bool valid_row = upper ? (i0 + 1 < nb) : true;
+      const long long tok = bh * prm.S + static_cast<long long>(i0) * 64 + row;
+      const uint32_t o0 = tmem + lane_base + C::kColO0, o1 = tmem + lane_base + C::kColO1;
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t ov[32];
-      if (have_o) {
-        tmem_ld32(tmem + lane_base + C::kColO + c0, ov);
+      for (int c0 = grp * (D / 2); c0 < (grp + 1) * (D / 2); c0 += 32) {
+        uint32_t a0[32], a1[32];
+        if (has0) tmem_ld32(o0 + c0, a0);
+        if (has1) tmem_ld32(o1 + c0, a1);
         tmem_wait_ld();
-      } else {
+        float* v = reinterpret_cast<float*>(a0);   // merged in place
 #pragma unroll
-        for (int c = 0; c < 32; ++c) ov[c] = 0u;
-      }
-      if (valid_row) {
-        if (prm.o_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(prm.o) + tok * D + c0);
+        for (int c = 0; c < 32; ++c)
+          v[c] = (has0 ? __uint_as_float(a0[c]) * w0 : 0.f) + (has1 ? __uint_as_float(a1[c]) * w1 : 0.f);
+        if (valid_row) {
+          if (prm.o_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(prm.o) + tok * D + c0);
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            dst[c] = make_float4(__uint_as_float(ov[4 * c]) * inv_l, __uint_as_float(ov[4 * c + 1]) * inv_l,
-                                 __uint_as_float(ov[4 * c + 2]) * inv_l, __uint_as_float(ov[4 * c + 3]) * inv_l);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.o) + tok * D + c0);
+            for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.o) + tok * D + c0);
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            dst[c] = make_uint4(pack_bf16x2(__uint_as_float(ov[8 * c]) * inv_l, __uint_as_float(ov[8 * c + 1]) * inv_l),
-                                pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv_l, __uint_as_float(ov[8 * c + 3]) * inv_l),
-                                pack_bf16x2(__uint_as_float(ov[8 * c + 4]) * inv_l, __uint_as_float(ov[8 * c + 5]) * inv_l),
-                                pack_bf16x2(__uint_as_float(ov[8 * c + 6]) * inv_l, __uint_as_float(ov[8 * c + 7]) * inv_l));
+            for (int c = 0; c < 4; ++c)
+              dst[c] = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                  pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+          }
         }
       }
+      if (grp == 0 && valid_row && prm.lse != nullptr)
+        prm.lse[tok] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+      tc_fence_before();
+      mbar_arrive(o_free);
+      g += n;
     }
-    if (valid_row && prm.lse != nullptr)
-      prm.lse[tok] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
   }
   // ------------------------------------------------------------------ teardown
   tc_fence_before();
@@ -425,14 +542,16 @@ cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& 
   CUtensorMap mq, mk, mv;
   const long long rows = static_cast<long long>(d.BH) * d.S;
   *map_ok = make_map_16(&mq, q, rows, D, 128, false) && make_map_16(&mk, k, rows, D, 64, false) &&
-            make_map_16(&mv, v, rows, D, 64, VF16);
+            make_map_16(&mv, v, rows, D, 64, VF16);   // K / V: one 64-row block per copy
   if (!*map_ok) return cudaErrorInvalidValue;
   using C = FwdCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, VF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const unsigned items = static_cast<unsigned>(d.BH) * static_cast<unsigned>((d.nb + 1) / 2);
-  attn_fwd_kernel<D, VF16><<<items, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, prm);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = prm.items < sms ? prm.items : sms;
+  attn_fwd_kernel<D, VF16><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 }  // namespace
@@ -448,17 +567,16 @@ extern "C" size_t nabla_fwd_workspace_bytes(nabla_shape s) {
 }
 
 extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void* v,
-                                       nabla_dtype v_dtype, const int32_t* row_idx, const int32_t* row_cnt,
+                                       nabla_dtype v_dtype, const uint32_t* mask_bits,
                                        nabla_shape s, float scale, void* o, nabla_dtype o_dtype,
                                        float* lse, void* workspace, size_t workspace_bytes,
                                        nabla_stream_t stream) {
   Dims d;
   nabla_status rc = check_shape(s, &d);
   if (rc != NABLA_OK) return rc;
-  if (!q || !k || !v || !o || !row_idx || !row_cnt) return NABLA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !mask_bits) return NABLA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return NABLA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(row_idx) & 3) || (reinterpret_cast<uintptr_t>(row_cnt) & 3) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+  if ((reinterpret_cast<uintptr_t>(mask_bits) & 3) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
     return NABLA_ERR_INVALID_ARG;
   if (o_dtype != NABLA_BF16 && o_dtype != NABLA_F32) return NABLA_ERR_INVALID_ARG;
   if (v_dtype != NABLA_BF16 && v_dtype != NABLA_F16) return NABLA_ERR_INVALID_ARG;
@@ -468,8 +586,8 @@ extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void*
     return NABLA_ERR_WORKSPACE;
   if (static_cast<long long>(d.BH) * d.S >= (1ll << 31)) return NABLA_ERR_UNSUPPORTED;
   FwdParams prm;
-  prm.row_idx = row_idx;
-  prm.row_cnt = row_cnt;
+  prm.bits = mask_bits;
+  prm.nw = d.nw;
   prm.o = o;
   prm.lse = lse;
   prm.status = static_cast<uint32_t*>(workspace);
@@ -481,10 +599,11 @@ extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void*
   cudaError_t ce = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
   if (ce != cudaSuccess) return cuda_status(ce);
   int32_t* order = nullptr;
-  ce = build_schedule(row_cnt, d, static_cast<char*>(workspace) + kStatusBytes, &order, st);
+  ce = build_schedule(nullptr, mask_bits, d, static_cast<char*>(workspace) + kStatusBytes, &order, st);
   if (ce != cudaSuccess) return cuda_status(ce);
   prm.order = order;
   prm.npairs = (d.nb + 1) / 2;
+  prm.items = d.BH * prm.npairs;
   bool map_ok = true;
   const bool vf16 = v_dtype == NABLA_F16;
   cudaError_t e = d.D == 64 ? (vf16 ? launch_fwd<64, true>(q, k, v, d, prm, st, &map_ok)

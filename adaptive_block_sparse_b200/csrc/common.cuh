@@ -33,8 +33,8 @@ nabla_status cuda_status(cudaError_t e);
 
 // Longest-first tile order (schedule.cu): scratch size and builder.
 size_t schedule_scratch_bytes(const Dims& d);
-cudaError_t build_schedule(const int32_t* cnt, const Dims& d, void* scratch, int32_t** order_out,
-                           cudaStream_t st);
+cudaError_t build_schedule(const int32_t* cnt, const uint32_t* bits, const Dims& d, void* scratch,
+                           int32_t** order_out, cudaStream_t st);
 
 // Device status codes (recorded in workspace word 0; first error wins).
 enum : uint32_t {

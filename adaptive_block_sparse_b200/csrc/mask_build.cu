@@ -37,7 +37,6 @@ namespace {
 
 constexpr int kThreads = 256;   // 8 warps; one pooled row per warp during selection
 constexpr int kWarps = kThreads / 32;
-constexpr int KC = 32;          // pooled key rows per shared-memory chunk
 constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
 constexpr double kFix = 4611686018427387904.0;  // 2^62
 constexpr int kRescueCtasPerHead = 16;
@@ -45,7 +44,7 @@ constexpr int kRescueCtasPerHead = 16;
 __device__ __forceinline__ unsigned long long to_fix(double p) { return __double2ull_rn(p * kFix); }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) mask_rows_kernel(
+__global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
     const double* __restrict__ qpool, const double* __restrict__ kpool, int nb, int nw, int R,
     double scale, double thr, int sta_on, int wt2, int wh2, int ww2, int Hb, int Wb,
     uint32_t* __restrict__ bits, int32_t* __restrict__ row_idx, int32_t* __restrict__ row_cnt,
@@ -56,9 +55,8 @@ __global__ void __launch_bounds__(kThreads) mask_rows_kernel(
   __shared__ int rows_s[8];
   unsigned long long* hmass = reinterpret_cast<unsigned long long*>(smem_raw);  // 8 x 256
   uint32_t* hcnt = reinterpret_cast<uint32_t*>(hmass + kWarps * 256);           // 8 x 256
-  double* qs = reinterpret_cast<double*>(hcnt + kWarps * 256);                  // R x D
-  double* ks = qs + R * D;                                                      // KC x (D+1)
-  double* prow = ks + KC * (D + 1);                                             // R x nb
+  double* qs = reinterpret_cast<double*>(hcnt + kWarps * 256);                  // 8 x D
+  double* prow = qs + 8 * D;                                                    // R x nb
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -81,29 +79,35 @@ __global__ void __launch_bounds__(kThreads) mask_rows_kernel(
                               : 0;
   __syncthreads();
 
-  for (int e = tid; e < R * D; e += kThreads) {
+  for (int e = tid; e < 8 * D; e += kThreads) {
     const int r = e / D;
     qs[e] = (r < nrows) ? qpool[(bh * nb + rows_s[r]) * D + (e - r * D)] : 0.0;
   }
-  // ---- pooled logits A = Qp Kp^T * scale (fp64) --------------------------------------
-  for (int j0 = 0; j0 < nb; j0 += KC) {
-    __syncthreads();
-    for (int e = tid; e < KC * D; e += kThreads) {
-      const int jj = e / D;
-      const int dd = e - jj * D;
-      ks[jj * (D + 1) + dd] = (j0 + jj < nb) ? kpool[(bh * nb + j0 + jj) * D + dd] : 0.0;
-    }
-    __syncthreads();
-    for (int e = tid; e < R * KC; e += kThreads) {
-      const int r = e / KC;
-      const int jj = e - r * KC;
-      if (r < nrows && j0 + jj < nb) {
-        const double* qr = qs + r * D;
-        const double* kr = ks + jj * (D + 1);
-        double acc = 0.0;
-#pragma unroll 16
-        for (int dd = 0; dd < D; ++dd) acc = fma(qr[dd], kr[dd], acc);
-        prow[r * nb + j0 + jj] = acc * scale;
+  // ---- pooled logits A = Qp Kp^T * scale (fp64 tensor-core MMA, m8n8k4) ---------------
+  // The (up to 8) rows of the group are the M = 8 side; each warp takes 8 key blocks at a
+  // time (N = 8) and walks D in steps of 4.  Fragments: A[row = lane/4][k = lane%4],
+  // B[k = lane%4][key = lane/4], C[row = lane/4][key = 2*(lane%4) + {0,1}].
+  __syncthreads();
+  {
+    const int gid = lane >> 2, tig = lane & 3;
+    double afrag[D / 4];
+#pragma unroll
+    for (int kk = 0; kk < D / 4; ++kk) afrag[kk] = qs[gid * D + kk * 4 + tig];
+    for (int jt = warp; jt * 8 < nb; jt += kWarps) {
+      const int key = jt * 8 + gid;
+      const double* kr = kpool + (bh * nb + (key < nb ? key : 0)) * D + tig;
+      double c0 = 0.0, c1 = 0.0;
+#pragma unroll
+      for (int kk = 0; kk < D / 4; ++kk) {
+        const double b = key < nb ? __ldg(kr + kk * 4) : 0.0;
+        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                     : "+d"(c0), "+d"(c1)
+                     : "d"(afrag[kk]), "d"(b));
+      }
+      const int key0 = jt * 8 + 2 * tig;
+      if (gid < nrows) {
+        if (key0 < nb) prow[gid * nb + key0] = c0 * scale;
+        if (key0 + 1 < nb) prow[gid * nb + key0 + 1] = c1 * scale;
       }
     }
   }
@@ -313,8 +317,8 @@ int rows_per_cta(int nb) {
 }
 
 size_t mask_rows_smem(int nb, int D, int R) {
-  return static_cast<size_t>(kWarps) * 256 * (8 + 4) + static_cast<size_t>(R) * D * 8 +
-         static_cast<size_t>(KC) * (D + 1) * 8 + static_cast<size_t>(R) * nb * 8;
+  return static_cast<size_t>(kWarps) * 256 * (8 + 4) + static_cast<size_t>(8) * D * 8 +
+         static_cast<size_t>(R) * nb * 8;
 }
 
 template <int D>

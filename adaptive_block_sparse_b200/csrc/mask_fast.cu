@@ -267,39 +267,80 @@ __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm
   };
   bool certified = false;
   uint32_t kcut = 0;
+  // rho: relative error of every probability (two logits' errors, exp, division);
+  // eta: error of a ranked mass.
+  const float eps = prm.scale * prm.qnorm[bh * nb + i] * __uint_as_float(prm.kmax_bits[bh]) * kLogitErr;
+  const float rho = 2.f * eps + 1e-5f;
+  const float eta = rho + 3.5e-6f;
+  // Certificate for a cut at value p_cut with ranked masses e_above (strictly above) and
+  // e_at (at or above), the next smaller value p_next and n_at values equal to p_cut.
+  // The kept set {P >= p_cut} must have exact mass > thr, and without its (exactly)
+  // smallest member -- at most e_above + eta + rho p_cut -- exact mass < thr.
+  auto certify = [&](float e_above, float e_at, float p_cut, float p_next, int n_at) {
+    return (thr - e_above > eta + rho * p_cut) && (e_at - thr > eta) && n_at == 1 &&
+           (p_cut - p_next > 2.f * rho * p_cut);
+  };
   if (prm.thr_mode != 0) {            // thr >= 1: keep every block; thr <= 0: none
     certified = true;
     kcut = prm.thr_mode > 0 ? 0u : 0xFFFFFFFFu;
-  } else if (mass_ge(0u) >= thr) {
-    uint32_t lo = 0u, hi = 0x3F800001u;      // mass_ge(lo) >= thr > mass_ge(hi)
-    while (hi - lo > 1u) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (mass_ge(mid) >= thr) lo = mid; else hi = mid;
-    }
-    kcut = lo;
-    const float e_above = mass_ge(kcut + 1u);
-    const float e_at = mass_ge(kcut);
-    int n_at = 0;
-    float p_next = 0.f;
+  } else {
+    // Fast path: take maxima in descending order (ties: lower block index first) while
+    // the running mass is below thr; most rows keep only a few blocks.
+    constexpr int kMaxExtract = 8;
+    uint64_t taken = 0;                 // bit t: p[t] of this lane already taken
+    float acc = 0.f, acc_prev = 0.f;
+    bool found = false;
+    float p_cut = 0.f;
+    for (int e = 0; e <= kMaxExtract; ++e) {
+      float best = -1.f;
+      int bj = 0x7FFFFFFF;
 #pragma unroll
-    for (int t = 0; t < TPL; ++t) {
-      const uint32_t key = __float_as_uint(p[t]);
-      n_at += key == kcut;
-      if (key < kcut) p_next = fmaxf(p_next, p[t]);
-    }
+      for (int t = 0; t < TPL; ++t)
+        if (!((taken >> t) & 1ull) && p[t] > best) { best = p[t]; bj = lane + 32 * t; }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n_at += __shfl_xor_sync(0xffffffffu, n_at, o);
-    p_next = warp_max(p_next);
-    const float p_cut = __uint_as_float(kcut);
-    // rho: relative error of every probability (two logits' errors, exp, division).
-    const float eps = prm.scale * prm.qnorm[bh * nb + i] * __uint_as_float(prm.kmax_bits[bh]) * kLogitErr;
-    const float rho = 2.f * eps + 1e-5f;
-    const float eta = rho + 3.5e-6f;
-    // The kept set is {P >= P_c}; its exact mass must exceed thr, and the exact mass of
-    // the set without its (exactly) smallest member -- at most e_above + eta + rho P_c --
-    // must stay below thr.
-    certified = (thr - e_above > eta + rho * p_cut) && (e_at - thr > eta) && n_at == 1 &&
-                (p_cut - p_next > 2.f * rho * p_cut);
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+        if (ov > best || (ov == best && oj < bj)) { best = ov; bj = oj; }
+      }
+      if (found) {                      // one more maximum: the first value below the cut
+        certified = certify(acc_prev, acc, p_cut, fmaxf(best, 0.f), best == p_cut ? 2 : 1);
+        break;
+      }
+      if (bj == 0x7FFFFFFF || e == kMaxExtract) break;
+      if ((bj & 31) == lane) taken |= 1ull << (bj >> 5);
+      acc_prev = acc;
+      acc += best;
+      if (acc >= thr) {
+        found = true;
+        p_cut = best;
+        kcut = __float_as_uint(best);
+      }
+    }
+    if (!found && mass_ge(0u) >= thr) {
+      // General path: bisection over the fp32 bit patterns for the largest key k with
+      // mass(P >= k) >= thr.
+      uint32_t lo = 0u, hi = 0x3F800001u;      // mass_ge(lo) >= thr > mass_ge(hi)
+      while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (mass_ge(mid) >= thr) lo = mid; else hi = mid;
+      }
+      kcut = lo;
+      const float e_above = mass_ge(kcut + 1u);
+      const float e_at = mass_ge(kcut);
+      int n_at = 0;
+      float p_next = 0.f;
+#pragma unroll
+      for (int t = 0; t < TPL; ++t) {
+        const uint32_t key = __float_as_uint(p[t]);
+        n_at += key == kcut;
+        if (key < kcut) p_next = fmaxf(p_next, p[t]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) n_at += __shfl_xor_sync(0xffffffffu, n_at, o);
+      p_next = warp_max(p_next);
+      certified = certify(e_above, e_at, __uint_as_float(kcut), p_next, n_at);
+    }
   }
   if (!certified) {
     if (lane == 0) {

@@ -1,95 +1,91 @@
-// Longest-first ordering of attention work items (tile = pair of consecutive blocks of
-// one head).  Heads of one problem can differ by two orders of magnitude in kept tiles,
-// so the tiles are dispatched in descending order of their list lengths (an upper bound
-// of the union walked by the tile): a counting sort on the device into caller-provided
-// scratch.  Ties keep no particular order; the result of every tile is independent of
-// the order, so outputs stay deterministic.
+// Order of attention work items (tile = pair of consecutive blocks of one head).
+//
+// Heads are taken one after another (head-major), so the tiles running at the same time
+// read K and V of one head and those stay resident in L2; inside a head, tiles run
+// longest first (descending length of their two kept lists, an upper bound of the
+// union a tile walks), which keeps the tail short.  One CTA sorts one head's tiles with
+// a bitonic sort on (length descending, tile index ascending): the order is fully
+// deterministic, and every tile's result is independent of the order anyway.
 #include "common.cuh"
 
 namespace nabla {
 namespace {
 
-__global__ void sched_hist_kernel(const int32_t* __restrict__ cnt, int nb, int npairs, long long items,
-                                  int32_t* __restrict__ cost_of, int32_t* __restrict__ hist) {
-  const long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (it >= items) return;
-  const long long bh = it / npairs;
-  const int p = static_cast<int>(it - bh * npairs);
-  const int i0 = 2 * p;
-  int c = min(max(cnt[bh * nb + i0], 0), nb);
-  if (i0 + 1 < nb) c += min(max(cnt[bh * nb + i0 + 1], 0), nb);
-  cost_of[it] = c;
-  atomicAdd(&hist[c], 1);
-}
-
-// Exclusive scan in descending cost order: offset[c] = #items with cost > c.
-__global__ void __launch_bounds__(1024) sched_scan_kernel(int32_t* __restrict__ hist, int nbins) {
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int base = 0; base < nbins; base += 1024) {
-    const int c = nbins - 1 - (base + threadIdx.x);   // descending cost
-    const int v = (c >= 0) ? hist[c] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      int w = warp_sums[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += t;
+// Tile length: with `bits` the exact union size popc(row 2e | row 2e+1); otherwise the
+// sum of the two list counts.
+__global__ void __launch_bounds__(512) sched_head_sort_kernel(const int32_t* __restrict__ cnt,
+                                                              const uint32_t* __restrict__ bits,
+                                                              int nb, int nw, int npairs, int npow2,
+                                                              int32_t* __restrict__ order) {
+  extern __shared__ unsigned long long keys[];
+  const long long bh = blockIdx.x;
+  for (int e = threadIdx.x; e < npow2; e += blockDim.x) {
+    unsigned long long key = ~0ull;
+    if (e < npairs) {
+      const int i0 = 2 * e;
+      int c = 0;
+      if (bits != nullptr) {
+        const uint32_t* r0 = bits + (bh * nb + i0) * static_cast<long long>(nw);
+        const uint32_t* r1 = (i0 + 1 < nb) ? r0 + nw : nullptr;
+        for (int w = 0; w < nw; ++w) {
+          uint32_t u = r0[w] | (r1 ? r1[w] : 0u);
+          if (w == nw - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
+          c += __popc(u);
+        }
+      } else {
+        c = min(max(cnt[bh * nb + i0], 0), nb);
+        if (i0 + 1 < nb) c += min(max(cnt[bh * nb + i0 + 1], 0), nb);
       }
-      warp_sums[lane] = w;
+      key = (static_cast<unsigned long long>(0x7FFFFFFF - c) << 32) | static_cast<unsigned>(e);
     }
-    __syncthreads();
-    const int prefix = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - v;
-    __syncthreads();
-    if (c >= 0) hist[c] = prefix;
-    if (threadIdx.x == 1023) carry = prefix + v;
-    __syncthreads();
+    keys[e] = key;
   }
+  __syncthreads();
+  for (int k = 2; k <= npow2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int e = threadIdx.x; e < npow2; e += blockDim.x) {
+        const int p = e ^ j;
+        if (p > e) {
+          const unsigned long long a = keys[e], b = keys[p];
+          const bool up = (e & k) == 0;
+          if ((a > b) == up) {
+            keys[e] = b;
+            keys[p] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int e = threadIdx.x; e < npairs; e += blockDim.x)
+    order[bh * npairs + e] = static_cast<int32_t>(bh * npairs + static_cast<long long>(keys[e] & 0xFFFFFFFFull));
 }
 
-__global__ void sched_scatter_kernel(const int32_t* __restrict__ cost_of, long long items,
-                                     int32_t* __restrict__ offset, int32_t* __restrict__ order) {
-  const long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (it >= items) return;
-  const int pos = atomicAdd(&offset[cost_of[it]], 1);
-  order[pos] = static_cast<int32_t>(it);
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
 }
 
 }  // namespace
 
 size_t schedule_scratch_bytes(const Dims& d) {
   const size_t items = static_cast<size_t>(d.BH) * ((d.nb + 1) / 2);
-  const size_t nbins = 2 * static_cast<size_t>(d.nb) + 1;
-  return align_up(items * 4, 256) * 2 + align_up(nbins * 4, 256);
+  return align_up(items * 4, 256);
 }
 
-// Writes the item order (descending cost) to the start of `scratch`; returns it.
-cudaError_t build_schedule(const int32_t* cnt, const Dims& d, void* scratch, int32_t** order_out,
-                           cudaStream_t st) {
-  const long long npairs = (d.nb + 1) / 2;
-  const long long items = static_cast<long long>(d.BH) * npairs;
-  const int nbins = 2 * d.nb + 1;
-  char* base = static_cast<char*>(scratch);
-  int32_t* order = reinterpret_cast<int32_t*>(base);
-  int32_t* cost_of = reinterpret_cast<int32_t*>(base + align_up(items * 4, 256));
-  int32_t* hist = reinterpret_cast<int32_t*>(base + 2 * align_up(items * 4, 256));
-  cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(nbins) * 4, st);
+// Writes the item order to the start of `scratch`; returns it.  Tile lengths from the
+// bitmask when `bits` is given, else from the list counts `cnt`.
+cudaError_t build_schedule(const int32_t* cnt, const uint32_t* bits, const Dims& d, void* scratch,
+                           int32_t** order_out, cudaStream_t st) {
+  const int npairs = (d.nb + 1) / 2;
+  const int npow2 = next_pow2(npairs);
+  int32_t* order = static_cast<int32_t*>(scratch);
+  const size_t smem = static_cast<size_t>(npow2) * 8;
+  cudaError_t e = cudaFuncSetAttribute(sched_head_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned blocks = static_cast<unsigned>((items + 255) / 256);
-  sched_hist_kernel<<<blocks, 256, 0, st>>>(cnt, d.nb, static_cast<int>(npairs), items, cost_of, hist);
-  sched_scan_kernel<<<1, 1024, 0, st>>>(hist, nbins);
-  sched_scatter_kernel<<<blocks, 256, 0, st>>>(cost_of, items, hist, order);
+  sched_head_sort_kernel<<<d.BH, 512, smem, st>>>(cnt, bits, d.nb, d.nw, npairs, npow2, order);
   *order_out = order;
   return cudaGetLastError();
 }

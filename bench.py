@@ -206,7 +206,7 @@ class Path:
                            col_cnt=self.ccnt, q_pool=self.qp, k_pool=self.kp,
                            workspace=self.mask_ws)
         self._mark("t_mask", timing)
-        m.nabla_attn_fwd(self.qf, self.kf, self.vf, self.ridx, self.rcnt, sh, o=self.o,
+        m.nabla_attn_fwd(self.qf, self.kf, self.vf, self.bits, sh, o=self.o,
                          o_dtype=self.o_dtype, lse=self.lse, workspace=self.fwd_ws)
         self._mark("t_fwd", timing)
         if wl.backward:
@@ -404,21 +404,16 @@ def main():
                                                    row_cnt=path.rcnt, workspace=path.mask_ws), 5)
     mask_bytes = 2 * BH * wl.S * wl.D * 2 + BH * nb * sh.nw * 4
     reorder_bytes = 3 * 2 * BH * wl.S * wl.D * 2 + 2 * BH * nb * wl.D * 8
-    ones = torch.full((wl.B, wl.H, nb, nb), True)
-    import oracle
-    dense_bits = torch.from_numpy(oracle.pack_mask_bits(ones.numpy()[:1, :1]).view(np.int32)).to(dev)
-    dense_bits = dense_bits.expand(wl.B, wl.H, nb, sh.nw).contiguous()
-    d_ridx = torch.empty(wl.B, wl.H, nb, nb, dtype=torch.int32, device=dev)
-    d_rcnt = torch.empty(wl.B, wl.H, nb, dtype=torch.int32, device=dev)
-    m.nabla_mask_lists(dense_bits, sh, d_ridx, d_rcnt)
+    # all-ones mask (padding bits are ignored by the kernels)
+    dense_bits = torch.full((wl.B, wl.H, nb, sh.nw), -1, dtype=torch.int32, device=dev)
     dense_iters = 2 if nb > 1000 else 5
-    dense_ms = time_call(lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, d_ridx, d_rcnt, sh,
+    dense_ms = time_call(lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, dense_bits, sh,
                                                   o=path.o, o_dtype=path.o_dtype, lse=path.lse,
                                                   workspace=path.fwd_ws), dense_iters, warm=1)
     dense_tflops = BH * nb * nb * fl_fwd / (dense_ms * 1e-3) / 1e12
     path.check_status()
     # restore the NABLA lists (the dense run reused the output buffers only)
-    del d_ridx, d_rcnt, dense_bits
+    del dense_bits
 
     # ---- end to end through the public API with host buffers --------------------------------
     hq, hk, hv = (t.cpu().pin_memory() for t in (path.q, path.k, path.v))

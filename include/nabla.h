@@ -139,10 +139,11 @@ nabla_status nabla_mask_lists(const uint32_t *mask_bits, nabla_shape s, int32_t 
  *   of row i;  LSE_r = ln sum_c exp(scale * Q_r . K_c).
  * A row with no kept block gives O = 0 and LSE = -inf.
  *
- * q, k       : bf16 [B,H,S,D] reordered.  row_idx / row_cnt as from nabla_build_mask.
+ * q, k       : bf16 [B,H,S,D] reordered.
  * v, v_dtype : [B,H,S,D] reordered, NABLA_BF16 or NABLA_F16.  With fp16 V the
  *              probabilities P enter the PV product as fp16 (11-bit significand)
  *              instead of bf16 (8-bit): about 8x smaller output error.
+ * mask_bits  : the block mask as from nabla_build_mask (padding bits are ignored).
  * o          : out [B,H,S,D], bf16 or f32 per o_dtype.   lse: out f32 [B,H,S] (natural
  *              log; nullable when not needed).
  * workspace  : >= nabla_fwd_workspace_bytes(s) bytes (tile schedule + status word).
@@ -150,9 +151,9 @@ nabla_status nabla_mask_lists(const uint32_t *mask_bits, nabla_shape s, int32_t 
  * --------------------------------------------------------------------------------- */
 size_t nabla_fwd_workspace_bytes(nabla_shape s);
 nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v, nabla_dtype v_dtype,
-                            const int32_t *row_idx, const int32_t *row_cnt, nabla_shape s,
-                            float scale, void *o, nabla_dtype o_dtype, float *lse,
-                            void *workspace, size_t workspace_bytes, nabla_stream_t stream);
+                            const uint32_t *mask_bits, nabla_shape s, float scale, void *o,
+                            nabla_dtype o_dtype, float *lse, void *workspace,
+                            size_t workspace_bytes, nabla_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Block-sparse attention backward (mask constant)                   [ZH-TS, LSD-2]
@@ -197,9 +198,9 @@ nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, nabla_d
  * device status word of the last call is not readable through this entry point.
  * --------------------------------------------------------------------------------- */
 nabla_status nabla_attn_fwd_noalloc(const void *q, const void *k, const void *v,
-                                    nabla_dtype v_dtype, const int32_t *row_idx,
-                                    const int32_t *row_cnt, nabla_shape s, float scale, void *o,
-                                    nabla_dtype o_dtype, float *lse, nabla_stream_t stream);
+                                    nabla_dtype v_dtype, const uint32_t *mask_bits, nabla_shape s,
+                                    float scale, void *o, nabla_dtype o_dtype, float *lse,
+                                    nabla_stream_t stream);
 
 /* Reads (synchronously on `stream`) the device status word that the kernels of the
  * last call on `workspace` recorded: 0 = fine, otherwise a code naming the barrier

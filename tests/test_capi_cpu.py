@@ -96,7 +96,7 @@ def test_host_validation_rejects_bad_arguments(lib):
     fws = lib.nabla_fwd_workspace_bytes(good)
 
     def fwd(q=A, o=Bp, scale=0.125, odt=0, ws=Bp, wsb=fws, ridx=A, vdt=0):
-        return lib.nabla_attn_fwd(q, A, A, vdt, ridx, A, good, scale, o, odt, None, ws, wsb, st)
+        return lib.nabla_attn_fwd(q, A, A, vdt, ridx, good, scale, o, odt, None, ws, wsb, st)
     assert fwd(q=None) == INV
     assert fwd(q=mis) == INV
     assert fwd(ridx=None) == INV

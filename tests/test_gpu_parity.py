@@ -104,7 +104,7 @@ def _fwd_case(data, wl, thr, window, o_dtype, v_dtype=torch.float16):
     bits, ridx, rcnt, _, _ = gpu_mask(qf, kf, shape, thr, window, cols=False)
     lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
     ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
-    o, _ = m.nabla_attn_fwd(qf, kf, vk, ridx, rcnt, shape, o_dtype=o_dtype, lse=lse, workspace=ws)
+    o, _ = m.nabla_attn_fwd(qf, kf, vk, bits, shape, o_dtype=o_dtype, lse=lse, workspace=ws)
     torch.cuda.synchronize()
     assert m.nabla_read_device_status(ws) == 0
     gm = bits_to_mask(bits, wl.nb)
@@ -151,7 +151,7 @@ def test_fwd_dense_and_empty_rows(data):
         m.nabla_mask_lists(bits, shape, ridx, rcnt)
         lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
         ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
-        o, _ = m.nabla_attn_fwd(qf, kf, vk, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse,
+        o, _ = m.nabla_attn_fwd(qf, kf, vk, bits, shape, o_dtype=m.NABLA_F32, lse=lse,
                                 workspace=ws)
         torch.cuda.synchronize()
         assert m.nabla_read_device_status(ws) == 0
@@ -182,7 +182,7 @@ def test_bwd_parity(data, name, thr, window):
     bits, ridx, rcnt, cidx, ccnt = gpu_mask(qf, kf, shape, thr, window)
     lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
     fws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
-    o, _ = m.nabla_attn_fwd(qf, kf, vk, ridx, rcnt, shape, o_dtype=m.NABLA_F32, lse=lse, workspace=fws)
+    o, _ = m.nabla_attn_fwd(qf, kf, vk, bits, shape, o_dtype=m.NABLA_F32, lse=lse, workspace=fws)
     do = make_dout(wl, device=DEV)
     bws = torch.zeros(m.nabla_bwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
     dq, dk, dv = m.nabla_attn_bwd(qf, kf, vk, o, do, lse, ridx, rcnt, cidx, ccnt, shape, workspace=bws)

@@ -26,18 +26,18 @@ def test_noalloc_forward_matches_regular_entry_point(name, o_dtype):
     qf, _ = gpu_reorder(q, shape)
     kf, _ = gpu_reorder(k, shape)
     vk, _ = gpu_reorder(v, shape, dtype=torch.float16)
-    _, ridx, rcnt, _, _ = gpu_mask(qf, kf, shape, wl.thrs[-1], (0, 0, 0), cols=False)
+    bits, _, _, _, _ = gpu_mask(qf, kf, shape, wl.thrs[-1], (0, 0, 0), cols=False)
     odt = m.NABLA_F32 if o_dtype == torch.float32 else m.NABLA_BF16
     lse_ref = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
     ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
-    o_ref, _ = m.nabla_attn_fwd(qf, kf, vk, ridx, rcnt, shape, o_dtype=odt, lse=lse_ref, workspace=ws)
+    o_ref, _ = m.nabla_attn_fwd(qf, kf, vk, bits, shape, o_dtype=odt, lse=lse_ref, workspace=ws)
     torch.cuda.synchronize()
     assert m.nabla_read_device_status(ws) == 0
     ref = o_ref.double().cpu().numpy()
     for call in range(2):                      # two calls in a row share the scratch array
         o = torch.full(q.shape, float("nan"), dtype=o_dtype, device=DEV)
         lse = torch.full((wl.B, wl.H, wl.S), float("nan"), dtype=torch.float32, device=DEV)
-        m.nabla_attn_fwd_noalloc(qf, kf, vk, ridx, rcnt, shape, o, lse)
+        m.nabla_attn_fwd_noalloc(qf, kf, vk, bits, shape, o, lse)
         torch.cuda.synchronize()
         err = np.abs(o.double().cpu().numpy() - ref)
         assert err.max() <= FWD_MAX_ABS and err.mean() <= FWD_MEAN_ABS, (call, err.max())
@@ -52,5 +52,5 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     x = torch.zeros(16, dtype=torch.bfloat16, device=DEV)    # never read: rejected first
     i = torch.zeros(16, dtype=torch.int32, device=DEV)
     with pytest.raises(m.NablaError) as e:
-        m.nabla_attn_fwd_noalloc(x, x, x.to(torch.float16), i, i, big, x)
+        m.nabla_attn_fwd_noalloc(x, x, x.to(torch.float16), i, big, x)
     assert e.value.status == m.NABLA_ERR_UNSUPPORTED
