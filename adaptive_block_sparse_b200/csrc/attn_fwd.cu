@@ -33,8 +33,9 @@
 namespace nabla {
 namespace {
 
-constexpr int kThreads = 384;             // 12 warps
+constexpr int kThreads = 512;             // 16 warps
 constexpr int kSoftmaxWarp0 = 4;          // warps 4..7 = group 0, 8..11 = group 1
+constexpr int kEpilogueWarp0 = 12;        // warps 12..15
 constexpr int kMaxWords = 512;            // bitmask words per row (nb <= 16384)
 
 template <int D>
@@ -69,10 +70,6 @@ struct FwdParams {
   int o_f32;
 };
 
-__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
 // Walks the set bits of w0 | w1 (two rows' bitmask words in shared memory) in ascending
 // order; f = bit0: kept by the first row, bit1: kept by the second.
 struct BitWalk {
@@ -95,6 +92,15 @@ struct BitWalk {
   }
 };
 
+// Roles (one CTA per SM, tiles taken in turn; tile t uses buffer set qb = t & 1):
+//   warp 2      tile loader: takes the next tile, copies its two bitmask rows to shared
+//               memory, counts the union and loads Q (q_full[qb]);
+//   warp 0      K/V streamer: walks the union two key blocks per step into the stages;
+//   warp 1      MMA issuer;
+//   warps 4-11  two softmax groups on alternate steps; at the end of a tile each writes
+//               its running (max, sum) and moves on (ml_ready[qb]);
+//   warps 12-15 epilogue: merges the two groups' accumulators and stores O and LSE,
+//               then frees the accumulators and the tile's buffer set (o_free[qb]).
 template <int D, bool VF16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q,
@@ -112,15 +118,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;                 // [NST]
   uint64_t* empty = full + NST;          // [NST]
-  uint64_t* q_full = empty + NST;        // [2]
-  uint64_t* q_empty = q_full + 2;        // [2]
-  uint64_t* s_full = q_empty + 2;        // [2]
-  uint64_t* p_full = s_full + 2;         // [2]
-  uint64_t* tile_done = p_full + 2;
-  uint64_t* o_free = tile_done + 1;
-  uint64_t* drain = o_free + 1;
-  uint32_t* meta = reinterpret_cast<uint32_t*>(drain + 1);   // [NST]
-  int32_t* qmeta = reinterpret_cast<int32_t*>(meta + NST);   // [2][2]: item, blocks
+  uint64_t* q_full = empty + NST;        // [2] loader -> all
+  uint64_t* q_empty = q_full + 2;        // [2] MMA: Q buffer no longer read
+  uint64_t* s_full = q_empty + 2;        // [2] per softmax group
+  uint64_t* p_full = s_full + 2;         // [2] per softmax group
+  uint64_t* tile_done = p_full + 2;      // [2] MMA: the tile's last PV landed
+  uint64_t* ml_ready = tile_done + 2;    // [2] softmax groups -> epilogue
+  uint64_t* o_free = ml_ready + 2;       // [2] epilogue: accumulators read, tile retired
+  uint64_t* drain = o_free + 2;
+  int32_t* qmeta = reinterpret_cast<int32_t*>(drain + 1);    // [2][2]: item, steps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qmeta + 4);
 
   const int warp = threadIdx.x >> 5;
@@ -139,9 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_empty[b], 1);
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 128);
+      mbar_init(&tile_done[b], 1);
+      mbar_init(&ml_ready[b], 256);
+      mbar_init(&o_free[b], 128);
     }
-    mbar_init(tile_done, 1);
-    mbar_init(o_free, 256);
     mbar_init(drain, 1);
     fence_mbarrier_init();
   }
@@ -154,20 +161,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
-    }
-    long long g = 0;   // global stage counter
+  if (warp == 2) {
+    // ------------------------------------------------------------------ tile loader
+    if (lane == 0) tma_prefetch_desc(&map_q);
     for (int tc = 0;; ++tc) {
       const int qb = tc & 1;
       int slot = 0;
       bool ok = true;
       if (lane == 0) {
-        if (tc >= 2) ok = mbar_wait(&q_empty[qb], ((tc - 2) >> 1) & 1, status, kDevTimeoutQFull);
+        if (tc >= 2) {
+          const uint32_t par = ((tc - 2) >> 1) & 1;
+          ok = mbar_wait(&q_empty[qb], par, status, kDevTimeoutQFull) &&
+               mbar_wait(&o_free[qb], par, status, kDevTimeoutOBar);
+        }
         slot = ok ? atomicAdd(status + 1, 1) : prm.items;
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -185,7 +191,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long bh = item / prm.npairs;
       const int i0 = 2 * (item - static_cast<int>(bh) * prm.npairs);
       const bool has_i1 = i0 + 1 < nb;
-      // The two rows' bitmask words -> shared memory; count the union.
       uint32_t* u0 = sWords + (qb * 2) * kMaxWords;
       uint32_t* u1 = u0 + kMaxWords;
       const uint32_t* r0 = prm.bits + (bh * nb + i0) * static_cast<long long>(nw);
@@ -205,16 +210,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
       __syncwarp();
       if (lane == 0) {
-        const int steps = (cnt + 1) >> 1;
         qmeta[2 * qb] = item;
-        qmeta[2 * qb + 1] = steps;
+        qmeta[2 * qb + 1] = (cnt + 1) >> 1;
         mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
         const int qrow = static_cast<int>(bh * prm.S + static_cast<long long>(i0) * 64);
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_2d(sQ + qb * C::kQBytes + pn * 16384, &map_q, &q_full[qb], pn * 64, qrow);
+      }
+      __syncwarp();
+    }
+    __syncwarp();
+  } else if (warp == 0) {
+    // ------------------------------------------------------------------ K/V streamer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      long long g = 0;   // global stage counter
+      bool ok = true;
+      for (int tc = 0; ok; ++tc) {
+        const int qb = tc & 1;
+        if (!mbar_wait(&q_full[qb], (tc >> 1) & 1, status, kDevTimeoutQFull)) break;
+        const int item = qmeta[2 * qb];
+        const int steps = qmeta[2 * qb + 1];
+        if (item < 0) break;
+        const long long bh = item / prm.npairs;
         BitWalk wk;
-        wk.init(u0, u1, nw);
+        wk.init(sWords + (qb * 2) * kMaxWords, sWords + (qb * 2 + 1) * kMaxWords, nw);
         for (int k = 0; k < steps; ++k, ++g) {
           uint32_t fa = 0, fb = 0;
           const int ja = wk.next(&fa);
@@ -223,7 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = static_cast<int>(g % NST);
           const long long r = g / NST;
           if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, status, kDevTimeoutKvEmpty)) { ok = false; break; }
-          meta[s] = static_cast<uint32_t>(ja) | (fa << 14) | (static_cast<uint32_t>(jb) << 16) | (fb << 30);
           mbar_arrive_expect_tx(&full[s], C::kStageBytes);
           unsigned char* kp = sStage + s * C::kStageBytes;
           unsigned char* vp = kp + C::kPairBytes;
@@ -238,11 +259,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      g = __shfl_sync(0xffffffffu, g, 0);
-      if (!ok) break;
-    }
-    if (lane == 0) {
       // Drain: copies still in flight must land before the CTA exits.
       for (long long x = g > NST ? g - NST : 0; x < g; ++x)
         mbar_wait(&full[x % NST], (x / NST) & 1, status, kDevTimeoutDrain);
@@ -289,8 +305,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               issue_s(qb, g1, (k + 1) & 1);
             }
-            if (k == 0 && tc > 0 &&
-                !mbar_wait(o_free, (tc - 1) & 1, status, kDevTimeoutOBar)) { ok = false; break; }
+            if (k == 0 && tc > 0) {
+              // The accumulators hold an earlier tile until its epilogue frees them; the
+              // epilogue retires tiles in order, so waiting for the previous tile suffices
+              // (its buffer set's previous use was retired before this tile was loaded).
+              const int pb = (tc - 1) & 1;
+              if (!mbar_wait(&o_free[pb], ((tc - 1) >> 1) & 1, status, kDevTimeoutOBar)) { ok = false; break; }
+              tc_fence_after();
+            }
             const int b = k & 1;
             if (!mbar_wait(&p_full[b], pcount[b] & 1, status, kDevTimeoutPFull)) { ok = false; break; }
             ++pcount[b];
@@ -311,17 +333,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           g += n;
-        } else if (tc > 0) {
-          if (!mbar_wait(o_free, (tc - 1) & 1, status, kDevTimeoutOBar)) break;
         }
         mma_commit(&q_empty[qb]);
-        mma_commit(tile_done);
+        mma_commit(&tile_done[qb]);
       }
       mma_commit(drain);
       mbar_wait(drain, 0, status, kDevTimeoutDrain);
     }
     __syncwarp();
-  } else if (warp >= kSoftmaxWarp0) {
+  } else if (warp >= kSoftmaxWarp0 && warp < kEpilogueWarp0) {
     // ------------------------------------------------------------------ softmax groups
     const int grp = (warp - kSoftmaxWarp0) >> 2;                  // 0 or 1
     const int row = ((warp - kSoftmaxWarp0) & 3) * 32 + lane;      // 0..127 = TMEM lane
@@ -329,7 +349,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool upper = row >= 64;
     const float sl2 = prm.scale_log2;
     const uint32_t s_col = tmem + lane_base + (grp ? C::kColS1 : C::kColS0);
-    long long g = 0;
     int my_iter = 0;
     bool ok = true;
     for (int tc = 0; ok; ++tc) {
@@ -341,12 +360,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (item < 0) break;
       float m_ref = -INFINITY;
       float l = 0.f;
-      for (int k = grp; k < n; k += 2) {
-        const long long gk = g + k;
-        ok = __all_sync(0xffffffffu, mbar_wait(&full[gk % NST], (gk / NST) & 1, status, kDevTimeoutTmaFull));
-        if (!ok) break;
-        const uint32_t mt = meta[gk % NST];
-        const uint32_t fa = (mt >> 14) & 3u, fb = (mt >> 30) & 3u;
+      // The step's key blocks and flags come from the tile's bitmask words (stable in
+      // shared memory for the whole tile), walked the same way as the K/V streamer does;
+      // the group then waits only on its own score buffer, never on a K/V stage whose
+      // previous phase it has not observed.
+      BitWalk wk;
+      wk.init(sWords + (qb * 2) * kMaxWords, sWords + (qb * 2 + 1) * kMaxWords, nw);
+      for (int k = 0; k < n; ++k) {
+        uint32_t fa = 0, fb = 0;
+        wk.next(&fa);
+        if (wk.next(&fb) < 0) fb = 0;
+        if ((k & 1) != grp) continue;
         const bool keep_a = upper ? (fa >> 1) : (fa & 1u);
         const bool keep_b = upper ? (fb >> 1) : (fb & 1u);
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[grp], my_iter & 1, status, kDevTimeoutSFull));
@@ -438,17 +462,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&p_full[grp]);
       }
       if (!ok) break;
-      // ---- tile epilogue: merge the two groups' partial results ---------------------------
-      ok = __all_sync(0xffffffffu, mbar_wait(tile_done, tc & 1, status, kDevTimeoutOBar));
+      // Hand the running (max, sum) to the epilogue and move on to the next tile.
+      ml[(qb * 2 + grp) * 128 + row] = m_ref;
+      ml[512 + (qb * 2 + grp) * 128 + row] = l;
+      mbar_arrive(&ml_ready[qb]);
+    }
+  } else if (warp >= kEpilogueWarp0) {
+    // ------------------------------------------------------------------ epilogue group
+    const int row = (warp - kEpilogueWarp0) * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>((warp - kEpilogueWarp0) * 32) << 16;
+    const bool upper = row >= 64;
+    bool ok = true;
+    for (int tc = 0; ok; ++tc) {
+      const int qb = tc & 1;
+      const uint32_t par = (tc >> 1) & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qb], par, status, kDevTimeoutQFull));
+      if (!ok) break;
+      const int item = qmeta[2 * qb];
+      const int n = qmeta[2 * qb + 1];
+      if (item < 0) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(&tile_done[qb], par, status, kDevTimeoutOBar) &&
+                                       mbar_wait(&ml_ready[qb], par, status, kDevTimeoutOBar));
       if (!ok) break;
       tc_fence_after();
-      float* m_sh = ml + (qb * 2) * 128;           // [group][row] for this tile parity
-      float* l_sh = ml + 512 + (qb * 2) * 128;
-      m_sh[grp * 128 + row] = m_ref;
-      l_sh[grp * 128 + row] = l;
-      named_barrier_sync(1, 256);
-      const float m0 = m_sh[row], m1 = m_sh[128 + row];
-      const float l0 = l_sh[row], l1 = l_sh[128 + row];
+      const float m0 = ml[(qb * 2) * 128 + row], m1 = ml[(qb * 2 + 1) * 128 + row];
+      const float l0 = ml[512 + (qb * 2) * 128 + row], l1 = ml[512 + (qb * 2 + 1) * 128 + row];
       const float M = fmaxf(m0, m1);
       const float f0 = l0 > 0.f ? fast_exp2(m0 - M) : 0.f;
       const float f1 = l1 > 0.f ? fast_exp2(m1 - M) : 0.f;
@@ -462,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long tok = bh * prm.S + static_cast<long long>(i0) * 64 + row;
       const uint32_t o0 = tmem + lane_base + C::kColO0, o1 = tmem + lane_base + C::kColO1;
 #pragma unroll 1
-      for (int c0 = grp * (D / 2); c0 < (grp + 1) * (D / 2); c0 += 32) {
+      for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t a0[32], a1[32];
         if (has0) tmem_ld32(o0 + c0, a0);
         if (has1) tmem_ld32(o1 + c0, a1);
@@ -485,11 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (grp == 0 && valid_row && prm.lse != nullptr)
+      if (valid_row && prm.lse != nullptr)
         prm.lse[tok] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
-      mbar_arrive(o_free);
-      g += n;
+      mbar_arrive(&o_free[qb]);
     }
   }
   // ------------------------------------------------------------------ teardown

@@ -76,6 +76,10 @@ WORKLOADS = {
                         sigma=(1.0, 6.0), seed=1002),
     "wan720p_sta": Workload("wan720p_sta", B=1, H=40, T=21, Hg=48, W=80, D=128,
                             thrs=(0.7,), window=(3, 3, 5), sigma=(1.0, 6.0), seed=1002),
+    # heads 0-7 of the 720p-like workload (identical draws: streams are seeded per head),
+    # a smaller case for profiler captures
+    "wan720p_h8": Workload("wan720p_h8", B=1, H=8, T=21, Hg=48, W=80, D=128, thrs=(0.8,),
+                           sigma=(1.0, 6.0), seed=1002),
     "train_mid": Workload("train_mid", B=2, H=24, T=11, Hg=32, W=56, D=128, thrs=(0.8,),
                           window=(3, 3, 3), sigma=(2.0, 2.0), backward=True, seed=1004),
 }

@@ -36,6 +36,15 @@ def _head(t, b, h, wl, reorder=False):
 def test_fullsize_mask_and_forward(name):
     wl, path = _run(name)
     thr = path.thr
+    # every output is computed in a fixed order: a second run is bitwise identical
+    o1, bits1 = path.o.clone(), path.bits.clone()
+    path.step()
+    torch.cuda.synchronize()
+    path.check_status()
+    assert torch.equal(path.bits, bits1), "mask differs between two runs"
+    assert torch.equal(path.o.view(torch.int16) if path.o.dtype == torch.bfloat16 else path.o, 
+                       o1.view(torch.int16) if o1.dtype == torch.bfloat16 else o1), \
+        "forward output differs between two runs"
     gm = bits_to_mask(path.bits, wl.nb)
     check_lists(path.ridx, path.rcnt, gm)
     mism = amb = 0
