@@ -8,17 +8,18 @@
 // final mask is the union with a static window mask.  lsdiaocha.cn article, section 4:
 // sort each row and accumulate the probability.
 //
-// Decision precision: the whole decision is taken in fp64 (pooled means, logits,
-// softmax, ranked mass), so it agrees with an fp64 statement of the method except for
-// blocks whose ranked mass lies within rounding (~1e-15) of thr.
+// Decision precision: this kernel takes the whole decision in fp64 (pooled means,
+// logits, softmax, ranked mass), so it agrees with an fp64 statement of the method
+// except for blocks whose ranked mass lies within rounding (~1e-15) of thr.  It serves
+// as the exact tier: for every row when the fast tier does not apply, and for the rows
+// the fast tier could not certify.
 //
 // Selection without a sort: block j is kept iff E_j < thr, where E_j is the mass ranked
 // strictly before j (probability descending, ties by lower index).  The kept set is a
-// prefix of that ranking, so it is found by a most-significant-digit radix select over
-// the fp64 bit patterns of the probabilities (non-negative doubles order like their bit
-// patterns), carrying per-digit counts and masses.  Masses are accumulated as 2^-62
-// fixed-point integers so the result does not depend on the order of the shared-memory
-// atomics (deterministic), with an error below 1e-15 per row.
+// prefix of that ranking, so it is found by bisecting over the fp64 bit patterns of the
+// probabilities (non-negative doubles order like their bit patterns) for the largest key
+// whose "mass at or above" still reaches thr; ties at that key are resolved by index.
+// The logits are computed with fp64 tensor-core MMA (m8n8k4).
 #include <math.h>
 
 #include "common.cuh"
@@ -38,10 +39,7 @@ namespace {
 constexpr int kThreads = 256;   // 8 warps; one pooled row per warp during selection
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
-constexpr double kFix = 4611686018427387904.0;  // 2^62
 constexpr int kRescueCtasPerHead = 16;
-
-__device__ __forceinline__ unsigned long long to_fix(double p) { return __double2ull_rn(p * kFix); }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
@@ -53,9 +51,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
   // rows rlist[bh*nb + ...], taken R at a time by the CTAs of the head in turn.
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int rows_s[8];
-  unsigned long long* hmass = reinterpret_cast<unsigned long long*>(smem_raw);  // 8 x 256
-  uint32_t* hcnt = reinterpret_cast<uint32_t*>(hmass + kWarps * 256);           // 8 x 256
-  double* qs = reinterpret_cast<double*>(hcnt + kWarps * 256);                  // 8 x D
+  double* qs = reinterpret_cast<double*>(smem_raw);                             // 8 x D
   double* prow = qs + 8 * D;                                                    // R x nb
 
   const int tid = threadIdx.x;
@@ -113,11 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
   }
   __syncthreads();
 
-  const unsigned long long T = to_fix(thr);
   const bool keep_all = thr >= 1.0;
   const bool keep_none = thr <= 0.0;
-  unsigned long long* mass = hmass + warp * 256;
-  uint32_t* cnt = hcnt + warp * 256;
   const uint32_t lt_mask = (1u << lane) - 1u;
 
   for (int r = warp; r < nrows; r += kWarps) {
@@ -139,82 +132,49 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
     for (int j = lane; j < nb; j += 32) row[j] = row[j] / ssum;
     __syncwarp();
 
-    // ---- radix select of the threshold key ---------------------------------------------
+    // ---- the cut: bisection over the fp64 bit patterns ----------------------------------
+    // Non-negative doubles order like their bit patterns.  kstar = the largest key k with
+    // mass(P >= k) >= thr: blocks with a larger key are kept, blocks with a smaller key
+    // dropped, and among blocks whose key equals kstar (ties) the first `tie_keep` by
+    // index.  Masses are summed per lane in index order, then by a fixed butterfly:
+    // deterministic, fp64-accurate.
     // mode 0: keep key >= kstar.  mode 1: keep key > kstar, plus the first `tie_keep`
     // blocks (by index) whose key == kstar.
     unsigned long long kstar = 0;
     int mode = 0;
     int tie_keep = 0;
     if (!keep_all && !keep_none) {
-      unsigned long long prefix = 0, pmask = 0, above = 0;
-      int shift = 56;
-      while (true) {
-        for (int k = lane; k < 256; k += 32) { cnt[k] = 0; mass[k] = 0ull; }
-        __syncwarp();
+      auto mass_ge = [&](unsigned long long kk) {
+        double acc = 0.0;
         for (int j = lane; j < nb; j += 32) {
-          const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(row[j]));
-          if ((key & pmask) == prefix) {
-            const int dg = static_cast<int>((key >> shift) & 255ull);
-            atomicAdd(&cnt[dg], 1u);
-            atomicAdd(&mass[dg], to_fix(row[j]));
-          }
+          const double pj = row[j];
+          if (static_cast<unsigned long long>(__double_as_longlong(pj)) >= kk) acc += pj;
         }
-        __syncwarp();
-        // lane l owns digits 255-8l .. 248-8l (descending)
-        unsigned long long msum = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) msum += mass[255 - 8 * lane - q];
-        unsigned long long incl = msum;
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        return acc;
+      };
+      if (mass_ge(0ull) >= thr) {
+        unsigned long long lo = 0ull, hi = 0x3FF0000000000001ull;   // just above 1.0
+        while (hi - lo > 1ull) {
+          const unsigned long long mid = lo + ((hi - lo) >> 1);
+          if (mass_ge(mid) >= thr) lo = mid; else hi = mid;
+        }
+        kstar = lo;
+        int n_at = 0;
+        for (int j = lane; j < nb; j += 32)
+          n_at += static_cast<unsigned long long>(__double_as_longlong(row[j])) == kstar;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        unsigned long long Bq = above + incl - msum;
-        int found = -1;
-        unsigned long long fB = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int dg = 255 - 8 * lane - q;
-          const unsigned long long mm = mass[dg];
-          if (found < 0 && Bq < T && T <= Bq + mm) { found = dg; fB = Bq; }
-          Bq += mm;
-        }
-        const uint32_t fb = __ballot_sync(0xffffffffu, found >= 0);
-        if (fb == 0) {  // the whole prefix range holds < thr: keep all of it
-          kstar = prefix;
-          mode = 0;
-          break;
-        }
-        const int src = __ffs(fb) - 1;
-        const int dg = __shfl_sync(0xffffffffu, found, src);
-        above = __shfl_sync(0xffffffffu, fB, src);
-        const uint32_t c = cnt[dg];
-        prefix |= static_cast<unsigned long long>(dg) << shift;
-        pmask |= 255ull << shift;
-        __syncwarp();
-        if (c == 1) {  // the crossing block is unique: keep every key >= its key
-          unsigned long long mine = 0;
-          for (int j = lane; j < nb; j += 32) {
-            const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(row[j]));
-            if ((key & pmask) == prefix) mine = key;
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mine |= __shfl_xor_sync(0xffffffffu, mine, o);
-          kstar = mine;
-          mode = 0;
-          break;
-        }
-        if (shift == 0) {  // c > 1 blocks with identical probability straddle thr
-          kstar = prefix;
+        for (int o = 16; o > 0; o >>= 1) n_at += __shfl_xor_sync(0xffffffffu, n_at, o);
+        if (n_at > 1) {
+          // ties at the cut: the r-th (by index) has ranked mass e_above + r * p
+          const double e_above = mass_ge(kstar + 1ull);
+          const double pt = __longlong_as_double(static_cast<long long>(kstar));
+          int r = 0;
+          while (r < n_at && e_above + r * pt < thr) ++r;
           mode = 1;
-          const unsigned long long f = to_fix(__longlong_as_double(static_cast<long long>(prefix)));
-          const unsigned long long room = T - above;   // > 0
-          unsigned long long need = (f == 0ull) ? c : (room + f - 1ull) / f;
-          tie_keep = static_cast<int>(need < c ? need : c);
-          break;
+          tie_keep = r;
         }
-        shift -= 8;
       }
     }
 
@@ -317,8 +277,7 @@ int rows_per_cta(int nb) {
 }
 
 size_t mask_rows_smem(int nb, int D, int R) {
-  return static_cast<size_t>(kWarps) * 256 * (8 + 4) + static_cast<size_t>(8) * D * 8 +
-         static_cast<size_t>(R) * nb * 8;
+  return static_cast<size_t>(8) * D * 8 + static_cast<size_t>(R) * nb * 8;
 }
 
 template <int D>
