@@ -31,10 +31,12 @@ nabla_status check_shape(const nabla_shape& s, Dims* d);
 bool aligned16(const void* p);
 nabla_status cuda_status(cudaError_t e);
 
-// Longest-first tile order (schedule.cu): scratch size and builder.
+// Longest-first tile order (schedule.cu): scratch size and builder.  With `frame_pairs`
+// a tile's two query blocks are the ones of tile_blocks() (same patch, consecutive
+// frames); otherwise blocks 2p and 2p+1.
 size_t schedule_scratch_bytes(const Dims& d);
 cudaError_t build_schedule(const int32_t* cnt, const uint32_t* bits, const Dims& d, void* scratch,
-                           int32_t** order_out, cudaStream_t st);
+                           int32_t** order_out, cudaStream_t st, bool frame_pairs = false);
 
 // Device status codes (recorded in workspace word 0; first error wins).
 enum : uint32_t {
@@ -47,6 +49,7 @@ enum : uint32_t {
   kDevTimeoutQFull = 0x106,
   kDevTimeoutDrain = 0x107,
   kDevTimeoutBwd = 0x108,
+  kDevTimeoutMeta = 0x109,
   kDevFp16Range = 0x201,   // backward: an input exceeds the fp16 range (|x| > 65504)
 };
 
@@ -67,6 +70,23 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code) {
   if (status != nullptr) atomicCAS(status, 0u, code);
+}
+
+// The two query blocks of forward work tile p (0 <= p < ceil(nb / 2)) of one head.  The
+// block at patch s of frame 2u pairs with the block at the same patch of frame 2u + 1:
+// in the fractal order the pooled neighbourhoods of a patch and of its successor in time
+// overlap far more than those of two side-by-side patches, so the 128-row tile wastes
+// fewer masked half-tiles.  With T odd the last frame pairs neighbouring patches, and a
+// lone last block gets -1.  Every block lands in exactly one tile.
+__device__ __forceinline__ int2 tile_blocks(int p, int T, int HW, int nb) {
+  const int full = (T >> 1) * HW;
+  if (p < full) {
+    const int u = p / HW;
+    const int a = 2 * u * HW + (p - u * HW);
+    return make_int2(a, a + HW);
+  }
+  const int a = (T - 1) * HW + 2 * (p - full);
+  return make_int2(a, a + 1 < nb ? a + 1 : -1);
 }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
@@ -242,6 +262,41 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Ties registers written by tcgen05.ld to a point after tcgen05.wait::ld: the empty asm
+// redefines them, so no use can be scheduled between the load and the wait.
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+  reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+  reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute the same one).
+// The block's total at launch bounds what the increases can take.
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -347,6 +402,28 @@ __device__ __forceinline__ float poly_exp2(float x) {
   p = fmaf(p, f, 0.6958335638046265f);
   p = fmaf(p, f, 0.9999251961708069f);
   return __int_as_float(__float_as_int(p) + (static_cast<int>(j) << 23));
+}
+
+// 2^x for a pair of values on the FMA and integer pipes (relieves the special-function
+// unit): x = j + f with j = x rounded to the nearest integer by the 1.5 * 2^23 shifter
+// (its low mantissa bits then hold j), f in [-0.5, 0.5]; 2^f from a degree-3 polynomial
+// (minimax fit of the relative error on [-0.5, 0.5], max relative error 7.5e-5, far below
+// the 2^-11 rounding of the fp16 probabilities it feeds); j is added to the exponent
+// field as (shifter bits << 23), the shifter's own bits falling off the top.  Inputs below
+// -126 are clamped (result ~1e-38).
+__device__ __forceinline__ float2 poly_exp2x2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 shifter = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = __fadd2_rn(x, shifter);
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
+  float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                        make_float2(0.2426111251115799f, 0.2426111251115799f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 #endif  // __CUDACC__

@@ -1,4 +1,5 @@
-// Order of attention work items (tile = pair of consecutive blocks of one head).
+// Order of attention work items (tile = two query blocks of one head: blocks 2p and 2p+1,
+// or with frame pairs the two blocks of tile_blocks()).
 //
 // Heads are taken one after another (head-major), so the tiles running at the same time
 // read K and V of one head and those stay resident in L2; inside a head, tiles run
@@ -11,22 +12,28 @@
 namespace nabla {
 namespace {
 
-// Tile length: with `bits` the exact union size popc(row 2e | row 2e+1); otherwise the
-// sum of the two list counts.
+// Tile length: with `bits` the exact union size popc(row a | row b); otherwise the sum of
+// the two list counts.
 __global__ void __launch_bounds__(512) sched_head_sort_kernel(const int32_t* __restrict__ cnt,
                                                               const uint32_t* __restrict__ bits,
                                                               int nb, int nw, int npairs, int npow2,
+                                                              int T, int HW, int frame_pairs,
                                                               int32_t* __restrict__ order) {
   extern __shared__ unsigned long long keys[];
   const long long bh = blockIdx.x;
   for (int e = threadIdx.x; e < npow2; e += blockDim.x) {
     unsigned long long key = ~0ull;
     if (e < npairs) {
-      const int i0 = 2 * e;
+      int i0 = 2 * e, i1 = i0 + 1 < nb ? i0 + 1 : -1;
+      if (frame_pairs) {
+        const int2 ab = tile_blocks(e, T, HW, nb);
+        i0 = ab.x;
+        i1 = ab.y;
+      }
       int c = 0;
       if (bits != nullptr) {
         const uint32_t* r0 = bits + (bh * nb + i0) * static_cast<long long>(nw);
-        const uint32_t* r1 = (i0 + 1 < nb) ? r0 + nw : nullptr;
+        const uint32_t* r1 = i1 >= 0 ? bits + (bh * nb + i1) * static_cast<long long>(nw) : nullptr;
         for (int w = 0; w < nw; ++w) {
           uint32_t u = r0[w] | (r1 ? r1[w] : 0u);
           if (w == nw - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
@@ -34,7 +41,7 @@ __global__ void __launch_bounds__(512) sched_head_sort_kernel(const int32_t* __r
         }
       } else {
         c = min(max(cnt[bh * nb + i0], 0), nb);
-        if (i0 + 1 < nb) c += min(max(cnt[bh * nb + i0 + 1], 0), nb);
+        if (i1 >= 0) c += min(max(cnt[bh * nb + i1], 0), nb);
       }
       key = (static_cast<unsigned long long>(0x7FFFFFFF - c) << 32) | static_cast<unsigned>(e);
     }
@@ -77,7 +84,7 @@ size_t schedule_scratch_bytes(const Dims& d) {
 // Writes the item order to the start of `scratch`; returns it.  Tile lengths from the
 // bitmask when `bits` is given, else from the list counts `cnt`.
 cudaError_t build_schedule(const int32_t* cnt, const uint32_t* bits, const Dims& d, void* scratch,
-                           int32_t** order_out, cudaStream_t st) {
+                           int32_t** order_out, cudaStream_t st, bool frame_pairs) {
   const int npairs = (d.nb + 1) / 2;
   const int npow2 = next_pow2(npairs);
   int32_t* order = static_cast<int32_t*>(scratch);
@@ -85,7 +92,8 @@ cudaError_t build_schedule(const int32_t* cnt, const uint32_t* bits, const Dims&
   cudaError_t e = cudaFuncSetAttribute(sched_head_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  sched_head_sort_kernel<<<d.BH, 512, smem, st>>>(cnt, bits, d.nb, d.nw, npairs, npow2, order);
+  sched_head_sort_kernel<<<d.BH, 512, smem, st>>>(cnt, bits, d.nb, d.nw, npairs, npow2, d.T,
+                                                   d.Hb * d.Wb, frame_pairs ? 1 : 0, order);
   *order_out = order;
   return cudaGetLastError();
 }

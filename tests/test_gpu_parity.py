@@ -141,9 +141,16 @@ def test_fwd_dense_and_empty_rows(data):
     nb, nw = wl.nb, shape.nw
     rng = np.random.default_rng(5)
     cases = {"dense": np.ones((wl.B, wl.H, nb, nb), dtype=bool),
-             "holes": rng.random((wl.B, wl.H, nb, nb)) < 0.1}
-    cases["holes"][:, :, 3] = False       # an empty row whose partner row is not empty
-    cases["holes"][:, :, 10:12] = False   # an empty pair of rows
+             "holes": rng.random((wl.B, wl.H, nb, nb)) < 0.1,
+             "mostly_empty": rng.random((wl.B, wl.H, nb, nb)) < 0.2}
+    hw = (wl.Hg // wl.P) * (wl.W // wl.P)
+    cases["holes"][:, :, 3] = False       # an empty row whose partner rows are not empty
+    # empty rows whose work tiles are empty under either pairing of query blocks
+    # (neighbours 2p, 2p+1 and the same patch of consecutive frames)
+    for r in (10, 11, 10 + hw, 11 + hw):
+        cases["holes"][:, :, r] = False
+    # runs of empty tiles between non-empty ones: 80% of the rows keep nothing
+    cases["mostly_empty"][rng.random((wl.B, wl.H, nb)) < 0.8] = False
     for name, mask in cases.items():
         bits = torch.from_numpy(oracle.pack_mask_bits(mask).view(np.int32)).to(DEV)
         ridx = torch.empty(wl.B, wl.H, nb, nb, dtype=torch.int32, device=DEV)
@@ -161,8 +168,9 @@ def test_fwd_dense_and_empty_rows(data):
         check_close(to64(o), O, f"O {name}")
         check_lse(lse.cpu().numpy().astype(np.float64), L)
         if name == "holes":
-            assert torch.all(o[:, :, 3 * 64:4 * 64] == 0)
-            assert torch.all(torch.isneginf(lse[:, :, 10 * 64:12 * 64]))
+            for r in (3, 10, 11, 10 + hw, 11 + hw):
+                assert torch.all(o[:, :, r * 64:(r + 1) * 64] == 0)
+                assert torch.all(torch.isneginf(lse[:, :, r * 64:(r + 1) * 64]))
 
 
 @pytest.mark.parametrize("name,thr,window", [("tiny", 0.8, (0, 0, 0)), ("small", 0.8, (3, 3, 3)),
