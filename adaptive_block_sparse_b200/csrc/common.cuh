@@ -143,22 +143,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the completion of the phase with the given parity.  Gives up after
 // ~`kWaitLimitNs` of wall time, records `code` in the status word and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kWaitSuspendNs = 20000;           // 20 us per suspended probe
 
 // A wait also gives up early once any CTA of the launch has recorded a failure.
+// Suspending probe: the thread sleeps until the phase completes (it is woken then) or
+// about `kWaitSuspendNs` pass, instead of spinning on the issue slots that the warps doing
+// the math need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kWaitSuspendNs)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
                                           uint32_t code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 63u) == 0) {
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        record_status(status, code);
-        return false;
-      }
-      if (status != nullptr && *reinterpret_cast<volatile uint32_t*>(status) != 0u) return false;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      record_status(status, code);
+      return false;
     }
+    if (status != nullptr && *reinterpret_cast<volatile uint32_t*>(status) != 0u) return false;
   }
 }
 
@@ -175,6 +187,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // ------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Asks L2 to fetch `bytes` (a multiple of 16) at the 16-byte aligned global address `p`;
+// no completion to wait for.
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* map, uint64_t* bar,
