@@ -453,20 +453,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(s_col + 96, c3);
         }
         tmem_wait_ld();
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
         if (keep_a) {
           reg_fence32(c0);
           reg_fence32(c1);
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc) m4[cc & 3] = fmaxf(m4[cc & 3], __uint_as_float(sv[cc]));
+          for (int cc = 0; cc < 64; ++cc) m8[cc & 7] = fmaxf(m8[cc & 7], __uint_as_float(sv[cc]));
         }
         if (keep_b) {
           reg_fence32(c2);
           reg_fence32(c3);
 #pragma unroll
-          for (int cc = 64; cc < 128; ++cc) m4[cc & 3] = fmaxf(m4[cc & 3], __uint_as_float(sv[cc]));
+          for (int cc = 64; cc < 128; ++cc) m8[cc & 7] = fmaxf(m8[cc & 7], __uint_as_float(sv[cc]));
         }
-        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         float factor = 1.f;
         bool rescale = false;
         if (mx != -INFINITY && mx * sl2 > m_ref + 8.0f) {
@@ -493,12 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               // output is an exact convex combination of them.
               uint32_t pk;
               if constexpr (VF16) {
-                // Non-negative fp16 halves widened exactly with integer ops: the fp16
-                // bits moved to f32 bits 13..27 read as the value times 2^-112 (fp16
-                // subnormals land on f32 subnormals); the sum is rescaled once below.
                 pk = pack_f16x2(pr.x, pr.y);
-                acc = __fadd2_rn(acc, make_float2(__uint_as_float((pk << 13) & 0x0FFFE000u),
-                                                  __uint_as_float((pk >> 3) & 0x0FFFE000u)));
+                acc = __fadd2_rn(acc, make_float2(f16lo(pk), f16hi(pk)));
               } else {
                 pk = pack_bf16x2(pr.x, pr.y);
                 acc = __fadd2_rn(acc, make_float2(bf16lo(pk), bf16hi(pk)));
@@ -526,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(o_col + o0, ov);
           }
         }
-        l = l * factor + (acc.x + acc.y) * (VF16 ? 0x1p112f : 1.0f);
+        l = l * factor + (acc.x + acc.y);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&B.p_full);
