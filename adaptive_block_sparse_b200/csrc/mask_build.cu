@@ -17,9 +17,10 @@
 // Selection without a sort: block j is kept iff E_j < thr, where E_j is the mass ranked
 // strictly before j (probability descending, ties by lower index).  The kept set is a
 // prefix of that ranking, so it is found by bisecting over the fp64 bit patterns of the
-// probabilities (non-negative doubles order like their bit patterns) for the largest key
-// whose "mass at or above" still reaches thr; ties at that key are resolved by index.
-// The logits are computed with fp64 tensor-core MMA (m8n8k4).
+// probabilities (non-negative doubles order like their bit patterns) until the interval
+// of keys where the "mass at or above" crosses thr holds at most a few blocks; those are
+// ranked (probability descending, index ascending) and walked in order.  The logits are
+// computed with fp64 tensor-core MMA (m8n8k4), two key tiles per warp at a time.
 #include <math.h>
 
 #include "common.cuh"
@@ -39,7 +40,8 @@ namespace {
 constexpr int kThreads = 256;   // 8 warps; one pooled row per warp during selection
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
-constexpr int kRescueCtasPerHead = 16;
+constexpr int kRescueCtasPerHead = 64;
+constexpr int kCand = 16;       // the cut's bisection stops at this many candidates
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
@@ -51,6 +53,9 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
   // rows rlist[bh*nb + ...], taken R at a time by the CTAs of the head in turn.
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int rows_s[8];
+  __shared__ unsigned long long cand_key[kWarps * kCand];   // per warp: cut candidates
+  __shared__ int cand_idx[kWarps * kCand];
+  __shared__ int cand_keep[kWarps * kCand];
   double* qs = reinterpret_cast<double*>(smem_raw);                             // 8 x D
   double* prow = qs + 8 * D;                                                    // R x nb
 
@@ -89,21 +94,34 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
     double afrag[D / 4];
 #pragma unroll
     for (int kk = 0; kk < D / 4; ++kk) afrag[kk] = qs[gid * D + kk * 4 + tig];
-    for (int jt = warp; jt * 8 < nb; jt += kWarps) {
-      const int key = jt * 8 + gid;
+    // Two 8-key tiles per iteration: two independent accumulation chains, their key
+    // loads in flight together.
+    for (int jt = warp; jt * 8 < nb; jt += 2 * kWarps) {
+      const int jt2 = jt + kWarps;
+      const bool two = jt2 * 8 < nb;               // warp-uniform
+      const int key = jt * 8 + gid, key2 = jt2 * 8 + gid;
       const double* kr = kpool + (bh * nb + (key < nb ? key : 0)) * D + tig;
-      double c0 = 0.0, c1 = 0.0;
+      const double* kr2 = kpool + (bh * nb + (key2 < nb ? key2 : 0)) * D + tig;
+      double c0 = 0.0, c1 = 0.0, c2 = 0.0, c3 = 0.0;
 #pragma unroll
       for (int kk = 0; kk < D / 4; ++kk) {
         const double b = key < nb ? __ldg(kr + kk * 4) : 0.0;
+        const double b2 = (two && key2 < nb) ? __ldg(kr2 + kk * 4) : 0.0;
         asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
                      : "+d"(c0), "+d"(c1)
                      : "d"(afrag[kk]), "d"(b));
+        if (two)
+          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                       : "+d"(c2), "+d"(c3)
+                       : "d"(afrag[kk]), "d"(b2));
       }
-      const int key0 = jt * 8 + 2 * tig;
       if (gid < nrows) {
+        const int key0 = jt * 8 + 2 * tig;
         if (key0 < nb) prow[gid * nb + key0] = c0 * scale;
         if (key0 + 1 < nb) prow[gid * nb + key0 + 1] = c1 * scale;
+        const int key1 = jt2 * 8 + 2 * tig;
+        if (two && key1 < nb) prow[gid * nb + key1] = c2 * scale;
+        if (two && key1 + 1 < nb) prow[gid * nb + key1 + 1] = c3 * scale;
       }
     }
   }
@@ -132,47 +150,103 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
     for (int j = lane; j < nb; j += 32) row[j] = row[j] / ssum;
     __syncwarp();
 
-    // ---- the cut: bisection over the fp64 bit patterns ----------------------------------
-    // Non-negative doubles order like their bit patterns.  kstar = the largest key k with
-    // mass(P >= k) >= thr: blocks with a larger key are kept, blocks with a smaller key
-    // dropped, and among blocks whose key equals kstar (ties) the first `tie_keep` by
-    // index.  Masses are summed per lane in index order, then by a fixed butterfly:
-    // deterministic, fp64-accurate.
-    // mode 0: keep key >= kstar.  mode 1: keep key > kstar, plus the first `tie_keep`
-    // blocks (by index) whose key == kstar.
-    unsigned long long kstar = 0;
+    // ---- the cut: bisection over the fp64 bit patterns, then the last few candidates -----
+    // Non-negative doubles order like their bit patterns.  The keep rule (keep j iff the
+    // mass ranked strictly above it is < thr; rank by P descending, index ascending) keeps
+    // every block with key >= hi and drops every block with key < lo, for any lo < hi with
+    // mass(P >= lo) >= thr > mass(P >= hi).  The bisection narrows [lo, hi) until it holds
+    // at most kCand blocks (or a single key, all ties); those candidates are ranked and
+    // walked in order from mass(P >= hi).  Masses are summed per lane in index order, then
+    // by a fixed butterfly: deterministic, fp64-accurate.
+    // mode 0: keep all.  mode 1: candidates in [lo, hi) decided by cand_keep.  mode 2:
+    // [lo, hi) is the single key lo, the first `tie_keep` of its blocks (by index) kept.
+    unsigned long long klo = 0, khi = 0;
     int mode = 0;
     int tie_keep = 0;
+    int ncand = 0;
     if (!keep_all && !keep_none) {
-      auto mass_ge = [&](unsigned long long kk) {
+      auto mass_cnt_ge = [&](unsigned long long kk, int* cnt) {
         double acc = 0.0;
+        int c = 0;
         for (int j = lane; j < nb; j += 32) {
           const double pj = row[j];
-          if (static_cast<unsigned long long>(__double_as_longlong(pj)) >= kk) acc += pj;
+          if (static_cast<unsigned long long>(__double_as_longlong(pj)) >= kk) {
+            acc += pj;
+            ++c;
+          }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        *cnt = __reduce_add_sync(0xffffffffu, c);
         return acc;
       };
-      if (mass_ge(0ull) >= thr) {
+      int clo = 0, chi = 0;
+      if (mass_cnt_ge(0ull, &clo) >= thr) {
         unsigned long long lo = 0ull, hi = 0x3FF0000000000001ull;   // just above 1.0
-        while (hi - lo > 1ull) {
+        double mass_hi = 0.0;
+        while (clo - chi > kCand && hi - lo > 1ull) {
           const unsigned long long mid = lo + ((hi - lo) >> 1);
-          if (mass_ge(mid) >= thr) lo = mid; else hi = mid;
+          int cm = 0;
+          const double mm = mass_cnt_ge(mid, &cm);
+          if (mm >= thr) {
+            lo = mid;
+            clo = cm;
+          } else {
+            hi = mid;
+            chi = cm;
+            mass_hi = mm;
+          }
         }
-        kstar = lo;
-        int n_at = 0;
-        for (int j = lane; j < nb; j += 32)
-          n_at += static_cast<unsigned long long>(__double_as_longlong(row[j])) == kstar;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) n_at += __shfl_xor_sync(0xffffffffu, n_at, o);
-        if (n_at > 1) {
-          // ties at the cut: the r-th (by index) has ranked mass e_above + r * p
-          const double e_above = mass_ge(kstar + 1ull);
-          const double pt = __longlong_as_double(static_cast<long long>(kstar));
-          int r = 0;
-          while (r < n_at && e_above + r * pt < thr) ++r;
+        klo = lo;
+        khi = hi;
+        if (clo - chi <= kCand) {
+          // gather the candidates (index order), rank them, walk them
           mode = 1;
+          unsigned long long* ck = cand_key + warp * kCand;
+          int* ci = cand_idx + warp * kCand;
+          for (int j0 = 0; j0 < nb; j0 += 32) {
+            const int j = j0 + lane;
+            unsigned long long key = 0;
+            bool in = false;
+            if (j < nb) {
+              key = static_cast<unsigned long long>(__double_as_longlong(row[j]));
+              in = key >= lo && key < hi;
+            }
+            const uint32_t bal = __ballot_sync(0xffffffffu, in);
+            if (in) {
+              const int pos = ncand + __popc(bal & lt_mask);
+              ck[pos] = key;
+              ci[pos] = j;
+            }
+            ncand += __popc(bal);
+          }
+          __syncwarp();
+          // rank by (key descending, index ascending); E of a candidate = mass above hi +
+          // the candidates ranked before it
+          int* cr = cand_keep + warp * kCand;      // ranks first, then the decisions
+          int rank = 0;
+          if (lane < ncand) {
+            const unsigned long long kc = ck[lane];
+            const int ic = ci[lane];
+            for (int d = 0; d < ncand; ++d) rank += (ck[d] > kc || (ck[d] == kc && ci[d] < ic)) ? 1 : 0;
+            cr[lane] = rank;
+          }
+          __syncwarp();
+          double e = mass_hi;
+          if (lane < ncand)
+            for (int d = 0; d < ncand; ++d)
+              if (cr[d] < rank) e += __longlong_as_double(static_cast<long long>(ck[d]));
+          __syncwarp();
+          if (lane < ncand) cr[lane] = e < thr ? 1 : 0;
+          __syncwarp();
+        } else {
+          // a single key holding more than kCand blocks: ties, ranked by index; the r-th
+          // has ranked mass mass_hi + r * p
+          mode = 2;
+          const double pt = __longlong_as_double(static_cast<long long>(lo));
+          const int n_at = clo - chi;
+          int r = 0;
+          while (r < n_at && mass_hi + r * pt < thr) ++r;
           tie_keep = r;
         }
       }
@@ -192,8 +266,14 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
         const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(row[j]));
         if (keep_all) k = true;
         else if (keep_none) k = false;
-        else if (mode == 0) k = key >= kstar;
-        else { k = key > kstar; is_tie = key == kstar; }
+        else if (mode == 0) k = true;
+        else if (key >= khi) k = true;
+        else if (key < klo) k = false;
+        else if (mode == 2) is_tie = true;
+        else {
+          for (int d = 0; d < ncand; ++d)
+            if (cand_idx[warp * kCand + d] == j) k = cand_keep[warp * kCand + d] != 0;
+        }
       }
       const uint32_t tb = __ballot_sync(0xffffffffu, is_tie);
       if (is_tie) k = (tie_seen + __popc(tb & lt_mask)) < tie_keep;

@@ -20,6 +20,8 @@ DEV = "cuda"
 
 ODD = Workload("odd", B=1, H=3, T=1, Hg=24, W=8, D=128, thrs=(0.8,), sigma=(1.5, 1.5), seed=77)
 ODD64 = Workload("odd64", B=2, H=1, T=3, Hg=8, W=8, D=64, thrs=(0.6,), sigma=(1.0, 1.0), seed=78)
+# nb = 2176 > 2048: every row goes through the fp64 tier of the mask build
+WIDE = Workload("wide", B=1, H=1, T=4, Hg=256, W=136, D=64, thrs=(0.8,), sigma=(1.5, 1.5), seed=79)
 
 
 @pytest.fixture(scope="module")
@@ -61,11 +63,12 @@ def test_reorder_and_pool_bit_exact(data, name):
 
 MASK_CASES = [("tiny", 0.8, (0, 0, 0)), ("small", 0.5, (0, 0, 0)), ("small", 0.8, (0, 0, 0)),
               ("small", 0.95, (0, 0, 0)), ("small", 0.7, (1, 3, 3)), ("tiny", 1.0, (0, 0, 0)),
-              ("small", 0.0, (3, 1, 3)), ("odd", 0.8, (1, 1, 1)), ("odd64", 0.6, (0, 0, 0))]
+              ("small", 0.0, (3, 1, 3)), ("odd", 0.8, (1, 1, 1)), ("odd64", 0.6, (0, 0, 0)),
+              ("wide", 0.8, (0, 0, 0)), ("wide", 0.5, (1, 3, 3))]
 
 
 def _wl(name):
-    return {"odd": ODD, "odd64": ODD64}.get(name) or WORKLOADS[name]
+    return {"odd": ODD, "odd64": ODD64, "wide": WIDE}.get(name) or WORKLOADS[name]
 
 
 @pytest.mark.parametrize("name,thr,window", MASK_CASES)
