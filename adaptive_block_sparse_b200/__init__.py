@@ -273,11 +273,12 @@ def nabla_read_device_status(workspace, stream=None) -> int:
 # ---------------------------------------------------------------------------------------
 # Convenience: allocate outputs and run the whole path (mask -> forward [-> backward]).
 # ---------------------------------------------------------------------------------------
-def alloc_mask(shape: Shape, device, lists=True, cols=True):
+def alloc_mask(shape: Shape, device, lists=True, cols=True, counts=True):
+    """Mask outputs: bitmask, row lists (lists), row counts (lists or counts), column lists."""
     B, H, nb = shape.B, shape.H, shape.nb
     bits = torch.empty(B, H, nb, shape.nw, dtype=torch.int32, device=device)
     ridx = torch.empty(B, H, nb, nb, dtype=torch.int32, device=device) if lists else None
-    rcnt = torch.empty(B, H, nb, dtype=torch.int32, device=device) if lists else None
+    rcnt = torch.empty(B, H, nb, dtype=torch.int32, device=device) if (lists or counts) else None
     cidx = torch.empty(B, H, nb, nb, dtype=torch.int32, device=device) if cols else None
     ccnt = torch.empty(B, H, nb, dtype=torch.int32, device=device) if cols else None
     return bits, ridx, rcnt, cidx, ccnt

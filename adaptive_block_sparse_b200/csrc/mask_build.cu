@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(32) col_lists_kernel(const uint32_t* __restric
       const uint32_t b = __ballot_sync(0xffffffffu, set);
       const int base = __shfl_sync(0xffffffffu, mycnt, c);
       const int col = 32 * w + c;
-      if (set && col < nb) col_idx[(bh * nb + col) * nb + base + __popc(b & lt_mask)] = i;
+      if (set && col < nb && col_idx != nullptr) col_idx[(bh * nb + col) * nb + base + __popc(b & lt_mask)] = i;
       if (lane == c) mycnt += __popc(b);
     }
   }
@@ -343,7 +343,8 @@ __global__ void __launch_bounds__(256) row_lists_kernel(const uint32_t* __restri
     int pos = run + incl - c;
     while (word) {
       const int b = __ffs(word) - 1;
-      row_idx[row * nb + pos++] = 32 * w + b;
+      if (row_idx != nullptr) row_idx[row * nb + pos] = 32 * w + b;
+      ++pos;
       word &= word - 1u;
     }
     run += __shfl_sync(0xffffffffu, incl, 31);
@@ -380,9 +381,10 @@ cudaError_t launch_mask_rows(const double* qp, const double* kp, const Dims& d, 
   return cudaGetLastError();
 }
 
+// A list needs its counts; counts may come without the list.
 nabla_status check_lists(const int32_t* idx, const int32_t* cnt) {
-  if ((idx == nullptr) != (cnt == nullptr)) return NABLA_ERR_INVALID_ARG;
-  if (idx && ((reinterpret_cast<uintptr_t>(idx) & 3) || (reinterpret_cast<uintptr_t>(cnt) & 3)))
+  if (idx != nullptr && cnt == nullptr) return NABLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) & 3) || (reinterpret_cast<uintptr_t>(cnt) & 3))
     return NABLA_ERR_INVALID_ARG;
   return NABLA_OK;
 }
@@ -469,7 +471,7 @@ extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const dou
                 : launch_mask_rows<128>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt,
                                         rlist, rlist_cnt, st);
   if (e != cudaSuccess) return cuda_status(e);
-  if (col_idx) {
+  if (col_cnt) {
     if ((e = launch_col_lists(mask_bits, d, col_idx, col_cnt, st)) != cudaSuccess) return cuda_status(e);
   }
   return NABLA_OK;
@@ -486,13 +488,13 @@ extern "C" nabla_status nabla_mask_lists(const uint32_t* mask_bits, nabla_shape 
   if ((rc = check_lists(col_idx, col_cnt)) != NABLA_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaSuccess;
-  if (row_idx) {
+  if (row_cnt) {
     const long long rows = static_cast<long long>(d.BH) * d.nb;
     row_lists_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(mask_bits, d.nb, d.nw,
                                                                           rows, row_idx, row_cnt);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
   }
-  if (col_idx) {
+  if (col_cnt) {
     if ((e = launch_col_lists(mask_bits, d, col_idx, col_cnt, st)) != cudaSuccess) return cuda_status(e);
   }
   return NABLA_OK;

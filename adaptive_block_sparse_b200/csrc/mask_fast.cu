@@ -16,9 +16,11 @@
 //  2. pooled_logits_kernel: A = scale * (q_hi k_hi^T + (q_hi k_lo^T + q_lo k_hi^T)) with
 //     tcgen05 (M = 128, N = 256, K = 16 per instruction, fp32 accumulate in TMEM; the
 //     dominant q_hi k_hi^T term has its own accumulator), written to an fp32 scratch.
-//  3. mask_select_kernel: one warp per row: softmax in fp32, bisection over the fp32 bit
-//     patterns of the probabilities for the cut value P_c (the largest value whose mass
-//     at or above it reaches thr), then the certificate: with rho the proven relative
+//  3. mask_select_kernel: one warp per row: softmax in fp32; the cut value P_c (the
+//     smallest kept probability) by extracting maxima while the running mass is below
+//     thr (rows keeping a few blocks), else by bisection over the fp32 bit patterns until
+//     the interval where the mass at or above crosses thr holds at most 16 blocks, which
+//     are then ranked and walked; then the certificate: with rho the proven relative
 //     error of every P_j,
 //        thr - E_above > eta,  E_at_or_above - thr > eta,  P_c unique,
 //        P_c - P_next > 2 rho P_c,
@@ -42,6 +44,7 @@ namespace {
 // (3 x 2^-22), eight fp32 accumulations of the leading product (8 x 2^-22, allowing
 // truncating adds), the correction products and the final add / scale (~2^-22).
 constexpr float kLogitErr = 4.0e-6f;
+constexpr int kSelCand = 16;   // the cut's bisection stops at this many candidates
 
 // ------------------------------------------------------------------------------------
 // 1. fp16 split of the pooled means + norms
@@ -317,29 +320,104 @@ __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm
         kcut = __float_as_uint(best);
       }
     }
-    if (!found && mass_ge(0u) >= thr) {
-      // General path: bisection over the fp32 bit patterns for the largest key k with
-      // mass(P >= k) >= thr.
-      uint32_t lo = 0u, hi = 0x3F800001u;      // mass_ge(lo) >= thr > mass_ge(hi)
-      while (hi - lo > 1u) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (mass_ge(mid) >= thr) lo = mid; else hi = mid;
-      }
-      kcut = lo;
-      const float e_above = mass_ge(kcut + 1u);
-      const float e_at = mass_ge(kcut);
-      int n_at = 0;
-      float p_next = 0.f;
+    if (!found) {
+      // General path: bisection over the fp32 bit patterns until the interval [lo, hi)
+      // where the mass at or above crosses thr holds at most kSelCand blocks, then the
+      // candidates are ranked (value descending, index ascending) and walked from
+      // mass(P >= hi); the last kept candidate is the cut.
+      auto mass_cnt_ge = [&](uint32_t k, int* cnt) {
+        float acc = 0.f;
+        int c = 0;
 #pragma unroll
-      for (int t = 0; t < TPL; ++t) {
-        const uint32_t key = __float_as_uint(p[t]);
-        n_at += key == kcut;
-        if (key < kcut) p_next = fmaxf(p_next, p[t]);
-      }
+        for (int t = 0; t < TPL; ++t) {
+          const bool ge = __float_as_uint(p[t]) >= k;
+          acc += ge ? p[t] : 0.f;
+          c += ge ? 1 : 0;
+        }
+        *cnt = __reduce_add_sync(0xffffffffu, c);
+        return warp_sum(acc);
+      };
+      int clo = 0, chi = 0;
+      if (mass_cnt_ge(0u, &clo) >= thr) {
+        uint32_t lo = 0u, hi = 0x3F800001u;      // mass_ge(lo) >= thr > mass_ge(hi)
+        float mass_hi = 0.f;
+        while (clo - chi > kSelCand && hi - lo > 1u) {
+          const uint32_t mid = lo + ((hi - lo) >> 1);
+          int cm = 0;
+          const float mm = mass_cnt_ge(mid, &cm);
+          if (mm >= thr) {
+            lo = mid;
+            clo = cm;
+          } else {
+            hi = mid;
+            chi = cm;
+            mass_hi = mm;
+          }
+        }
+        if (clo - chi <= kSelCand) {
+          // gather the candidates in index order: candidate n goes to lane n (each lane
+          // holds the blocks lane + 32 t)
+          uint32_t ck = 0u;
+          int ci = 0x7FFFFFFF;
+          int ncand = 0;
+          float below = 0.f;                      // largest value below the interval
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) n_at += __shfl_xor_sync(0xffffffffu, n_at, o);
-      p_next = warp_max(p_next);
-      certified = certify(e_above, e_at, __uint_as_float(kcut), p_next, n_at);
+          for (int t = 0; t < TPL; ++t) {
+            const uint32_t key = __float_as_uint(p[t]);
+            const bool valid = lane + 32 * t < nb;
+            const bool in = valid && key >= lo && key < hi;
+            if (valid && key < lo) below = fmaxf(below, p[t]);
+            uint32_t bal = __ballot_sync(0xffffffffu, in);
+            while (bal != 0u) {                   // warp-uniform
+              const int src = __ffs(bal) - 1;
+              bal &= bal - 1u;
+              const uint32_t kv = __shfl_sync(0xffffffffu, key, src);
+              if (lane == ncand) {
+                ck = kv;
+                ci = src + 32 * t;
+              }
+              ++ncand;
+            }
+          }
+          below = warp_max(below);
+          // rank and exclusive mass of each candidate (lanes 0..ncand-1)
+          int rank = 0;
+          for (int d = 0; d < ncand; ++d) {
+            const uint32_t kd = __shfl_sync(0xffffffffu, ck, d);
+            const int id = __shfl_sync(0xffffffffu, ci, d);
+            rank += (lane < ncand && (kd > ck || (kd == ck && id < ci))) ? 1 : 0;
+          }
+          float e = mass_hi;
+          for (int d = 0; d < ncand; ++d) {
+            const int rd = __shfl_sync(0xffffffffu, rank, d);
+            const float pd = __uint_as_float(__shfl_sync(0xffffffffu, ck, d));
+            if (lane < ncand && rd < rank) e += pd;
+          }
+          // the cut: the candidate whose exclusive mass is below thr and inclusive mass
+          // reaches it
+          const float pc = __uint_as_float(ck);
+          const bool is_cut = lane < ncand && e < thr && e + pc >= thr;
+          const uint32_t cb = __ballot_sync(0xffffffffu, is_cut);
+          if (cb != 0u) {
+            const int cl = __ffs(cb) - 1;
+            const int crank = __shfl_sync(0xffffffffu, rank, cl);
+            const float e_above = __shfl_sync(0xffffffffu, e, cl);
+            const float p_cut = __uint_as_float(__shfl_sync(0xffffffffu, ck, cl));
+            // next value below the cut: the candidate ranked right after it, else the
+            // largest value below the interval
+            float p_next = below;
+            int n_at = 0;
+            for (int d = 0; d < ncand; ++d) {
+              const int rd = __shfl_sync(0xffffffffu, rank, d);
+              const float pd = __uint_as_float(__shfl_sync(0xffffffffu, ck, d));
+              if (rd == crank + 1) p_next = pd;
+              n_at += pd == p_cut ? 1 : 0;
+            }
+            kcut = __float_as_uint(p_cut);
+            certified = certify(e_above, e_above + p_cut, p_cut, p_next, n_at);
+          }
+        }
+      }
     }
   }
   if (!certified) {
@@ -353,6 +431,9 @@ __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm
   const int ti = i / (prm.Hb * prm.Wb), hi_ = (i / prm.Wb) % prm.Hb, wi = i % prm.Wb;
   const uint32_t lt_mask = (1u << lane) - 1u;
   int run = 0;
+  uint32_t word[(TPL + 31) / 32];                     // lane l keeps bitmask word l + 32 w
+#pragma unroll
+  for (int w = 0; w < (TPL + 31) / 32; ++w) word[w] = 0u;
 #pragma unroll
   for (int t = 0; t < TPL; ++t) {
     if (t >= prm.nw) break;
@@ -363,10 +444,15 @@ __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm
       k = k || (abs(ti - tj) <= prm.wt2 && abs(hi_ - hj) <= prm.wh2 && abs(wi - wj) <= prm.ww2);
     }
     const uint32_t kb = __ballot_sync(0xffffffffu, k);
-    if (lane == 0) prm.bits[(bh * nb + i) * prm.nw + t] = kb;
+    if (lane == (t & 31)) word[t >> 5] = kb;
     if (prm.row_idx != nullptr && k) prm.row_idx[(bh * nb + i) * static_cast<long long>(nb) + run + __popc(kb & lt_mask)] = j;
     run += __popc(kb);
   }
+  // the row's bitmask words in one coalesced store
+  uint32_t* brow = prm.bits + (bh * nb + i) * prm.nw;
+#pragma unroll
+  for (int w = 0; w < (TPL + 31) / 32; ++w)
+    if (lane + 32 * w < prm.nw) brow[lane + 32 * w] = word[w];
   if (prm.row_cnt != nullptr && lane == 0) prm.row_cnt[bh * nb + i] = run;
 }
 

@@ -191,8 +191,9 @@ class Path:
         self.vf = torch.empty(self.q.shape, dtype=torch.float16, device=dev)   # fp16 V operand
         self.qp = torch.empty(wl.B, wl.H, sh.nb, wl.D, dtype=torch.float64, device=dev)
         self.kp = torch.empty_like(self.qp)
+        # the forward reads the bitmask only; the lists serve the backward
         self.bits, self.ridx, self.rcnt, self.cidx, self.ccnt = m.alloc_mask(
-            sh, dev, cols=wl.backward)
+            sh, dev, lists=wl.backward, cols=wl.backward)
         self.mask_ws = torch.zeros(m.nabla_mask_workspace_bytes(sh), dtype=torch.uint8, device=dev)
         self.fwd_ws = torch.zeros(m.nabla_fwd_workspace_bytes(sh), dtype=torch.uint8, device=dev)
         self.o_dtype = m.NABLA_F32 if wl.backward else m.NABLA_BF16

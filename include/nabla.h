@@ -109,10 +109,11 @@ nabla_status nabla_reorder(const void *src, nabla_dtype src_dtype, void *dst,
  *              iff query block i attends to key block j.  Padding bits are 0.
  * row_idx    : out, nullable, int32 [B,H,nb,nb]: kept key blocks of row i ascending in
  *              row_idx[..,i,0:row_cnt[..,i]]; the rest is not written.
- * row_cnt    : out int32 [B,H,nb] (required iff row_idx is given).
+ * row_cnt    : out, nullable, int32 [B,H,nb]: kept blocks per row (required when row_idx
+ *              is given; may be given alone for the counts only).
  * col_idx,
  * col_cnt    : out, nullable: the transpose (query blocks that keep key block j,
- *              ascending), same shapes; used by the backward pass.
+ *              ascending), same shapes and the same rule; used by the backward pass.
  * workspace  : >= nabla_mask_workspace_bytes(s) bytes, 256-byte aligned.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  * --------------------------------------------------------------------------------- */

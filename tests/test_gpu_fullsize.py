@@ -46,7 +46,15 @@ def test_fullsize_mask_and_forward(name):
                        o1.view(torch.int16) if o1.dtype == torch.bfloat16 else o1), \
         "forward output differs between two runs"
     gm = bits_to_mask(path.bits, wl.nb)
-    check_lists(path.ridx, path.rcnt, gm)
+    # counts from the mask build; row lists rebuilt from the bitmask when the step did not
+    # ask for them (the forward reads only the bitmask)
+    ridx = path.ridx
+    if ridx is None:
+        ridx = torch.empty(wl.B, wl.H, wl.nb, wl.nb, dtype=torch.int32, device=path.bits.device)
+        rcnt2 = torch.empty_like(path.rcnt)
+        path.m.nabla_mask_lists(path.bits, path.shape, ridx, rcnt2)
+        assert torch.equal(rcnt2, path.rcnt)
+    check_lists(ridx, path.rcnt, gm)
     mism = amb = 0
     qn, kn = path.q.cpu(), path.k.cpu()
     for b in range(wl.B):
