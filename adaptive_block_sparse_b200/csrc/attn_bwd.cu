@@ -66,34 +66,61 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
     __half* __restrict__ q16, __half* __restrict__ k16, __half* __restrict__ v16,
     __half* __restrict__ do16, float* __restrict__ delta, float* __restrict__ lse2,
     long long rows, uint32_t* status) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  // D / 8 lanes per row, 8 contiguous elements (16 bytes of a 16-bit tensor) per lane.
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  constexpr int E = D / 32;  // elements per lane (contiguous)
-  const long long base = row * D + lane * E;
+  const long long row = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kRowsPerWarp +
+                        lane / kLanesPerRow;
+  const bool active = row < rows;
+  const long long base = (active ? row : 0) * D + (lane % kLanesPerRow) * 8;
   float acc = 0.f;
   bool range_ok = true;
+  if (active) {
+    auto widen = [](uint4 u, float* f) {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const float g = __bfloat162float(dout[base + e]);
-    const float of = o_f32 ? static_cast<const float*>(o)[base + e]
-                           : __bfloat162float(static_cast<const __nv_bfloat16*>(o)[base + e]);
-    acc = fmaf(g, of, acc);
-    const float qv = __bfloat162float(q[base + e]);
-    const float kv = __bfloat162float(k[base + e]);
-    const float vv = v_f16 ? __half2float(static_cast<const __half*>(v)[base + e])
-                           : __bfloat162float(static_cast<const __nv_bfloat16*>(v)[base + e]);
-    range_ok = range_ok && fabsf(g) <= 65504.f && fabsf(qv) <= 65504.f && fabsf(kv) <= 65504.f &&
-               fabsf(vv) <= 65504.f;
-    do16[base + e] = __float2half_rn(g);
-    q16[base + e] = __float2half_rn(qv);
-    k16[base + e] = __float2half_rn(kv);
-    v16[base + e] = __float2half_rn(vv);
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    };
+    auto to_f16 = [&](const float* f) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        range_ok = range_ok && fabsf(f[2 * i]) <= 65504.f && fabsf(f[2 * i + 1]) <= 65504.f;
+        const __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      return make_uint4(w[0], w[1], w[2], w[3]);
+    };
+    float g[8], of[8], t[8];
+    widen(*reinterpret_cast<const uint4*>(dout + base), g);
+    if (o_f32) {
+      const float4 o0 = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + base);
+      const float4 o1 = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + base + 4);
+      of[0] = o0.x; of[1] = o0.y; of[2] = o0.z; of[3] = o0.w;
+      of[4] = o1.x; of[5] = o1.y; of[6] = o1.z; of[7] = o1.w;
+    } else {
+      widen(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + base), of);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc = fmaf(g[i], of[i], acc);
+    *reinterpret_cast<uint4*>(do16 + base) = to_f16(g);
+    widen(*reinterpret_cast<const uint4*>(q + base), t);
+    *reinterpret_cast<uint4*>(q16 + base) = to_f16(t);
+    widen(*reinterpret_cast<const uint4*>(k + base), t);
+    *reinterpret_cast<uint4*>(k16 + base) = to_f16(t);
+    if (!v_f16) {   // an fp16 V is used as it is
+      widen(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(v) + base), t);
+      *reinterpret_cast<uint4*>(v16 + base) = to_f16(t);
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (!__all_sync(0xffffffffu, range_ok) && lane == 0) record_status(status, kDevFp16Range);
-  if (lane == 0) {
+  if (active && lane % kLanesPerRow == 0) {
     delta[row] = acc;
     lse2[row] = lse[row] * kLog2e;
   }
@@ -724,7 +751,9 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   cudaError_t e = build_schedule(ccnt, nullptr, d, sched, &order_cols, st);
   if (e == cudaSuccess) e = build_schedule(rcnt, nullptr, d, sched + schedule_scratch_bytes(d), &order_rows, st);
   if (e != cudaSuccess) return e;
-  bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+  constexpr int kRowsPerCta = 8 * (256 / D);
+  if (v_f16) v16 = static_cast<__half*>(const_cast<void*>(v));   // used as it is
+  bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
       o, o_f32, static_cast<const __nv_bfloat16*>(dout), lse, static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), v, v_f16, q16, k16, v16,
       do16, delta, lse2, rows, status);
