@@ -135,16 +135,22 @@ class ClockSampler:
 # --------------------------------------------------------------------------------------
 # distributed plumbing
 # --------------------------------------------------------------------------------------
-def init_dist():
+def init_dist(backend=None):
+    """One process per GPU (torchrun environment).  NCCL on GPUs; gloo when there is no
+    GPU (the rank logic is exercised on the host).  Returns (world, rank, local rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        timeout = datetime.timedelta(seconds=300)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
     return world, rank, local
 
 
@@ -355,7 +361,7 @@ def run_reference(args, wl, world, rank):
     est = statistics.median(times)
     flops = 4.0 * 64 * 64 * wl.D * kept_all
     val = flops / est / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": 0,
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "H": wl.H,
