@@ -184,7 +184,7 @@ def nabla_build_mask(q, k, shape: Shape, thr: float, window=(0, 0, 0), scale=Non
                      mask_bits=None, row_idx=None, row_cnt=None, col_idx=None, col_cnt=None,
                      q_pool=None, k_pool=None, workspace=None, stream=None):
     """NABLA block mask.  Returns (mask_bits, row_idx, row_cnt, col_idx, col_cnt)."""
-    dev = (q if q is not None else q_pool).device
+    dev = next(t.device for t in (q, q_pool, mask_bits, workspace) if t is not None)
     BH = shape.B * shape.H
     if mask_bits is None:
         mask_bits = torch.empty(shape.B, shape.H, shape.nb, shape.nw, dtype=torch.int32, device=dev)

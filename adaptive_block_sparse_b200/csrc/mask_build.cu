@@ -320,6 +320,33 @@ __global__ void __launch_bounds__(32) col_lists_kernel(const uint32_t* __restric
   if (32 * w + lane < nb) col_cnt[bh * nb + 32 * w + lane] = mycnt;
 }
 
+// Masks that do not depend on the data: thr >= 1 keeps every block; thr <= 0 keeps none,
+// which leaves the static window alone ([ZH-TS] "hybrid integration with STA": the union
+// with an empty NABLA mask is the STA mask).  One warp per row, one ballot per word.
+__global__ void __launch_bounds__(256) static_mask_kernel(int nb, int nw, long long rows, int keep_all,
+                                                          int sta_on, int wt2, int wh2, int ww2,
+                                                          int Hb, int Wb, uint32_t* __restrict__ bits) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int i = static_cast<int>(row % nb);
+  const int ti = i / (Hb * Wb), hi = (i / Wb) % Hb, wi = i % Wb;
+  for (int w = 0; w < nw; ++w) {
+    const int j = 32 * w + lane;
+    bool k = false;
+    if (j < nb) {
+      if (keep_all) {
+        k = true;
+      } else if (sta_on) {
+        const int tj = j / (Hb * Wb), hj = (j / Wb) % Hb, wj = j % Wb;
+        k = abs(ti - tj) <= wt2 && abs(hi - hj) <= wh2 && abs(wi - wj) <= ww2;
+      }
+    }
+    const uint32_t kb = __ballot_sync(0xffffffffu, k);
+    if (lane == 0) bits[row * nw + w] = kb;
+  }
+}
+
 // Row lists from a bitmask: one warp per row.
 __global__ void __launch_bounds__(256) row_lists_kernel(const uint32_t* __restrict__ bits, int nb,
                                                         int nw, long long rows,
@@ -427,6 +454,25 @@ extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const dou
   if (!mask_bits || (reinterpret_cast<uintptr_t>(mask_bits) & 3)) return NABLA_ERR_INVALID_ARG;
   if ((rc = check_lists(row_idx, row_cnt)) != NABLA_OK) return rc;
   if ((rc = check_lists(col_idx, col_cnt)) != NABLA_OK) return rc;
+  const bool data_free = thr <= 0.0 || thr >= 1.0;   // the mask ignores Q and K
+  if (data_free) {
+    const size_t need0 = nabla_mask_workspace_bytes(s);
+    if (!workspace || workspace_bytes < need0 || (reinterpret_cast<uintptr_t>(workspace) & 255))
+      return NABLA_ERR_WORKSPACE;
+    cudaStream_t st0 = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kStatusBytes, st0) != cudaSuccess) return NABLA_ERR_CUDA;
+    const long long rows = static_cast<long long>(d.BH) * d.nb;
+    static_mask_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st0>>>(
+        d.nb, d.nw, rows, thr >= 1.0 ? 1 : 0, sta_off ? 0 : 1, sta.t / 2, sta.h / 2, sta.w / 2,
+        d.Hb, d.Wb, mask_bits);
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 == cudaSuccess && row_cnt)
+      row_lists_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st0>>>(mask_bits, d.nb, d.nw,
+                                                                              rows, row_idx, row_cnt);
+    if (e0 == cudaSuccess) e0 = cudaGetLastError();
+    if (e0 == cudaSuccess && col_cnt) e0 = launch_col_lists(mask_bits, d, col_idx, col_cnt, st0);
+    return cuda_status(e0);
+  }
   if (!q_pool && (!q || !aligned16(q))) return NABLA_ERR_INVALID_ARG;
   if (!k_pool && (!k || !aligned16(k))) return NABLA_ERR_INVALID_ARG;
   if ((q_pool && (reinterpret_cast<uintptr_t>(q_pool) & 7)) ||

@@ -103,7 +103,9 @@ nabla_status nabla_reorder(const void *src, nabla_dtype src_dtype, void *dst,
  * q_pool,
  * k_pool     : nullable fp64 [B,H,nb,D] block means from nabla_reorder; when given, the
  *              call reads them instead of q / k (q / k may then be NULL).
- * thr        : in [0, 1]; scale > 0 (usually 1/sqrt(D)).
+ * thr        : in [0, 1]; scale > 0 (usually 1/sqrt(D)).  thr >= 1 keeps every block
+ *              and thr <= 0 keeps none but the static window (pure STA); neither depends
+ *              on the data, and q, k, q_pool and k_pool may then all be NULL.
  * sta        : window, {0,0,0} = off; each size must be 0 (all off) or odd >= 1.
  * mask_bits  : out uint32 [B,H,nb,ceil(nb/32)]; bit (j%32) of word j/32 of row i is 1
  *              iff query block i attends to key block j.  Padding bits are 0.

@@ -71,6 +71,24 @@ def _wl(name):
     return {"odd": ODD, "odd64": ODD64, "wide": WIDE}.get(name) or WORKLOADS[name]
 
 
+def test_mask_without_data():
+    """thr <= 0 (pure STA) and thr >= 1 (keep all) need neither Q, K nor pooled means."""
+    m = nbl()
+    wl = WORKLOADS["small"]
+    shape = shape_of(wl)
+    bits = torch.empty(wl.B, wl.H, wl.nb, shape.nw, dtype=torch.int32, device=DEV)
+    rcnt = torch.empty(wl.B, wl.H, wl.nb, dtype=torch.int32, device=DEV)
+    for thr, window in ((0.0, (3, 1, 3)), (0.0, (0, 0, 0)), (1.0, (0, 0, 0)), (1.0, (1, 1, 1))):
+        m.nabla_build_mask(None, None, shape, thr, window, mask_bits=bits, row_cnt=rcnt)
+        torch.cuda.synchronize()
+        gm = bits_to_mask(bits, wl.nb)
+        sta = oracle.sta_mask(wl.T, wl.Hg // wl.P, wl.W // wl.P, window) if window != (0, 0, 0) \
+            else np.zeros((wl.nb, wl.nb), dtype=bool)
+        want = np.ones_like(sta) if thr >= 1.0 else sta
+        assert np.array_equal(gm, np.broadcast_to(want, gm.shape)), (thr, window)
+        assert np.array_equal(rcnt.cpu().numpy(), gm.sum(-1))
+
+
 @pytest.mark.parametrize("name,thr,window", MASK_CASES)
 def test_mask_parity(data, name, thr, window):
     wl = _wl(name)
