@@ -35,6 +35,8 @@ NABLA_ERR_DEVICE_CHECK = 5
 NABLA_BF16 = 0
 NABLA_F32 = 1
 NABLA_F16 = 2
+NABLA_LAYOUT_REORDERED = 0
+NABLA_LAYOUT_NATURAL = 1
 
 EXPORTED = (
     "nabla_status_string", "nabla_reorder", "nabla_mask_workspace_bytes", "nabla_build_mask",
@@ -65,14 +67,15 @@ _sigs = {
     "nabla_mask_lists": (ctypes.c_int, [_vp, _Shape, _vp, _vp, _vp, _vp, _vp]),
     "nabla_fwd_workspace_bytes": (_sz, [_Shape]),
     "nabla_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape, ctypes.c_float,
-                                      _vp, ctypes.c_int, _vp, _vp, _sz, _vp]),
+                                      _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _sz, _vp]),
     "nabla_bwd_workspace_bytes": (_sz, [_Shape]),
     "nabla_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp,
                                       _vp, _vp, _vp, _Shape, ctypes.c_float, _vp, _vp, _vp, _vp,
                                       _sz, _vp]),
     "nabla_read_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
     "nabla_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape,
-                                              ctypes.c_float, _vp, ctypes.c_int, _vp, _vp]),
+                                              ctypes.c_float, _vp, ctypes.c_int, _vp, ctypes.c_int,
+                                              _vp]),
 }
 
 
@@ -161,8 +164,10 @@ def nabla_reorder(src, dst, shape: Shape, inverse=False, pool_out=None, stream=N
     """Natural <-> reordered token order ([B,H,S,D]); optional fp64 block means.
 
     Forward: bf16 ``src`` into a bf16 or fp16 ``dst``.  Inverse: same dtype both sides.
+    Forward with ``dst=None`` and ``pool_out``: the block means only.
     """
-    _check(load_library().nabla_reorder(_ptr(src), dtype_code(src), _ptr(dst), dtype_code(dst),
+    _check(load_library().nabla_reorder(_ptr(src), dtype_code(src), _ptr(dst),
+                                        dtype_code(dst) if dst is not None else NABLA_BF16,
                                         _ptr(pool_out), shape.c(), int(bool(inverse)),
                                         _stream(stream)), "nabla_reorder")
     return dst
@@ -209,8 +214,10 @@ def nabla_mask_lists(mask_bits, shape: Shape, row_idx=None, row_cnt=None, col_id
 
 
 def nabla_attn_fwd(q, k, v, mask_bits, shape: Shape, scale=None, o=None,
-                   o_dtype=NABLA_BF16, lse=None, workspace=None, stream=None):
-    """Block-sparse attention forward.  Returns (o, lse)."""
+                   o_dtype=NABLA_BF16, lse=None, workspace=None, stream=None,
+                   layout=NABLA_LAYOUT_REORDERED):
+    """Block-sparse attention forward.  Returns (o, lse).  ``layout``: token order of
+    q, k, v, o and lse (reordered, or the latent's natural order)."""
     if scale is None:
         scale = 1.0 / math.sqrt(shape.D)
     if o is None:
@@ -220,8 +227,8 @@ def nabla_attn_fwd(q, k, v, mask_bits, shape: Shape, scale=None, o=None,
         workspace = torch.zeros(nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=q.device)
     _check(load_library().nabla_attn_fwd(_ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(mask_bits),
                                shape.c(),
-                               float(scale), _ptr(o), int(o_dtype), _ptr(lse), _ptr(workspace),
-                               workspace.numel(), _stream(stream)), "nabla_attn_fwd")
+                               float(scale), _ptr(o), int(o_dtype), _ptr(lse), int(layout),
+                               _ptr(workspace), workspace.numel(), _stream(stream)), "nabla_attn_fwd")
     return o, lse
 
 
@@ -246,7 +253,7 @@ def nabla_attn_bwd(q, k, v, o, dout, lse, row_idx, row_cnt, col_idx, col_cnt, sh
 
 
 def nabla_attn_fwd_noalloc(q, k, v, mask_bits, shape: Shape, o, lse=None, scale=None,
-                           stream=None):
+                           stream=None, layout=NABLA_LAYOUT_REORDERED):
     """Forward without a caller workspace, for callers that cannot allocate device memory.
 
     Same results as :func:`nabla_attn_fwd`; the workspace is a fixed 1 MiB array inside
@@ -258,7 +265,8 @@ def nabla_attn_fwd_noalloc(q, k, v, mask_bits, shape: Shape, o, lse=None, scale=
         scale = 1.0 / math.sqrt(shape.D)
     _check(load_library().nabla_attn_fwd_noalloc(
         _ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(mask_bits), shape.c(),
-        float(scale), _ptr(o), dtype_code(o), _ptr(lse), _stream(stream)), "nabla_attn_fwd_noalloc")
+        float(scale), _ptr(o), dtype_code(o), _ptr(lse), int(layout), _stream(stream)),
+        "nabla_attn_fwd_noalloc")
     return o, lse
 
 

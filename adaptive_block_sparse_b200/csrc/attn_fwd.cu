@@ -73,6 +73,7 @@ struct FwdParams {
   uint32_t* status;          // word 0: status, word 1: work counter
   int nb;
   int T, HW;                 // frames, blocks per frame
+  int Hb, Wb, Hg, W;         // blocks per frame row / column; latent height and width
   long long S;
   float scale_log2;
   int o_f32;
@@ -147,7 +148,10 @@ struct SlotBars {
 //                 (meta_full), loads Q, K, V;
 //   warp 2 s + 1  MMA issuer of slot s (one lane);
 //   warps 4-7 (slot 0), 8-11 (slot 1): softmax and epilogue of the slot's tiles.
-template <int D, bool VF16>
+// NAT: q, k, v, o, lse in the latent's natural token order; a block (an 8 x 8 patch of a
+// frame) is then fetched with a 4-D copy (channels, patch columns, patch rows, frames of
+// the head) that lands in shared memory exactly as the 64 reordered rows would.
+template <int D, bool VF16, bool NAT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k,
@@ -217,6 +221,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t code) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
       };
+      // one 64-column panel of block blk of head bh: 64 rows of 128 bytes
+      auto load_block = [&](unsigned char* dst, const CUtensorMap* map, uint64_t* bar, int pn, int bh,
+                            int blk) {
+        if constexpr (NAT) {
+          const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+          tma_load_4d(dst, map, bar, pn * 64, wb * 8, hb * 8, bh * prm.T + tf);
+        } else {
+          tma_load_2d(dst, map, bar, pn * 64, static_cast<int>(bh * prm.S + static_cast<long long>(blk) * 64));
+        }
+      };
+      // the rows of block blk of head bh into L2 (contiguous in the reordered order; eight
+      // patch rows of 8 tokens in the natural one)
+      auto prefetch_block = [&](int bh, int blk) {
+        const char* qg = static_cast<const char*>(prm.q);
+        if constexpr (NAT) {
+          const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+#pragma unroll 1
+          for (int hh = 0; hh < 8; ++hh)
+            l2_prefetch(qg + ((static_cast<long long>(bh * prm.T + tf) * prm.Hg + hb * 8 + hh) * prm.W + wb * 8) * D * 2,
+                        8 * D * 2);
+        } else {
+          l2_prefetch(qg + (static_cast<long long>(bh) * prm.S + static_cast<long long>(blk) * 64) * D * 2, 64 * D * 2);
+        }
+      };
       // Takes the next work item for tile c of this slot and publishes its descriptor in
       // ring entry c % R.  Returns 1 (tile), 0 (end of the work: terminator published) or
       // -1 (error).
@@ -251,10 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
         if (lane == 0) {
           // the tile's Q rows into L2 ahead of their TMA copy
-          const char* qg = static_cast<const char*>(prm.q);
-          l2_prefetch(qg + (static_cast<long long>(bh) * prm.S + static_cast<long long>(ab.x) * 64) * D * 2, 64 * D * 2);
-          if (ab.y >= 0)
-            l2_prefetch(qg + (static_cast<long long>(bh) * prm.S + static_cast<long long>(ab.y) * 64) * D * 2, 64 * D * 2);
+          prefetch_block(bh, ab.x);
+          if (ab.y >= 0) prefetch_block(bh, ab.y);
           mt[0] = item;
           mt[1] = bh;
           mt[2] = ab.x;
@@ -284,12 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c > 0 && !wait_all(&B.q_empty, (c - 1) & 1, kDevTimeoutQFull)) { ok = false; break; }
         if (lane == 0) {
           mbar_arrive_expect_tx(&B.q_full, C::kTileBytes);
-          const int rowa = static_cast<int>(t.bh * prm.S + static_cast<long long>(t.ia) * 64);
-          const int rowb = static_cast<int>(t.bh * prm.S + static_cast<long long>(t.ib >= 0 ? t.ib : t.ia) * 64);
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn) {
-            tma_load_2d(sQ + pn * 16384, &map_q, &B.q_full, pn * 64, rowa);
-            tma_load_2d(sQ + pn * 16384 + 8192, &map_q, &B.q_full, pn * 64, rowb);
+            load_block(sQ + pn * 16384, &map_q, &B.q_full, pn, t.bh, t.ia);
+            load_block(sQ + pn * 16384 + 8192, &map_q, &B.q_full, pn, t.bh, t.ib >= 0 ? t.ib : t.ia);
           }
         }
         __syncwarp();
@@ -302,15 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ja = wk.next(&fa);
           int jb = wk.next(&fb);
           if (jb < 0) jb = ja;                      // odd tail: a masked duplicate
-          const int ra = static_cast<int>(t.bh * prm.S + static_cast<long long>(ja) * 64);
-          const int rb = static_cast<int>(t.bh * prm.S + static_cast<long long>(jb) * 64);
           if (gk > 0 && !wait_all(&B.k_empty, (gk - 1) & 1, kDevTimeoutKvEmpty)) { ok = false; break; }
           if (lane == 0) {
             mbar_arrive_expect_tx(&B.k_full, C::kTileBytes);
 #pragma unroll
             for (int pn = 0; pn < C::kPanels; ++pn) {
-              tma_load_2d(sK + pn * 16384, &map_k, &B.k_full, pn * 64, ra);
-              tma_load_2d(sK + pn * 16384 + 8192, &map_k, &B.k_full, pn * 64, rb);
+              load_block(sK + pn * 16384, &map_k, &B.k_full, pn, t.bh, ja);
+              load_block(sK + pn * 16384 + 8192, &map_k, &B.k_full, pn, t.bh, jb);
             }
           }
           __syncwarp();
@@ -320,8 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&B.v_full, C::kTileBytes);
 #pragma unroll
             for (int pn = 0; pn < C::kPanels; ++pn) {
-              tma_load_2d(sV + pn * 16384, &map_v, &B.v_full, pn * 64, ra);
-              tma_load_2d(sV + pn * 16384 + 8192, &map_v, &B.v_full, pn * 64, rb);
+              load_block(sV + pn * 16384, &map_v, &B.v_full, pn, t.bh, ja);
+              load_block(sV + pn * 16384 + 8192, &map_v, &B.v_full, pn, t.bh, jb);
             }
           }
           __syncwarp();
@@ -538,7 +560,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int blk = upper ? t.ib : t.ia;
       const bool valid_row = blk >= 0;
-      const long long tok = static_cast<long long>(t.bh) * prm.S + static_cast<long long>(valid_row ? blk : 0) * 64 + (row & 63);
+      long long tok;   // the row's token: reordered index, or natural (t, h, w) index
+      if constexpr (NAT) {
+        const int bb = valid_row ? blk : 0;
+        const int tf = bb / prm.HW, hb = (bb / prm.Wb) % prm.Hb, wb = bb % prm.Wb;
+        tok = static_cast<long long>(t.bh) * prm.S +
+              (static_cast<long long>(tf) * prm.Hg + hb * 8 + ((row & 63) >> 3)) * prm.W + wb * 8 + (row & 7);
+      } else {
+        tok = static_cast<long long>(t.bh) * prm.S + static_cast<long long>(valid_row ? blk : 0) * 64 + (row & 63);
+      }
 #pragma unroll 1
       for (int d0 = 0; d0 < D; d0 += 32) {
         uint32_t a0[32];
@@ -614,23 +644,50 @@ bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int 
   return r == CUDA_SUCCESS;
 }
 
+// 4-D map of 16-bit elements over a natural-order tensor viewed as [B*H*T, Hg, W, D]:
+// box = 64 channels x 8 columns x 8 rows x 1 frame (one P x P patch = one block),
+// 128-byte swizzle: the box lands as 64 rows of 128 bytes in the patch's row-major order,
+// the order of the reordered layout.
+bool make_map_nat(CUtensorMap* map, const void* base, long long frames, int Hg, int W, int D, bool fp16) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(W),
+                        static_cast<cuuint64_t>(Hg), static_cast<cuuint64_t>(frames)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(W) * D * 2,
+                           static_cast<cuuint64_t>(Hg) * W * D * 2};
+  cuuint32_t box[4] = {64u, 8u, 8u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
-template <int D, bool VF16>
+template <int D, bool VF16, bool NAT>
 cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& d,
                        const FwdParams& prm, cudaStream_t st, bool* map_ok, bool* regs_ok) {
   CUtensorMap mq, mk, mv;
   const long long rows = static_cast<long long>(d.BH) * d.S;
-  *map_ok = make_map_16(&mq, q, rows, D, 64, false) && make_map_16(&mk, k, rows, D, 64, false) &&
-            make_map_16(&mv, v, rows, D, 64, VF16);   // one 64-row block per copy
+  const long long frames = static_cast<long long>(d.BH) * d.T;
+  if constexpr (NAT) {
+    *map_ok = make_map_nat(&mq, q, frames, d.Hg, d.W, D, false) &&
+              make_map_nat(&mk, k, frames, d.Hg, d.W, D, false) &&
+              make_map_nat(&mv, v, frames, d.Hg, d.W, D, VF16);
+  } else {
+    *map_ok = make_map_16(&mq, q, rows, D, 64, false) && make_map_16(&mk, k, rows, D, 64, false) &&
+              make_map_16(&mv, v, rows, D, 64, VF16);   // one 64-row block per copy
+  }
   if (!*map_ok) return cudaErrorInvalidValue;
   using C = FwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, VF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, VF16, NAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
   // The warpgroups' register split assumes the block launches with kLaunchRegs registers
   // per thread; with fewer, the increases could never be granted.  Refuse to launch.
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, VF16>);
+  e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, VF16, NAT>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kLaunchRegs) {
     *regs_ok = false;
@@ -639,7 +696,7 @@ cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& 
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = prm.items < sms ? prm.items : sms;
-  attn_fwd_kernel<D, VF16><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, prm);
+  attn_fwd_kernel<D, VF16, NAT><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 }  // namespace
@@ -657,8 +714,8 @@ extern "C" size_t nabla_fwd_workspace_bytes(nabla_shape s) {
 extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void* v,
                                        nabla_dtype v_dtype, const uint32_t* mask_bits,
                                        nabla_shape s, float scale, void* o, nabla_dtype o_dtype,
-                                       float* lse, void* workspace, size_t workspace_bytes,
-                                       nabla_stream_t stream) {
+                                       float* lse, nabla_layout layout, void* workspace,
+                                       size_t workspace_bytes, nabla_stream_t stream) {
   Dims d;
   nabla_status rc = check_shape(s, &d);
   if (rc != NABLA_OK) return rc;
@@ -668,6 +725,7 @@ extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void*
     return NABLA_ERR_INVALID_ARG;
   if (o_dtype != NABLA_BF16 && o_dtype != NABLA_F32) return NABLA_ERR_INVALID_ARG;
   if (v_dtype != NABLA_BF16 && v_dtype != NABLA_F16) return NABLA_ERR_INVALID_ARG;
+  if (layout != NABLA_LAYOUT_REORDERED && layout != NABLA_LAYOUT_NATURAL) return NABLA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < nabla_fwd_workspace_bytes(s) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -684,6 +742,10 @@ extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void*
   prm.S = d.S;
   prm.T = d.T;
   prm.HW = d.Hb * d.Wb;
+  prm.Hb = d.Hb;
+  prm.Wb = d.Wb;
+  prm.Hg = d.Hg;
+  prm.W = d.W;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.o_f32 = o_dtype == NABLA_F32;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -698,10 +760,18 @@ extern "C" nabla_status nabla_attn_fwd(const void* q, const void* k, const void*
   prm.items = d.BH * prm.npairs;
   bool map_ok = true, regs_ok = true;
   const bool vf16 = v_dtype == NABLA_F16;
-  cudaError_t e = d.D == 64 ? (vf16 ? launch_fwd<64, true>(q, k, v, d, prm, st, &map_ok, &regs_ok)
-                                    : launch_fwd<64, false>(q, k, v, d, prm, st, &map_ok, &regs_ok))
-                            : (vf16 ? launch_fwd<128, true>(q, k, v, d, prm, st, &map_ok, &regs_ok)
-                                    : launch_fwd<128, false>(q, k, v, d, prm, st, &map_ok, &regs_ok));
+  const bool nat = layout == NABLA_LAYOUT_NATURAL;
+  cudaError_t e;
+  if (nat)
+    e = d.D == 64 ? (vf16 ? launch_fwd<64, true, true>(q, k, v, d, prm, st, &map_ok, &regs_ok)
+                          : launch_fwd<64, false, true>(q, k, v, d, prm, st, &map_ok, &regs_ok))
+                  : (vf16 ? launch_fwd<128, true, true>(q, k, v, d, prm, st, &map_ok, &regs_ok)
+                          : launch_fwd<128, false, true>(q, k, v, d, prm, st, &map_ok, &regs_ok));
+  else
+    e = d.D == 64 ? (vf16 ? launch_fwd<64, true, false>(q, k, v, d, prm, st, &map_ok, &regs_ok)
+                          : launch_fwd<64, false, false>(q, k, v, d, prm, st, &map_ok, &regs_ok))
+                  : (vf16 ? launch_fwd<128, true, false>(q, k, v, d, prm, st, &map_ok, &regs_ok)
+                          : launch_fwd<128, false, false>(q, k, v, d, prm, st, &map_ok, &regs_ok));
   if (!regs_ok) return NABLA_ERR_UNSUPPORTED;
   return cuda_status(e);
 }

@@ -49,7 +49,7 @@ extern "C" nabla_status nabla_attn_fwd_noalloc(const void* q, const void* k, con
                                                nabla_dtype v_dtype, const uint32_t* mask_bits,
                                                nabla_shape s, float scale, void* o,
                                                nabla_dtype o_dtype, float* lse,
-                                               nabla_stream_t stream) {
+                                               nabla_layout layout, nabla_stream_t stream) {
   nabla::Dims d;
   nabla_status rc = nabla::check_shape(s, &d);
   if (rc != NABLA_OK) return rc;
@@ -61,6 +61,6 @@ extern "C" nabla_status nabla_attn_fwd_noalloc(const void* q, const void* k, con
   if (rc != NABLA_OK) return rc;
   // The regular entry point clears the status word and the schedule histogram in the
   // scratch before its kernels run, so nothing left by an earlier call is read.
-  return nabla_attn_fwd(q, k, v, v_dtype, mask_bits, s, scale, o, o_dtype, lse, scratch,
+  return nabla_attn_fwd(q, k, v, v_dtype, mask_bits, s, scale, o, o_dtype, lse, layout, scratch,
                         kNoAllocScratchBytes, stream);
 }

@@ -96,6 +96,8 @@ cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims&
     return esz == 4 ? go<D, 4, false, true, true, false, false>(src, dst, nullptr, d, st)
                     : go<D, 2, false, true, true, false, false>(src, dst, nullptr, d, st);
   }
+  if (dst == nullptr)   // pool only: the fp64 block means of a natural-order tensor
+    return go<D, 2, true, false, false, true, false>(src, nullptr, pool, d, st);
   if (to_f16) {
     return pool ? go<D, 2, true, false, true, true, true>(src, dst, pool, d, st)
                 : go<D, 2, true, false, true, false, true>(src, dst, nullptr, d, st);
@@ -122,8 +124,9 @@ extern "C" nabla_status nabla_reorder(const void* src, nabla_dtype src_dtype, vo
   Dims d;
   nabla_status rc = check_shape(s, &d);
   if (rc != NABLA_OK) return rc;
-  if (!src || !dst) return NABLA_ERR_INVALID_ARG;
-  if (!aligned16(src) || !aligned16(dst)) return NABLA_ERR_INVALID_ARG;
+  // dst may be NULL for the pool alone (forward direction, pool_out given)
+  if (!src || (!dst && (inverse || !pool_out))) return NABLA_ERR_INVALID_ARG;
+  if (!aligned16(src) || (dst && !aligned16(dst))) return NABLA_ERR_INVALID_ARG;
   const bool dt_ok = inverse ? (src_dtype == dst_dtype &&
                                 (src_dtype == NABLA_BF16 || src_dtype == NABLA_F16 || src_dtype == NABLA_F32))
                              : (src_dtype == NABLA_BF16 && (dst_dtype == NABLA_BF16 || dst_dtype == NABLA_F16));
@@ -133,7 +136,7 @@ extern "C" nabla_status nabla_reorder(const void* src, nabla_dtype src_dtype, vo
   const size_t bytes = static_cast<size_t>(d.BH) * d.S * d.D * esz;
   const char* a = static_cast<const char*>(src);
   const char* b = static_cast<const char*>(dst);
-  if (a < b + bytes && b < a + bytes) return NABLA_ERR_INVALID_ARG;   // overlap
+  if (b && a < b + bytes && b < a + bytes) return NABLA_ERR_INVALID_ARG;   // overlap
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool to_f16 = !inverse && dst_dtype == NABLA_F16;
   cudaError_t e = d.D == 64 ? launch_reorder<64>(src, dst, pool_out, d, inverse, esz, to_f16, st)

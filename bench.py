@@ -193,8 +193,14 @@ class Path:
         sh = self.shape
         self.thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
         self.q, self.k, self.v = make_qkv(wl, device=dev)          # natural order
-        self.qf, self.kf = (torch.empty_like(self.q) for _ in range(2))
-        self.vf = torch.empty(self.q.shape, dtype=torch.float16, device=dev)   # fp16 V operand
+        # Inference (forward only): the forward reads Q, K, V in their natural order and
+        # writes O in it; only the pooled means are computed beforehand.  Training: the
+        # tensors are reordered once (fp16 V for the P V products) and the backward reads
+        # the reordered copies.
+        self.natural = not wl.backward
+        if not self.natural:
+            self.qf, self.kf = (torch.empty_like(self.q) for _ in range(2))
+            self.vf = torch.empty(self.q.shape, dtype=torch.float16, device=dev)
         self.qp = torch.empty(wl.B, wl.H, sh.nb, wl.D, dtype=torch.float64, device=dev)
         self.kp = torch.empty_like(self.qp)
         # the forward reads the bitmask only; the lists serve the backward
@@ -216,12 +222,13 @@ class Path:
     def launches_per_step(self):
         """Kernels of this library launched by one step (memsets not counted).
 
-        reorder x3; mask rows (+ column lists for the backward); forward: 3 schedule
-        kernels + attention; backward: 2 x 3 schedule kernels + preprocess + dK/dV + dQ.
+        Inference: pool Q, pool K; mask (split, logits, select, fp64 rescue); forward
+        (schedule, attention).  Training: reorder Q, K, V; the mask as above + column
+        lists; forward; backward (2 schedules, preprocess, dK/dV, dQ).
         """
-        fwd = 3 + 1 + 4
-        bwd = 1 + 9 if self.wl.backward else 0
-        return fwd + bwd
+        if self.natural:
+            return 2 + 4 + 2
+        return 3 + 4 + 1 + 2 + 5
 
     def _mark(self, name, timing):
         if timing:
@@ -232,17 +239,26 @@ class Path:
     def step(self, timing=False):
         m, sh, wl = self.m, self.shape, self.wl
         self._mark("t0", timing)
-        m.nabla_reorder(self.q, self.qf, sh, pool_out=self.qp)
-        m.nabla_reorder(self.k, self.kf, sh, pool_out=self.kp)
-        m.nabla_reorder(self.v, self.vf, sh)
+        if self.natural:
+            m.nabla_reorder(self.q, None, sh, pool_out=self.qp)
+            m.nabla_reorder(self.k, None, sh, pool_out=self.kp)
+        else:
+            m.nabla_reorder(self.q, self.qf, sh, pool_out=self.qp)
+            m.nabla_reorder(self.k, self.kf, sh, pool_out=self.kp)
+            m.nabla_reorder(self.v, self.vf, sh)
         self._mark("t_reorder", timing)
         m.nabla_build_mask(None, None, sh, self.thr, wl.window, mask_bits=self.bits,
                            row_idx=self.ridx, row_cnt=self.rcnt, col_idx=self.cidx,
                            col_cnt=self.ccnt, q_pool=self.qp, k_pool=self.kp,
                            workspace=self.mask_ws)
         self._mark("t_mask", timing)
-        m.nabla_attn_fwd(self.qf, self.kf, self.vf, self.bits, sh, o=self.o,
-                         o_dtype=self.o_dtype, lse=self.lse, workspace=self.fwd_ws)
+        if self.natural:
+            m.nabla_attn_fwd(self.q, self.k, self.v, self.bits, sh, o=self.o,
+                             o_dtype=self.o_dtype, lse=self.lse, workspace=self.fwd_ws,
+                             layout=m.NABLA_LAYOUT_NATURAL)
+        else:
+            m.nabla_attn_fwd(self.qf, self.kf, self.vf, self.bits, sh, o=self.o,
+                             o_dtype=self.o_dtype, lse=self.lse, workspace=self.fwd_ws)
         self._mark("t_fwd", timing)
         if wl.backward:
             m.nabla_attn_bwd(self.qf, self.kf, self.vf, self.o, self.do, self.lse, self.ridx,
@@ -434,17 +450,36 @@ def main():
 
     # ---- side measurements (outside the timed region) ----------------------------------------
     m, sh = path.m, path.shape
-    mask_ms = time_call(lambda: m.nabla_build_mask(path.qf, path.kf, sh, path.thr, wl.window,
-                                                   mask_bits=path.bits, row_idx=path.ridx,
-                                                   row_cnt=path.rcnt, workspace=path.mask_ws), 5)
+    # the mask from bf16 Q and K (pooling included): natural order -> pool alone, then the
+    # mask from the means; reordered order -> the mask call pools itself
+    if path.natural:
+        def mask_from_qk():
+            m.nabla_reorder(path.q, None, sh, pool_out=path.qp)
+            m.nabla_reorder(path.k, None, sh, pool_out=path.kp)
+            m.nabla_build_mask(None, None, sh, path.thr, wl.window, mask_bits=path.bits,
+                               row_idx=path.ridx, row_cnt=path.rcnt, q_pool=path.qp,
+                               k_pool=path.kp, workspace=path.mask_ws)
+    else:
+        def mask_from_qk():
+            m.nabla_build_mask(path.qf, path.kf, sh, path.thr, wl.window, mask_bits=path.bits,
+                               row_idx=path.ridx, row_cnt=path.rcnt, workspace=path.mask_ws)
+    mask_ms = time_call(mask_from_qk, 5)
     mask_bytes = 2 * BH * wl.S * wl.D * 2 + BH * nb * sh.nw * 4
-    reorder_bytes = 3 * 2 * BH * wl.S * wl.D * 2 + 2 * BH * nb * wl.D * 8
+    # bytes of the pass before the mask: pooling of Q, K (natural path) or reorder of Q,
+    # K, V with pooling (training path)
+    reorder_bytes = (2 * BH * wl.S * wl.D * 2 if path.natural else 3 * 2 * BH * wl.S * wl.D * 2) \
+        + 2 * BH * nb * wl.D * 8
     # all-ones mask (padding bits are ignored by the kernels)
     dense_bits = torch.full((wl.B, wl.H, nb, sh.nw), -1, dtype=torch.int32, device=dev)
     dense_iters = 2 if nb > 1000 else 5
-    dense_ms = time_call(lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, dense_bits, sh,
-                                                  o=path.o, o_dtype=path.o_dtype, lse=path.lse,
-                                                  workspace=path.fwd_ws), dense_iters, warm=1)
+    if path.natural:
+        dense_call = lambda: m.nabla_attn_fwd(path.q, path.k, path.v, dense_bits, sh, o=path.o,
+                                              o_dtype=path.o_dtype, lse=path.lse,
+                                              workspace=path.fwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
+    else:
+        dense_call = lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, dense_bits, sh, o=path.o,
+                                              o_dtype=path.o_dtype, lse=path.lse, workspace=path.fwd_ws)
+    dense_ms = time_call(dense_call, dense_iters, warm=1)
     dense_tflops = BH * nb * nb * fl_fwd / (dense_ms * 1e-3) / 1e12
     path.check_status()
     # restore the NABLA lists (the dense run reused the output buffers only)
@@ -499,7 +534,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.T, wl.Hg, wl.W],
                    "D": wl.D, "P": wl.P, "thr": path.thr, "sta": list(wl.window),
-                   "step": "reorder+pool, mask, attn fwd" + (", attn bwd" if wl.backward else ""),
+                   "step": ("pool Q/K, mask, attn fwd on natural-order Q/K/V" if path.natural
+                            else "reorder+pool, mask, attn fwd, attn bwd"),
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"heads-replicated x{world}"},
         "fwd_ms": fwd_ms, "fwd_tflops_kept": fwd_tflops,
         "dense_fwd_ms": dense_ms, "dense_tflops": dense_tflops, "speedup_vs_dense": dense_ms / fwd_ms,

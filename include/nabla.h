@@ -50,6 +50,11 @@ typedef enum {
 
 typedef enum { NABLA_BF16 = 0, NABLA_F32 = 1, NABLA_F16 = 2 } nabla_dtype;
 
+/* Token order of the attention tensors: the reordered order of nabla_reorder (blocks of
+ * N = P*P consecutive tokens), or the natural order (t, h, w) of the latent, in which a
+ * block is an 8 x 8 spatial patch of one frame, gathered by the kernel as it loads. */
+typedef enum { NABLA_LAYOUT_REORDERED = 0, NABLA_LAYOUT_NATURAL = 1 } nabla_layout;
+
 /* Problem shape.  S = T*Hg*W, N = P*P, nb = S/N.  Hg is the (padded) latent height. */
 typedef struct {
   int32_t B, H, T, Hg, W, D, P;
@@ -77,7 +82,9 @@ const char *nabla_status_string(nabla_status s);
  *   magnitudes become +-inf).
  * inverse != 0: dst[b,h,n(r),:] = src[b,h,r,:] (reordered -> natural), src_dtype ==
  *   dst_dtype in {NABLA_BF16, NABLA_F16, NABLA_F32} (e.g. to restore an output O).
- * src, dst: [B,H,S,D] of those dtypes; must not overlap.
+ * src, dst: [B,H,S,D] of those dtypes; must not overlap.  With inverse == 0 and pool_out
+ *   given, dst may be NULL: only the block means are computed, src is read once and
+ *   nothing is reordered (the natural-layout forward then reads src directly).
  * pool_out (nullable, only with inverse == 0): fp64 [B,H,nb,D], the mean of each
  *   block's N reordered token vectors (sum in token order in fp64, then / N), i.e.
  *   the pooled Q or K of [ZH-TS] "downsampling", ready for nabla_build_mask.
@@ -142,21 +149,25 @@ nabla_status nabla_mask_lists(const uint32_t *mask_bits, nabla_shape s, int32_t 
  *   of row i;  LSE_r = ln sum_c exp(scale * Q_r . K_c).
  * A row with no kept block gives O = 0 and LSE = -inf.
  *
- * q, k       : bf16 [B,H,S,D] reordered.
- * v, v_dtype : [B,H,S,D] reordered, NABLA_BF16 or NABLA_F16.  With fp16 V the
+ * q, k       : bf16 [B,H,S,D] in the token order given by layout.
+ * v, v_dtype : [B,H,S,D] in that order, NABLA_BF16 or NABLA_F16.  With fp16 V the
  *              probabilities P enter the PV product as fp16 (11-bit significand)
  *              instead of bf16 (8-bit): about 8x smaller output error.
  * mask_bits  : the block mask as from nabla_build_mask (padding bits are ignored).
  * o          : out [B,H,S,D], bf16 or f32 per o_dtype.   lse: out f32 [B,H,S] (natural
- *              log; nullable when not needed).
+ *              log; nullable when not needed).  Both in the token order given by layout.
+ * layout     : NABLA_LAYOUT_REORDERED, or NABLA_LAYOUT_NATURAL: q, k, v, o and lse in
+ *              the natural order of the latent, nothing reordered beforehand (the
+ *              fractal flatten of [ZH-TS] "token reordering" is done by the loads; the
+ *              mask and block indices are unchanged).
  * workspace  : >= nabla_fwd_workspace_bytes(s) bytes (tile schedule + status word).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  * --------------------------------------------------------------------------------- */
 size_t nabla_fwd_workspace_bytes(nabla_shape s);
 nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v, nabla_dtype v_dtype,
                             const uint32_t *mask_bits, nabla_shape s, float scale, void *o,
-                            nabla_dtype o_dtype, float *lse, void *workspace,
-                            size_t workspace_bytes, nabla_stream_t stream);
+                            nabla_dtype o_dtype, float *lse, nabla_layout layout,
+                            void *workspace, size_t workspace_bytes, nabla_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Block-sparse attention backward (mask constant)                   [ZH-TS, LSD-2]
@@ -203,7 +214,7 @@ nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, nabla_d
 nabla_status nabla_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                                     nabla_dtype v_dtype, const uint32_t *mask_bits, nabla_shape s,
                                     float scale, void *o, nabla_dtype o_dtype, float *lse,
-                                    nabla_stream_t stream);
+                                    nabla_layout layout, nabla_stream_t stream);
 
 /* Reads (synchronously on `stream`) the device status word that the kernels of the
  * last call on `workspace` recorded: 0 = fine, otherwise a code naming the barrier

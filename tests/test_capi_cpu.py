@@ -72,6 +72,9 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert ro(src=mis) == INV
     assert ro(dst=A) == INV                                               # overlap
     assert ro(pool=A, inv=1) == INV                                       # pool with inverse
+    assert ro(dst=None) == INV                                            # no dst and no pool
+    assert ro(dst=None, pool=ctypes.c_void_p(0x20000004)) == INV          # misaligned pool
+    assert ro(dst=None, inv=1, pool=None) == INV                          # inverse needs dst
     assert ro(sd=F16) == INV                                              # forward needs bf16 source
     assert ro(dd=F32) == INV                                              # no f32 forward output
     assert ro(sd=F32, dd=BF, inv=1) == INV                                # inverse keeps the dtype
@@ -95,8 +98,8 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert bm(ws=ctypes.c_void_p(0x20000010)) == WS                       # misaligned workspace
     fws = lib.nabla_fwd_workspace_bytes(good)
 
-    def fwd(q=A, o=Bp, scale=0.125, odt=0, ws=Bp, wsb=fws, ridx=A, vdt=0):
-        return lib.nabla_attn_fwd(q, A, A, vdt, ridx, good, scale, o, odt, None, ws, wsb, st)
+    def fwd(q=A, o=Bp, scale=0.125, odt=0, ws=Bp, wsb=fws, ridx=A, vdt=0, layout=0):
+        return lib.nabla_attn_fwd(q, A, A, vdt, ridx, good, scale, o, odt, None, layout, ws, wsb, st)
     assert fwd(q=None) == INV
     assert fwd(q=mis) == INV
     assert fwd(ridx=None) == INV
@@ -105,5 +108,6 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert fwd(odt=2) == INV
     assert fwd(vdt=1) == INV
     assert fwd(wsb=fws - 1) == WS
+    assert fwd(layout=2) == INV                                            # unknown layout
     assert lib.nabla_fwd_workspace_bytes(_shape(nb, D=96)) == 0
     assert lib.nabla_status_string(3) == b"NABLA_ERR_WORKSPACE"

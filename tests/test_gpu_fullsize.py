@@ -71,15 +71,17 @@ def test_fullsize_mask_and_forward(name):
     bf16_out = path.o.dtype == torch.bfloat16
     scale = 1 / math.sqrt(wl.D)
     heads = [(int(b), int(h)) for b, h in zip(rng.integers(0, wl.B, 4), rng.integers(0, wl.H, 4))]
+    perm = oracle.fractal_permutation(wl.T, wl.Hg, wl.W, wl.P)
     for b, h in heads:
-        q, k = (_head(t, b, h, wl) for t in (path.qf, path.kf))
-        v = _head(path.v, b, h, wl, reorder=True)        # bf16 values (the kernel reads fp16 V)
+        q, k, v = (_head(t, b, h, wl, reorder=True) for t in (path.q, path.k, path.v))
         blocks = rng.choice(wl.nb, size=6, replace=False)
         rows = (blocks[:, None] * wl.N + np.arange(wl.N)[None, :]).reshape(-1)
         O, L = oracle.block_sparse_attention_rows(q, k, v, gm[b, h], wl.N, scale, rows)
-        got = path.o[b, h, torch.from_numpy(rows).cuda()].detach().cpu().double().numpy()
+        # outputs in natural order (the inference path) sit at the tokens' natural indices
+        at = torch.from_numpy(perm[rows] if path.natural else rows).cuda()
+        got = path.o[b, h, at].detach().cpu().double().numpy()
         check_close(got, O, f"O {name} head {b},{h}", storage_bf16=bf16_out)
-        lse = path.lse[b, h, torch.from_numpy(rows).cuda()].cpu().double().numpy()
+        lse = path.lse[b, h, at].cpu().double().numpy()
         check_lse(lse, L)
 
 

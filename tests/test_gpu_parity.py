@@ -71,6 +71,21 @@ def _wl(name):
     return {"odd": ODD, "odd64": ODD64, "wide": WIDE}.get(name) or WORKLOADS[name]
 
 
+@pytest.mark.parametrize("name", ["tiny", "small", "odd64"])
+def test_pool_only_matches_reorder_pool(data, name):
+    """nabla_reorder with dst = NULL: the block means alone, bit-identical to the ones the
+    reorder-and-pool pass produces."""
+    m = nbl()
+    wl = _wl(name)
+    shape = shape_of(wl)
+    q, _, _ = data(wl)
+    _, qp = gpu_reorder(q, shape, pool=True)
+    qp2 = torch.empty_like(qp)
+    m.nabla_reorder(q, None, shape, pool_out=qp2)
+    torch.cuda.synchronize()
+    assert torch.equal(qp, qp2)
+
+
 def test_mask_without_data():
     """thr <= 0 (pure STA) and thr >= 1 (keep all) need neither Q, K nor pooled means."""
     m = nbl()
@@ -147,6 +162,37 @@ def test_fwd_parity(data, name, thr, window, o_dtype, v_dtype):
     check_lse(lse.cpu().numpy().astype(np.float64), L)
     print(f"{name} thr={thr}: density {gm.mean():.4f} max|O| {np.abs(O).max():.2f} "
           f"max err {mx:.2e} mean err {mean:.2e}")
+
+
+@pytest.mark.parametrize("name,thr,window", [("tiny", 0.8, (0, 0, 0)), ("small", 0.8, (0, 0, 0)),
+                                             ("small", 0.5, (1, 3, 3)), ("odd", 0.8, (0, 0, 0)),
+                                             ("odd64", 0.6, (0, 0, 0))])
+@pytest.mark.parametrize("v_dtype", ["f16", "bf16"])
+def test_fwd_natural_layout(data, name, thr, window, v_dtype):
+    """Natural-order q, k, v in, natural-order O and LSE out (the reorder done by the
+    kernel's loads); same mask, compared with the oracle's output in natural order."""
+    m = nbl()
+    wl = _wl(name)
+    shape = shape_of(wl)
+    q, k, v = data(wl)
+    qf, _ = gpu_reorder(q, shape)
+    kf, _ = gpu_reorder(k, shape)
+    vf, _ = gpu_reorder(v, shape)
+    bits, *_ = gpu_mask(qf, kf, shape, thr, window, cols=False)
+    vn = v.half() if v_dtype == "f16" else v
+    lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
+    ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    o, _ = m.nabla_attn_fwd(q, k, vn, bits, shape, o_dtype=m.NABLA_F32, lse=lse, workspace=ws,
+                            layout=m.NABLA_LAYOUT_NATURAL)
+    torch.cuda.synchronize()
+    assert m.nabla_read_device_status(ws) == 0
+    gm = bits_to_mask(bits, wl.nb)
+    O, L = oracle.block_sparse_attention(to64(qf), to64(kf), to64(vf), gm, wl.N, 1 / math.sqrt(wl.D))
+    On = oracle.inverse_reorder(O, wl.T, wl.Hg, wl.W, wl.P)
+    Ln = oracle.inverse_reorder(L[..., None], wl.T, wl.Hg, wl.W, wl.P)[..., 0]
+    mx, mean = check_close(to64(o), On, f"O natural {name}")
+    check_lse(lse.cpu().numpy().astype(np.float64), Ln)
+    print(f"natural {name} thr={thr} V {v_dtype}: max err {mx:.2e} mean err {mean:.2e}")
 
 
 def test_fwd_dense_and_empty_rows(data):
