@@ -296,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int fetched = 0;            // descriptors published
       bool end = false, ok = true;
       for (int c = 0; ok; ++c) {
-        // descriptors of this tile and the next one
-        while (!end && fetched <= c + 1) {
+        // the descriptor of this tile (normally fetched one tile ahead)
+        while (!end && fetched <= c) {
           const int f = fetch(fetched);
           if (f < 0) { ok = false; break; }
           ++fetched;
@@ -306,7 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok || c >= fetched) break;
         const TileMeta t = read_meta(meta + (c % R) * kMetaInts);
         if (t.item < 0) break;
-        // Q: the buffer frees once the previous tile's last S has run.
+        // Q: the buffer frees once the previous tile's last S has run.  It is copied before
+        // the next descriptor is fetched (three dependent global round trips), which would
+        // otherwise delay every tile's first S.
         if (c > 0 && !wait_all(&B.q_empty, (c - 1) & 1, kDevTimeoutQFull)) { ok = false; break; }
         if (lane == 0) {
           mbar_arrive_expect_tx(&B.q_full, C::kTileBytes);
@@ -318,6 +320,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         ++nq;
+        // the next tile's descriptor, while this tile's copies run
+        if (!end && fetched == c + 1) {
+          const int f = fetch(fetched);
+          if (f < 0) { ok = false; break; }
+          ++fetched;
+          if (f == 0) end = true;
+        }
         WarpBitWalk wk;
         wk.init(prm.bits + (static_cast<long long>(t.bh) * nb + t.ia) * nw,
                 t.ib >= 0 ? prm.bits + (static_cast<long long>(t.bh) * nb + t.ib) * nw : nullptr, nw, nb);
@@ -569,33 +578,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         tok = static_cast<long long>(t.bh) * prm.S + static_cast<long long>(valid_row ? blk : 0) * 64 + (row & 63);
       }
+      if (prm.o_f32) {
 #pragma unroll 1
-      for (int d0 = 0; d0 < D; d0 += 32) {
-        uint32_t a0[32];
-        if (n > 0) {
-          tmem_ld32(o_col + d0, a0);
-          tmem_wait_ld();
-          reg_fence32(a0);
-        }
-        float v[32];
+        for (int d0 = 0; d0 < D; d0 += 32) {
+          uint32_t a0[32];
+          if (n > 0) {
+            tmem_ld32(o_col + d0, a0);
+            tmem_wait_ld();
+            reg_fence32(a0);
+          } else {
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) v[cc] = n > 0 ? __uint_as_float(a0[cc]) * inv : 0.f;
-        if (valid_row) {
-          if (prm.o_f32) {
+            for (int cc = 0; cc < 32; ++cc) a0[cc] = 0u;
+          }
+          if (valid_row) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(prm.o) + tok * D + d0);
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) dst[cc] = make_float4(v[4 * cc], v[4 * cc + 1], v[4 * cc + 2], v[4 * cc + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.o) + tok * D + d0);
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-              dst[cc] = make_uint4(pack_bf16x2(v[8 * cc], v[8 * cc + 1]), pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]),
-                                   pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]), pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]));
+            for (int cc = 0; cc < 8; ++cc)
+              dst[cc] = make_float4(__uint_as_float(a0[4 * cc]) * inv, __uint_as_float(a0[4 * cc + 1]) * inv,
+                                    __uint_as_float(a0[4 * cc + 2]) * inv, __uint_as_float(a0[4 * cc + 3]) * inv);
           }
         }
+        tc_fence_before();
+        mbar_arrive(&B.o_free);
+      } else {
+        // bf16 output: the whole row is read and packed first (D / 2 registers), so that the
+        // next tile's P V may overwrite the accumulator while the row is being stored.
+        uint32_t packed[D / 2];
+#pragma unroll
+        for (int d0 = 0; d0 < D; d0 += 32) {
+          uint32_t a0[32];
+          if (n > 0) {
+            tmem_ld32(o_col + d0, a0);
+            tmem_wait_ld();
+            reg_fence32(a0);
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) a0[cc] = 0u;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc)
+            packed[d0 / 2 + cc] = pack_bf16x2(__uint_as_float(a0[2 * cc]) * inv, __uint_as_float(a0[2 * cc + 1]) * inv);
+        }
+        tc_fence_before();
+        mbar_arrive(&B.o_free);
+        if (valid_row) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.o) + tok * D);
+#pragma unroll
+          for (int cc = 0; cc < D / 8; ++cc)
+            dst[cc] = make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2], packed[4 * cc + 3]);
+        }
       }
-      tc_fence_before();
-      mbar_arrive(&B.o_free);
       if (valid_row && prm.lse != nullptr)
         prm.lse[tok] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       mbar_arrive(&B.meta_empty[c % R]);

@@ -2,11 +2,17 @@
 // or with frame pairs the two blocks of tile_blocks()).
 //
 // Heads are taken one after another (head-major), so the tiles running at the same time
-// read K and V of one head and those stay resident in L2; inside a head, tiles run
-// longest first (descending length of their two kept lists, an upper bound of the
-// union a tile walks), which keeps the tail short.  One CTA sorts one head's tiles with
-// a bitonic sort on (length descending, tile index ascending): the order is fully
-// deterministic, and every tile's result is independent of the order anyway.
+// read K and V of one or two heads and those stay resident in L2.  Inside a head, tiles
+// run longest first (descending length of their two kept lists, an upper bound of the
+// union a tile walks).  The heads themselves run in descending order of their longest
+// tile: the kept-block counts differ by two orders of magnitude between heads (a head
+// with flat pooled scores keeps hundreds of blocks per row, a peaked one a handful), and
+// a long tile that starts late would leave the other SMs idle at the end.  Two launches:
+// one CTA per head sorts the head's tiles with a bitonic sort on (length descending,
+// tile index ascending) and records the head's longest tile; then one CTA per head finds
+// the head's rank (longest tile descending, head index ascending) and copies its tiles
+// to that position.  The order is fully deterministic, and every tile's result is
+// independent of the order anyway.
 #include "common.cuh"
 
 namespace nabla {
@@ -18,7 +24,8 @@ __global__ void __launch_bounds__(512) sched_head_sort_kernel(const int32_t* __r
                                                               const uint32_t* __restrict__ bits,
                                                               int nb, int nw, int npairs, int npow2,
                                                               int T, int HW, int frame_pairs,
-                                                              int32_t* __restrict__ order) {
+                                                              int32_t* __restrict__ sorted,
+                                                              int32_t* __restrict__ head_len) {
   extern __shared__ unsigned long long keys[];
   const long long bh = blockIdx.x;
   for (int e = threadIdx.x; e < npow2; e += blockDim.x) {
@@ -65,7 +72,34 @@ __global__ void __launch_bounds__(512) sched_head_sort_kernel(const int32_t* __r
     }
   }
   for (int e = threadIdx.x; e < npairs; e += blockDim.x)
-    order[bh * npairs + e] = static_cast<int32_t>(bh * npairs + static_cast<long long>(keys[e] & 0xFFFFFFFFull));
+    sorted[bh * npairs + e] = static_cast<int32_t>(bh * npairs + static_cast<long long>(keys[e] & 0xFFFFFFFFull));
+  if (threadIdx.x == 0) head_len[bh] = npairs > 0 ? 0x7FFFFFFF - static_cast<int>(keys[0] >> 32) : 0;
+}
+
+// Places head bh's sorted tiles at its rank among the heads: longest tile descending,
+// head index ascending.
+__global__ void __launch_bounds__(256) sched_head_place_kernel(const int32_t* __restrict__ sorted,
+                                                               const int32_t* __restrict__ head_len,
+                                                               int BH, int npairs,
+                                                               int32_t* __restrict__ order) {
+  __shared__ int part[8];
+  const int bh = blockIdx.x;
+  const int mine = head_len[bh];
+  int before = 0;
+  for (int h = threadIdx.x; h < BH; h += blockDim.x) {
+    const int len = head_len[h];
+    before += (len > mine || (len == mine && h < bh)) ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = before;
+  __syncthreads();
+  int rank = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) rank += part[w];
+  const long long src = static_cast<long long>(bh) * npairs;
+  const long long dst = static_cast<long long>(rank) * npairs;
+  for (int e = threadIdx.x; e < npairs; e += blockDim.x) order[dst + e] = sorted[src + e];
 }
 
 int next_pow2(int x) {
@@ -78,7 +112,8 @@ int next_pow2(int x) {
 
 size_t schedule_scratch_bytes(const Dims& d) {
   const size_t items = static_cast<size_t>(d.BH) * ((d.nb + 1) / 2);
-  return align_up(items * 4, 256);
+  // the order, the per-head sorted tiles, the per-head longest tile
+  return 2 * align_up(items * 4, 256) + align_up(static_cast<size_t>(d.BH) * 4, 256);
 }
 
 // Writes the item order to the start of `scratch`; returns it.  Tile lengths from the
@@ -87,13 +122,19 @@ cudaError_t build_schedule(const int32_t* cnt, const uint32_t* bits, const Dims&
                            int32_t** order_out, cudaStream_t st, bool frame_pairs) {
   const int npairs = (d.nb + 1) / 2;
   const int npow2 = next_pow2(npairs);
+  const size_t items_bytes = align_up(static_cast<size_t>(d.BH) * npairs * 4, 256);
   int32_t* order = static_cast<int32_t*>(scratch);
+  int32_t* sorted = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + items_bytes);
+  int32_t* head_len = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + 2 * items_bytes);
   const size_t smem = static_cast<size_t>(npow2) * 8;
   cudaError_t e = cudaFuncSetAttribute(sched_head_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   sched_head_sort_kernel<<<d.BH, 512, smem, st>>>(cnt, bits, d.nb, d.nw, npairs, npow2, d.T,
-                                                   d.Hb * d.Wb, frame_pairs ? 1 : 0, order);
+                                                   d.Hb * d.Wb, frame_pairs ? 1 : 0, sorted, head_len);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sched_head_place_kernel<<<d.BH, 256, 0, st>>>(sorted, head_len, d.BH, npairs, order);
   *order_out = order;
   return cudaGetLastError();
 }

@@ -223,12 +223,13 @@ class Path:
         """Kernels of this library launched by one step (memsets not counted).
 
         Inference: pool Q, pool K; mask (split, logits, select, fp64 rescue); forward
-        (schedule, attention).  Training: reorder Q, K, V; the mask as above + column
-        lists; forward; backward (2 schedules, preprocess, dK/dV, dQ).
+        (schedule: per-head sort + head placement; attention).  Training: reorder Q, K,
+        V; the mask as above + column lists; forward; backward (2 schedules of 2
+        launches, preprocess, dK/dV, dQ).
         """
         if self.natural:
-            return 2 + 4 + 2
-        return 3 + 4 + 1 + 2 + 5
+            return 2 + 4 + 3
+        return 3 + 4 + 1 + 3 + 7
 
     def _mark(self, name, timing):
         if timing:

@@ -203,7 +203,7 @@ nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, nabla_d
  * array in the library's own device memory (every GPU that loads the library holds it
  * until the process exits).  Problems whose workspace (nabla_fwd_workspace_bytes)
  * exceeds 1 MiB are rejected with NABLA_ERR_UNSUPPORTED before anything is enqueued
- * (the 720p-like 40-head problem needs about 210 KB).  The first call on a device looks
+ * (the 720p-like 40-head problem needs about 200 KB).  The first call on a device looks
  * up that array's device address (cudaGetSymbolAddress, with the device current); make
  * that first call before any stream capture.  The call allocates nothing.  All calls
  * share the one array, which keeps the last call's contents (each call clears what
