@@ -11,16 +11,19 @@
 //
 // Deterministic, no floating-point atomics, three launches:
 //   1. preprocess: Dr = rowsum(dO * O) and LSE in log2 units (HBM-bound);
-//   2. dK/dV: one CTA per pair of key blocks (128 key rows -> M = 128 MMAs) walks the
-//      ascending union of the two blocks' query-block (column) lists.  Per query block:
-//      S^T = K Q^T and dP^T = V dO^T into TMEM (double-buffered), P^T and dS^T in
-//      registers (one key row per thread) -> bf16 in shared memory, then
-//      dV += P^T dO and dK += dS^T Q into TMEM accumulators;
+//   2. dK/dV: one CTA per pair of key blocks (the same patch in frames 2u and 2u + 1, as
+//      the forward pairs query blocks: their column lists overlap most; 128 key rows ->
+//      M = 128 MMAs) walks the ascending union of the two blocks' query-block (column)
+//      lists.  Per query block: S^T = K Q^T and dP^T = V dO^T into TMEM (double-buffered);
+//      P^T and dS^T are formed in registers and written back over them as 16-bit
+//      operands; dV += P^T dO and dK += dS^T Q read those from TMEM (A operand) and
+//      accumulate in TMEM;
 //   3. dQ: one CTA per pair of query blocks walks the union of the row lists:
-//      S = Q K^T and dP = dO V^T into TMEM, dS in registers -> shared memory,
-//      dQ += dS K.
-// Warp roles as in the forward kernel: warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warps 4-7 = element-wise math and epilogue.  Every wait is bounded.
+//      S = Q K^T and dP = dO V^T into TMEM, dS written back over dP, dQ += dS K.
+// Warp roles: warp 0 = TMA producer (four-stage ring), warp 1 = MMA issuer and TMEM owner,
+// warps 4-11 = element-wise math (a key or query row per TMEM lane, each 64-wide tile
+// split in two column halves between warps w and w + 4) and epilogue.  Every wait is
+// bounded.
 #include <math.h>
 
 #include <cudaTypedefs.h>
@@ -36,8 +39,9 @@ bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int 
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;             // warp 0 TMA, warp 1 MMA, warps 4-11 element-wise
 constexpr int kMathWarp0 = 4;
+constexpr int kMathThreads = 256;
 constexpr uint32_t kEnd = 0xFFFFFFFFu;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -137,6 +141,7 @@ struct BwdParams {
   float* out1;               // dK (dK/dV pass)
   uint32_t* status;
   int nb;
+  int T, HW;                 // frames, blocks per frame (pairing of blocks, tile_blocks())
   long long S;
   float scale_log2;
   float scale;
@@ -166,11 +171,17 @@ struct BwdCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPairBytes = 128 * D * 2;       // one 128-row operand (resident)
   static constexpr int kTileBytes = 64 * D * 2;        // one 64-row operand (streamed)
-  static constexpr int kPBytes = 128 * 64 * 2;         // one bf16 128 x 64 tile
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM: buffer b at columns [128b, 128b+64) = S (or S^T), [128b+64, 128b+128) = dP.
+  // TMEM: buffer b at columns [128b, 128b+64) = S (or S^T), [128b+64, 128b+128) = dP (or
+  // dP^T); the element-wise pass overwrites them in place with the 16-bit P and dS
+  // operands of the next MMAs.  Accumulators from column 256.
   static constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
 };
+
+// Column of the packed 16-bit operand for K chunk kk (16 values, 8 columns) of a 64-wide
+// tile written in place by two thread groups: group h packs its 32 values into the first
+// 16 of the 32 columns it read, [32h, 32h+16).
+__device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 2 ? kk * 8 : 32 + (kk - 2) * 8; }
 
 // -------------------------------------------------------------------------------------
 // 2. dK / dV over column lists
@@ -178,24 +189,24 @@ struct BwdCfg {
 template <int D>
 struct DkdvLayout {
   using C = BwdCfg<D>;
-  static constexpr int kStages = 2;
+  static constexpr int kStages = 4;
   static constexpr int kStageBytes = 2 * C::kTileBytes + 512;    // Q_i, dO_i, lse2_i, delta_i
+  static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + C::kPairBytes;
   static constexpr int kOffStage = kOffV + C::kPairBytes;
-  static constexpr int kOffPT = kOffStage + kStages * ((kStageBytes + 1023) / 1024 * 1024);
-  static constexpr int kOffDST = kOffPT + 2 * C::kPBytes;
-  static constexpr int kOffBar = kOffDST + 2 * C::kPBytes;
-  static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+  static constexpr int kOffBar = kOffStage + kStages * kStageStride;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
 };
 
+// One CTA per pair of key blocks (ja, jb) = tile_blocks(pair): rows 0-63 of the resident
+// K and V operands are block ja, rows 64-127 block jb.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_q64,
                          const __grid_constant__ CUtensorMap map_do64,
-                         const __grid_constant__ CUtensorMap map_k128,
-                         const __grid_constant__ CUtensorMap map_v128, const BwdParams prm) {
+                         const __grid_constant__ CUtensorMap map_k64,
+                         const __grid_constant__ CUtensorMap map_v64, const BwdParams prm) {
   using C = BwdCfg<D>;
   using L = DkdvLayout<D>;
   extern __shared__ unsigned char smem_raw[];
@@ -204,8 +215,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sK = smem + L::kOffK;
   unsigned char* sV = smem + L::kOffV;
   unsigned char* sStage = smem + L::kOffStage;
-  unsigned char* sPT = smem + L::kOffPT;
-  unsigned char* sDST = smem + L::kOffDST;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* full = bars;                    // [kStages]
   uint64_t* empty = bars + L::kStages;      // [kStages]
@@ -222,8 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int item = prm.order[blockIdx.x];
   const long long bh = item / prm.npairs;
   const int nb = prm.nb;
-  const int j0 = 2 * (item - static_cast<int>(bh) * prm.npairs);
-  const bool has_j1 = (j0 + 1) < nb;
+  const int2 jab = tile_blocks(item - static_cast<int>(bh) * prm.npairs, prm.T, prm.HW, nb);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -233,8 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(kv_full, 1);
     mbar_init(&sd_full[0], 1);
     mbar_init(&sd_full[1], 1);
-    mbar_init(&p_full[0], 128);
-    mbar_init(&p_full[1], 128);
+    mbar_init(&p_full[0], kMathThreads);
+    mbar_init(&p_full[1], kMathThreads);
     mbar_init(acc_bar, 1);
     mbar_init(drain, 1);
     fence_mbarrier_init();
@@ -252,20 +260,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&map_q64);
       tma_prefetch_desc(&map_do64);
-      tma_prefetch_desc(&map_k128);
-      tma_prefetch_desc(&map_v128);
-      const int krow = static_cast<int>(bh * prm.S + static_cast<long long>(j0) * 64);
+      tma_prefetch_desc(&map_k64);
+      tma_prefetch_desc(&map_v64);
+      // a lone block (jab.y < 0) is loaded twice; its upper rows are never kept
+      const int ka = static_cast<int>(bh * prm.S + static_cast<long long>(jab.x) * 64);
+      const int kb = static_cast<int>(bh * prm.S + static_cast<long long>(jab.y >= 0 ? jab.y : jab.x) * 64);
       mbar_arrive_expect_tx(kv_full, 2 * C::kPairBytes);
 #pragma unroll
       for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_2d(sK + pn * 16384, &map_k128, kv_full, pn * 64, krow);
-        tma_load_2d(sV + pn * 16384, &map_v128, kv_full, pn * 64, krow);
+        tma_load_2d(sK + pn * 16384, &map_k64, kv_full, pn * 64, ka);
+        tma_load_2d(sK + pn * 16384 + 8192, &map_k64, kv_full, pn * 64, kb);
+        tma_load_2d(sV + pn * 16384, &map_v64, kv_full, pn * 64, ka);
+        tma_load_2d(sV + pn * 16384 + 8192, &map_v64, kv_full, pn * 64, kb);
       }
       UnionWalk wk;
-      wk.l0 = prm.list_idx + (bh * nb + j0) * static_cast<long long>(nb);
-      wk.l1 = wk.l0 + nb;
-      wk.c0 = min(max(prm.list_cnt[bh * nb + j0], 0), nb);
-      wk.c1 = has_j1 ? min(max(prm.list_cnt[bh * nb + j0 + 1], 0), nb) : 0;
+      wk.l0 = prm.list_idx + (bh * nb + jab.x) * static_cast<long long>(nb);
+      wk.l1 = prm.list_idx + (bh * nb + (jab.y >= 0 ? jab.y : jab.x)) * static_cast<long long>(nb);
+      wk.c0 = min(max(prm.list_cnt[bh * nb + jab.x], 0), nb);
+      wk.c1 = jab.y >= 0 ? min(max(prm.list_cnt[bh * nb + jab.y], 0), nb) : 0;
       wk.a = wk.b = 0;
       int it = 0;
       bool ended = false;
@@ -310,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_acc = idesc_f16_f32(128, D, false, true);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       const uint32_t st_addr = smem_u32(sStage);
-      const uint32_t pt_addr = smem_u32(sPT), dst_addr = smem_u32(sDST);
+      // S^T = K Q_i^T and dP^T = V dO_i^T into buffer x & 1
       auto issue_sd = [&](int x) {
         const int s = x % L::kStages;
         const uint32_t qa = st_addr + s * L::kStageStride;
@@ -330,17 +342,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&sd_full[x & 1]);
       };
+      // dV += P^T dO_i and dK += dS^T Q_i, with P^T and dS^T read from TMEM
       auto issue_acc = [&](int x) {
         const int s = x % L::kStages;
         const uint32_t qa = st_addr + s * L::kStageStride;
         const uint32_t da = qa + C::kTileBytes;
-        const uint32_t b = x & 1;
+        const uint32_t col = (x & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16_ss(tmem + C::kColAcc0, sdesc_sw128(pt_addr + b * C::kPBytes + kk * 32, 16, 1024),
-                      sdesc_sw128(da + kk * 2048, 8192, 1024), idesc_acc, (x > 0 || kk > 0));
-          mma_bf16_ss(tmem + C::kColAcc1, sdesc_sw128(dst_addr + b * C::kPBytes + kk * 32, 16, 1024),
-                      sdesc_sw128(qa + kk * 2048, 8192, 1024), idesc_acc, (x > 0 || kk > 0));
+          mma_bf16_ts(tmem + C::kColAcc0, tmem + col + packed_col(kk), sdesc_sw128(da + kk * 2048, 8192, 1024),
+                      idesc_acc, (x > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::kColAcc1, tmem + col + 64 + packed_col(kk),
+                      sdesc_sw128(qa + kk * 2048, 8192, 1024), idesc_acc, (x > 0 || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(kv_full, 0, prm.status, kDevTimeoutQFull);
@@ -353,6 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&full[s1], ((it + 1) / L::kStages) & 1, prm.status, kDevTimeoutTmaFull)) break;
           const bool end1 = meta[s1] == kEnd;
           tc_fence_after();
+          // buffer (it + 1) & 1 was last read by issue_acc(it - 1), issued before: MMAs of
+          // one thread run in order
           if (!end1) issue_sd(it + 1);
           if (!mbar_wait(&p_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutPFull)) break;
           tc_fence_after();
@@ -367,12 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= kMathWarp0) {
-    const int row = threadIdx.x - kMathWarp0 * 32;          // key row within the pair
-    const uint32_t lane_base = static_cast<uint32_t>((warp - kMathWarp0) * 32) << 16;
+    // 8 warps: key row = TMEM lane ((warp & 3) * 32 + lane), column half h of each 64-wide
+    // tile (warps 4-7: queries 0-31, warps 8-11: queries 32-63)
+    const int mw = warp - kMathWarp0;
+    const int h = mw >> 2;
+    const int row = (mw & 3) * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>((mw & 3) * 32) << 16;
     const bool upper = row >= 64;
     const float sl2 = prm.scale_log2;
-    unsigned char* ptrow = sPT + row * 128;
-    unsigned char* dsrow = sDST + row * 128;
     int it = 0;
     bool ok = true;
     for (;; ++it) {
@@ -382,49 +399,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t mt = meta[s];
       if (mt == kEnd) break;
       const bool keep = upper ? ((mt >> 29) & 1u) : ((mt >> 28) & 1u);
-      const float* s_lse = reinterpret_cast<const float*>(sStage + s * L::kStageStride + 2 * C::kTileBytes);
+      const float* s_lse = reinterpret_cast<const float*>(sStage + s * L::kStageStride + 2 * C::kTileBytes) + 32 * h;
       const float* s_del = s_lse + 64;
       ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutSFull));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t col = (it & 1) * 128;
-      uint32_t pk[32], dk[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      const uint32_t col = tmem + lane_base + (it & 1) * 128 + 32 * h;
+      uint32_t pk[16], dk[16];
+      if (keep) {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_base + col + half * 32, sv);
-        tmem_ld32(tmem + lane_base + col + 64 + half * 32, dv);
+        tmem_ld32(col, sv);
+        tmem_ld32(col + 64, dv);
         tmem_wait_ld();
-        if (keep) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const int q0 = half * 32 + c;
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -s_lse[q0]));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -s_lse[q0 + 1]));
-            const float d0 = p0 * (__uint_as_float(dv[c]) - s_del[q0]);
-            const float d1 = p1 * (__uint_as_float(dv[c + 1]) - s_del[q0 + 1]);
-            pk[half * 16 + (c >> 1)] = pack_f16x2(p0, p1);
-            dk[half * 16 + (c >> 1)] = pack_f16x2(d0, d1);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) { pk[half * 16 + c] = 0u; dk[half * 16 + c] = 0u; }
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -s_lse[c]));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -s_lse[c + 1]));
+          pk[c >> 1] = pack_f16x2(p0, p1);
+          dk[c >> 1] = pack_f16x2(p0 * (__uint_as_float(dv[c]) - s_del[c]),
+                                  p1 * (__uint_as_float(dv[c + 1]) - s_del[c + 1]));
         }
-      }
-      const int b = it & 1;
+      } else {
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const int off = b * C::kPBytes + ((ch ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(ptrow + off) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(dsrow + off) = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+        for (int c = 0; c < 16; ++c) { pk[c] = 0u; dk[c] = 0u; }
       }
-      fence_proxy_async_smem();
+      tmem_st16(col, pk);
+      tmem_st16(col + 64, dk);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[b]);
+      mbar_arrive(&p_full[it & 1]);
     }
-    // ---- epilogue: dV and scale * dK (fp32) ----------------------------------------------
-    const bool valid = upper ? has_j1 : true;
-    const long long tok = bh * prm.S + static_cast<long long>(j0) * 64 + row;
+    // ---- epilogue: dV and scale * dK (fp32), columns [64h, 64h + 64) of the row ----------
+    const int blk = upper ? jab.y : jab.x;
+    const bool valid = blk >= 0;
+    const long long tok = bh * prm.S + static_cast<long long>(valid ? blk : 0) * 64 + (row & 63);
     bool have = ok && it > 0;
     if (have) {
       have = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, prm.status, kDevTimeoutOBar));
@@ -434,9 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int which = 0; which < 2; ++which) {
       float* out = which == 0 ? prm.out0 : prm.out1;
       const float mul = which == 0 ? 1.f : prm.scale;
-      const uint32_t colbase = which == 0 ? C::kColAcc0 : C::kColAcc1;
+      const uint32_t colbase = (which == 0 ? C::kColAcc0 : C::kColAcc1) + (D / 2) * h;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
         uint32_t ov[32];
         if (have) {
           tmem_ld32(tmem + lane_base + colbase + c0, ov);
@@ -446,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 32; ++c) ov[c] = 0u;
         }
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(out + tok * D + c0);
+          float4* dst = reinterpret_cast<float4*>(out + tok * D + (D / 2) * h + c0);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             dst[c] = make_float4(__uint_as_float(ov[4 * c]) * mul, __uint_as_float(ov[4 * c + 1]) * mul,
@@ -469,20 +477,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 struct DqLayout {
   using C = BwdCfg<D>;
-  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kStages = 4;
   static constexpr int kStageBytes = 2 * C::kTileBytes;        // K_j, V_j
   static constexpr int kOffQ = 0;
   static constexpr int kOffDO = kOffQ + C::kPairBytes;
   static constexpr int kOffStage = kOffDO + C::kPairBytes;
-  static constexpr int kOffDS = kOffStage + kStages * kStageBytes;
-  static constexpr int kOffBar = kOffDS + 2 * C::kPBytes;
+  static constexpr int kOffBar = kOffStage + kStages * kStageBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
 };
 
+// One CTA per pair of query blocks (ia, ib) = tile_blocks(pair).
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q128,
-                       const __grid_constant__ CUtensorMap map_do128,
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q64,
+                       const __grid_constant__ CUtensorMap map_do64,
                        const __grid_constant__ CUtensorMap map_k64,
                        const __grid_constant__ CUtensorMap map_v64, const BwdParams prm) {
   using C = BwdCfg<D>;
@@ -493,7 +501,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sQ = smem + L::kOffQ;
   unsigned char* sDO = smem + L::kOffDO;
   unsigned char* sStage = smem + L::kOffStage;
-  unsigned char* sDS = smem + L::kOffDS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + L::kStages;
@@ -510,8 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int item = prm.order[blockIdx.x];
   const long long bh = item / prm.npairs;
   const int nb = prm.nb;
-  const int i0 = 2 * (item - static_cast<int>(bh) * prm.npairs);
-  const bool has_i1 = (i0 + 1) < nb;
+  const int2 iab = tile_blocks(item - static_cast<int>(bh) * prm.npairs, prm.T, prm.HW, nb);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -521,8 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(&sd_full[0], 1);
     mbar_init(&sd_full[1], 1);
-    mbar_init(&p_full[0], 128);
-    mbar_init(&p_full[1], 128);
+    mbar_init(&p_full[0], kMathThreads);
+    mbar_init(&p_full[1], kMathThreads);
     mbar_init(acc_bar, 1);
     mbar_init(drain, 1);
     fence_mbarrier_init();
@@ -538,22 +544,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&map_q128);
-      tma_prefetch_desc(&map_do128);
+      tma_prefetch_desc(&map_q64);
+      tma_prefetch_desc(&map_do64);
       tma_prefetch_desc(&map_k64);
       tma_prefetch_desc(&map_v64);
-      const int qrow = static_cast<int>(bh * prm.S + static_cast<long long>(i0) * 64);
+      const int qa = static_cast<int>(bh * prm.S + static_cast<long long>(iab.x) * 64);
+      const int qb = static_cast<int>(bh * prm.S + static_cast<long long>(iab.y >= 0 ? iab.y : iab.x) * 64);
       mbar_arrive_expect_tx(q_full, 2 * C::kPairBytes);
 #pragma unroll
       for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_2d(sQ + pn * 16384, &map_q128, q_full, pn * 64, qrow);
-        tma_load_2d(sDO + pn * 16384, &map_do128, q_full, pn * 64, qrow);
+        tma_load_2d(sQ + pn * 16384, &map_q64, q_full, pn * 64, qa);
+        tma_load_2d(sQ + pn * 16384 + 8192, &map_q64, q_full, pn * 64, qb);
+        tma_load_2d(sDO + pn * 16384, &map_do64, q_full, pn * 64, qa);
+        tma_load_2d(sDO + pn * 16384 + 8192, &map_do64, q_full, pn * 64, qb);
       }
       UnionWalk wk;
-      wk.l0 = prm.list_idx + (bh * nb + i0) * static_cast<long long>(nb);
-      wk.l1 = wk.l0 + nb;
-      wk.c0 = min(max(prm.list_cnt[bh * nb + i0], 0), nb);
-      wk.c1 = has_i1 ? min(max(prm.list_cnt[bh * nb + i0 + 1], 0), nb) : 0;
+      wk.l0 = prm.list_idx + (bh * nb + iab.x) * static_cast<long long>(nb);
+      wk.l1 = prm.list_idx + (bh * nb + (iab.y >= 0 ? iab.y : iab.x)) * static_cast<long long>(nb);
+      wk.c0 = min(max(prm.list_cnt[bh * nb + iab.x], 0), nb);
+      wk.c1 = iab.y >= 0 ? min(max(prm.list_cnt[bh * nb + iab.y], 0), nb) : 0;
       wk.a = wk.b = 0;
       int it = 0;
       bool ended = false;
@@ -580,9 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++it;
       }
-      // Copies still in flight: the last kStages iterations, except that placing the end
-      // marker waited for the oldest of them to be consumed (its stage was reused), and a
-      // parity wait on that stage would now look two phases back.
+      // Copies still in flight (as in the dK/dV pass).
       const int keep = ended ? L::kStages - 1 : L::kStages;
       const int first = it > keep ? it - keep : 0;
       for (int x = first; x < it; ++x)
@@ -595,7 +602,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = idesc_f16_f32(128, 64, false, false);
       constexpr uint32_t idesc_acc = idesc_f16_f32(128, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
-      const uint32_t st_addr = smem_u32(sStage), ds_addr = smem_u32(sDS);
+      const uint32_t st_addr = smem_u32(sStage);
+      // S = Q K_j^T and dP = dO V_j^T into buffer x & 1
       auto issue_sd = [&](int x) {
         const int s = x % L::kStages;
         const uint32_t ka = st_addr + s * L::kStageBytes;
@@ -615,14 +623,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&sd_full[x & 1]);
       };
+      // dQ += dS K_j with dS read from TMEM (written over dP)
       auto issue_acc = [&](int x) {
         const int s = x % L::kStages;
         const uint32_t ka = st_addr + s * L::kStageBytes;
-        const uint32_t b = x & 1;
+        const uint32_t col = (x & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tmem + C::kColAcc0, sdesc_sw128(ds_addr + b * C::kPBytes + kk * 32, 16, 1024),
-                      sdesc_sw128(ka + kk * 2048, 8192, 1024), idesc_acc, (x > 0 || kk > 0));
+          mma_bf16_ts(tmem + C::kColAcc0, tmem + col + 64 + packed_col(kk), sdesc_sw128(ka + kk * 2048, 8192, 1024),
+                      idesc_acc, (x > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(q_full, 0, prm.status, kDevTimeoutQFull);
       if (ok) ok = mbar_wait(&full[0], 0, prm.status, kDevTimeoutTmaFull);
@@ -648,15 +657,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= kMathWarp0) {
-    const int row = threadIdx.x - kMathWarp0 * 32;
-    const uint32_t lane_base = static_cast<uint32_t>((warp - kMathWarp0) * 32) << 16;
+    // 8 warps: query row = TMEM lane, column half h of each 64-key tile
+    const int mw = warp - kMathWarp0;
+    const int h = mw >> 2;
+    const int row = (mw & 3) * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>((mw & 3) * 32) << 16;
     const bool upper = row >= 64;
-    const bool valid = upper ? has_i1 : true;
-    const long long tok = bh * prm.S + static_cast<long long>(i0) * 64 + row;
+    const int blk = upper ? iab.y : iab.x;
+    const bool valid = blk >= 0;
+    const long long tok = bh * prm.S + static_cast<long long>(valid ? blk : 0) * 64 + (row & 63);
     const float my_lse2 = valid ? prm.lse2[tok] : 0.f;
     const float my_delta = valid ? prm.delta[tok] : 0.f;
     const float sl2 = prm.scale_log2;
-    unsigned char* dsrow = sDS + row * 128;
     int it = 0;
     bool ok = true;
     for (;; ++it) {
@@ -669,35 +681,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[it & 1], (it >> 1) & 1, prm.status, kDevTimeoutSFull));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t col = (it & 1) * 128;
-      uint32_t dk[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      const uint32_t col = tmem + lane_base + (it & 1) * 128 + 32 * h;
+      uint32_t dk[16];
+      if (keep) {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tmem + lane_base + col + half * 32, sv);
-        tmem_ld32(tmem + lane_base + col + 64 + half * 32, dv);
+        tmem_ld32(col, sv);
+        tmem_ld32(col + 64, dv);
         tmem_wait_ld();
-        if (keep) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -my_lse2));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -my_lse2));
-            dk[half * 16 + (c >> 1)] = pack_f16x2(p0 * (__uint_as_float(dv[c]) - my_delta),
-                                                  p1 * (__uint_as_float(dv[c + 1]) - my_delta));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) dk[half * 16 + c] = 0u;
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -my_lse2));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -my_lse2));
+          dk[c >> 1] = pack_f16x2(p0 * (__uint_as_float(dv[c]) - my_delta),
+                                  p1 * (__uint_as_float(dv[c + 1]) - my_delta));
         }
-      }
-      const int b = it & 1;
+      } else {
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(dsrow + b * C::kPBytes + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
-      fence_proxy_async_smem();
+        for (int c = 0; c < 16; ++c) dk[c] = 0u;
+      }
+      tmem_st16(col + 64, dk);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[b]);
+      mbar_arrive(&p_full[it & 1]);
     }
     bool have = ok && it > 0;
     if (have) {
@@ -705,17 +710,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
     }
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = 0; c0 < D / 2; c0 += 32) {
       uint32_t ov[32];
       if (have) {
-        tmem_ld32(tmem + lane_base + C::kColAcc0 + c0, ov);
+        tmem_ld32(tmem + lane_base + C::kColAcc0 + (D / 2) * h + c0, ov);
         tmem_wait_ld();
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) ov[c] = 0u;
       }
       if (valid) {
-        float4* dst = reinterpret_cast<float4*>(prm.out0 + tok * D + c0);
+        float4* dst = reinterpret_cast<float4*>(prm.out0 + tok * D + (D / 2) * h + c0);
         const float mul = prm.scale;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -748,8 +753,11 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   uint32_t* status = static_cast<uint32_t*>(ws);
   int32_t* order_cols = nullptr;
   int32_t* order_rows = nullptr;
-  cudaError_t e = build_schedule(ccnt, nullptr, d, sched, &order_cols, st);
-  if (e == cudaSuccess) e = build_schedule(rcnt, nullptr, d, sched + schedule_scratch_bytes(d), &order_rows, st);
+  // key-block pairs and query-block pairs both follow tile_blocks() (same patch, frames
+  // 2u and 2u + 1), whose kept lists overlap most
+  cudaError_t e = build_schedule(ccnt, nullptr, d, sched, &order_cols, st, /*frame_pairs=*/true);
+  if (e == cudaSuccess)
+    e = build_schedule(rcnt, nullptr, d, sched + schedule_scratch_bytes(d), &order_rows, st, /*frame_pairs=*/true);
   if (e != cudaSuccess) return e;
   constexpr int kRowsPerCta = 8 * (256 / D);
   if (v_f16) v16 = static_cast<__half*>(const_cast<void*>(v));   // used as it is
@@ -759,10 +767,8 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
       do16, delta, lse2, rows, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128, mk64, mv64;
+  CUtensorMap mq64, mdo64, mk64, mv64;
   *map_ok = make_map_16(&mq64, q16, rows, D, 64, true) && make_map_16(&mdo64, do16, rows, D, 64, true) &&
-            make_map_16(&mk128, k16, rows, D, 128, true) && make_map_16(&mv128, v16, rows, D, 128, true) &&
-            make_map_16(&mq128, q16, rows, D, 128, true) && make_map_16(&mdo128, do16, rows, D, 128, true) &&
             make_map_16(&mk64, k16, rows, D, 64, true) && make_map_16(&mv64, v16, rows, D, 64, true);
   if (!*map_ok) return cudaErrorInvalidValue;
 
@@ -771,6 +777,8 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   p.lse2 = lse2;
   p.status = status;
   p.nb = d.nb;
+  p.T = d.T;
+  p.HW = d.Hb * d.Wb;
   p.S = d.S;
   p.scale_log2 = scale * kLog2e;
   p.scale = scale;
@@ -785,7 +793,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DkdvLayout<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk128, mv128, p);
+  attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk64, mv64, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   p.order = order_rows;
@@ -796,7 +804,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DqLayout<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kSmemBytes, st>>>(mq128, mdo128, mk64, mv64, p);
+  attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk64, mv64, p);
   return cudaGetLastError();
 }
 
