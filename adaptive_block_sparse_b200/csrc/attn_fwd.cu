@@ -491,13 +491,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           reg_fence32(c0);
           reg_fence32(c1);
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc) m8[cc & 7] = fmaxf(m8[cc & 7], __uint_as_float(sv[cc]));
+          for (int cc = 0; cc < 64; cc += 2)
+            m8[(cc >> 1) & 7] = fmax3(m8[(cc >> 1) & 7], __uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1]));
         }
         if (keep_b) {
           reg_fence32(c2);
           reg_fence32(c3);
 #pragma unroll
-          for (int cc = 64; cc < 128; ++cc) m8[cc & 7] = fmaxf(m8[cc & 7], __uint_as_float(sv[cc]));
+          for (int cc = 64; cc < 128; cc += 2)
+            m8[(cc >> 1) & 7] = fmax3(m8[(cc >> 1) & 7], __uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1]));
         }
         const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
