@@ -42,7 +42,7 @@ EXPORTED = (
     "nabla_status_string", "nabla_reorder", "nabla_mask_workspace_bytes", "nabla_build_mask",
     "nabla_mask_lists", "nabla_fwd_workspace_bytes", "nabla_attn_fwd",
     "nabla_bwd_workspace_bytes", "nabla_attn_bwd", "nabla_read_device_status",
-    "nabla_attn_fwd_noalloc",
+    "nabla_attn_fwd_noalloc", "nabla_build_mask_sweep",
 )
 
 
@@ -65,6 +65,8 @@ _sigs = {
     "nabla_build_mask": (ctypes.c_int, [_vp, _vp, _vp, _vp, _Shape, ctypes.c_double, _Window,
                                         ctypes.c_double, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "nabla_mask_lists": (ctypes.c_int, [_vp, _Shape, _vp, _vp, _vp, _vp, _vp]),
+    "nabla_build_mask_sweep": (ctypes.c_int, [_vp, _vp, _vp, _vp, _Shape, _vp, ctypes.c_int, _Window,
+                                              ctypes.c_double, _vp, _vp, _vp, _sz, _vp]),
     "nabla_fwd_workspace_bytes": (_sz, [_Shape]),
     "nabla_attn_fwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape, ctypes.c_float,
                                       _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _sz, _vp]),
@@ -204,6 +206,39 @@ def nabla_build_mask(q, k, shape: Shape, thr: float, window=(0, 0, 0), scale=Non
            "nabla_build_mask")
     del BH
     return mask_bits, row_idx, row_cnt, col_idx, col_cnt
+
+
+def nabla_build_mask_sweep(q, k, shape: Shape, thrs, window=(0, 0, 0), scale=None,
+                           mask_bits=None, row_cnt=None, counts=True, q_pool=None, k_pool=None,
+                           workspace=None, stream=None):
+    """NABLA block masks of several thresholds from one pooled map.
+
+    Returns (mask_bits [n_thr, B, H, nb, nw], row_cnt [n_thr, B, H, nb] or None).
+    """
+    thrs = [float(t) for t in thrs]
+    n = len(thrs)
+    dev = next(t.device for t in (q, q_pool, mask_bits, workspace) if t is not None)
+    if mask_bits is None:
+        mask_bits = torch.empty(n, shape.B, shape.H, shape.nb, shape.nw, dtype=torch.int32, device=dev)
+    if row_cnt is None and counts:
+        row_cnt = torch.empty(n, shape.B, shape.H, shape.nb, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(nabla_mask_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(shape.D)
+    arr = (ctypes.c_double * max(n, 1))(*thrs)
+    _check(load_library().nabla_build_mask_sweep(
+        _ptr(q), _ptr(k), _ptr(q_pool), _ptr(k_pool), shape.c(), ctypes.cast(arr, ctypes.c_void_p), n,
+        _Window(*window), float(scale), _ptr(mask_bits), _ptr(row_cnt), _ptr(workspace),
+        workspace.numel(), _stream(stream)), "nabla_build_mask_sweep")
+    return mask_bits, row_cnt
+
+
+def sparsity_curve(row_cnt, shape: Shape):
+    """Sparsity 1 - kept / (B*H*nb^2) of each mask of a sweep, from its row counts."""
+    kept = row_cnt.to(torch.int64).reshape(row_cnt.shape[0], -1).sum(dim=1)
+    total = shape.B * shape.H * shape.nb * shape.nb
+    return [1.0 - int(x) / total for x in kept.cpu()]
 
 
 def nabla_mask_lists(mask_bits, shape: Shape, row_idx=None, row_cnt=None, col_idx=None,

@@ -30,6 +30,11 @@ namespace nabla {
 cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st);
 size_t mask_fast_scratch_bytes(const Dims& d);
 bool mask_fast_supported(const Dims& d);
+cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d, double scale,
+                              void* scratch, uint32_t* status, cudaStream_t st);
+cudaError_t mask_fast_select(const Dims& d, double scale, double thr, const nabla_window& w,
+                             uint32_t* bits, int32_t* ridx, int32_t* rcnt, void* scratch,
+                             int32_t** rescue_list, int32_t** rescue_cnt, cudaStream_t st);
 cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, double scale, double thr,
                           const nabla_window& w, uint32_t* bits, int32_t* ridx, int32_t* rcnt,
                           void* scratch, uint32_t* status, int32_t** rescue_list,
@@ -428,6 +433,8 @@ cudaError_t launch_col_lists(const uint32_t* bits, const Dims& d, int32_t* cidx,
 
 using namespace nabla;
 
+constexpr int kMaxSweep = 64;   // thresholds per nabla_build_mask_sweep call
+
 extern "C" size_t nabla_mask_workspace_bytes(nabla_shape s) {
   Dims d;
   if (check_shape(s, &d) != NABLA_OK) return 0;
@@ -542,6 +549,103 @@ extern "C" nabla_status nabla_mask_lists(const uint32_t* mask_bits, nabla_shape 
   }
   if (col_cnt) {
     if ((e = launch_col_lists(mask_bits, d, col_idx, col_cnt, st)) != cudaSuccess) return cuda_status(e);
+  }
+  return NABLA_OK;
+}
+
+// Several thresholds on one pooled map: the pooled means and the pooled logits are
+// formed once, then the cut (and the fp64 rescue of the rows it cannot certify) runs per
+// threshold.  Mask t goes to mask_bits + t * (B*H*nb*nw), its per-row counts (optional)
+// to row_cnt + t * (B*H*nb).
+extern "C" nabla_status nabla_build_mask_sweep(const void* q, const void* k, const double* q_pool,
+                                               const double* k_pool, nabla_shape s,
+                                               const double* thrs, int n_thr, nabla_window sta,
+                                               double scale, uint32_t* mask_bits, int32_t* row_cnt,
+                                               void* workspace, size_t workspace_bytes,
+                                               nabla_stream_t stream) {
+  Dims d;
+  nabla_status rc = check_shape(s, &d);
+  if (rc != NABLA_OK) return rc;
+  if (!thrs || n_thr < 1 || n_thr > kMaxSweep) return NABLA_ERR_INVALID_ARG;
+  bool any_data = false;
+  for (int t = 0; t < n_thr; ++t) {
+    if (!(thrs[t] >= 0.0 && thrs[t] <= 1.0)) return NABLA_ERR_INVALID_ARG;   // also NaN
+    any_data = any_data || (thrs[t] > 0.0 && thrs[t] < 1.0);
+  }
+  if (!(scale > 0.0) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
+  const int sizes[3] = {sta.t, sta.h, sta.w};
+  const bool sta_off = sta.t == 0 && sta.h == 0 && sta.w == 0;
+  if (!sta_off)
+    for (int a = 0; a < 3; ++a)
+      if (sizes[a] < 1 || (sizes[a] % 2) == 0) return NABLA_ERR_INVALID_ARG;
+  if (!mask_bits || (reinterpret_cast<uintptr_t>(mask_bits) & 3)) return NABLA_ERR_INVALID_ARG;
+  if (row_cnt && (reinterpret_cast<uintptr_t>(row_cnt) & 3)) return NABLA_ERR_INVALID_ARG;
+  if (any_data) {
+    if (!q_pool && (!q || !aligned16(q))) return NABLA_ERR_INVALID_ARG;
+    if (!k_pool && (!k || !aligned16(k))) return NABLA_ERR_INVALID_ARG;
+    if ((q_pool && (reinterpret_cast<uintptr_t>(q_pool) & 7)) ||
+        (k_pool && (reinterpret_cast<uintptr_t>(k_pool) & 7)))
+      return NABLA_ERR_INVALID_ARG;
+  }
+  const size_t need = nabla_mask_workspace_bytes(s);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return NABLA_ERR_WORKSPACE;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long rows = static_cast<long long>(d.BH) * d.nb;
+  const size_t mask_words = static_cast<size_t>(rows) * d.nw;
+  const size_t pool_bytes = align_up(static_cast<size_t>(d.BH) * d.nb * d.D * sizeof(double), 256);
+  if (cudaMemsetAsync(workspace, 0, kStatusBytes, st) != cudaSuccess) return NABLA_ERR_CUDA;
+  cudaError_t e = cudaSuccess;
+  const double* qp = q_pool;
+  const double* kp = k_pool;
+  void* fast_scratch = static_cast<char*>(workspace) + kStatusBytes + 2 * pool_bytes;
+  const bool fast = mask_fast_supported(d);
+  if (any_data) {
+    double* qp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes);
+    double* kp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes + pool_bytes);
+    if (!qp) {
+      if ((e = pool_blocks_device(q, qp_ws, d, st)) != cudaSuccess) return cuda_status(e);
+      qp = qp_ws;
+    }
+    if (!kp) {
+      if ((e = pool_blocks_device(k, kp_ws, d, st)) != cudaSuccess) return cuda_status(e);
+      kp = kp_ws;
+    }
+    if (fast && (e = mask_fast_prepare(qp, kp, d, scale, fast_scratch, static_cast<uint32_t*>(workspace), st)) !=
+                    cudaSuccess)
+      return cuda_status(e);
+  }
+  for (int t = 0; t < n_thr; ++t) {
+    const double thr = thrs[t];
+    uint32_t* bits = mask_bits + t * mask_words;
+    int32_t* cnt = row_cnt ? row_cnt + t * static_cast<size_t>(rows) : nullptr;
+    if (thr <= 0.0 || thr >= 1.0) {
+      static_mask_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+          d.nb, d.nw, rows, thr >= 1.0 ? 1 : 0, sta_off ? 0 : 1, sta.t / 2, sta.h / 2, sta.w / 2,
+          d.Hb, d.Wb, bits);
+      if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+      if (cnt) {
+        row_lists_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(bits, d.nb, d.nw, rows,
+                                                                              nullptr, cnt);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+      }
+      continue;
+    }
+    const int32_t* rlist = nullptr;
+    const int32_t* rlist_cnt = nullptr;
+    if (fast) {
+      int32_t* rl = nullptr;
+      int32_t* rcn = nullptr;
+      if ((e = mask_fast_select(d, scale, thr, sta, bits, nullptr, cnt, fast_scratch, &rl, &rcn, st)) !=
+          cudaSuccess)
+        return cuda_status(e);
+      rlist = rl;
+      rlist_cnt = rcn;
+    }
+    e = d.D == 64 ? launch_mask_rows<64>(qp, kp, d, scale, thr, sta, bits, nullptr, cnt, rlist, rlist_cnt, st)
+                  : launch_mask_rows<128>(qp, kp, d, scale, thr, sta, bits, nullptr, cnt, rlist, rlist_cnt, st);
+    if (e != cudaSuccess) return cuda_status(e);
   }
   return NABLA_OK;
 }

@@ -478,45 +478,61 @@ size_t mask_fast_scratch_bytes(const Dims& d) {
 
 bool mask_fast_supported(const Dims& d) { return d.nb <= 2048; }
 
-// Runs tiers 1-2 (split, logits, certified select).  Rows that are not certified are
-// listed per head in rescue_list / rescue_cnt (returned) for the fp64 kernel.
-cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, double scale, double thr,
-                          const nabla_window& w, uint32_t* bits, int32_t* ridx, int32_t* rcnt,
-                          void* scratch, uint32_t* status, int32_t** rescue_list,
-                          int32_t** rescue_cnt, cudaStream_t st) {
+namespace {
+
+// Scratch layout of the fast tier (see mask_fast_scratch_bytes).
+struct FastScratch {
+  __half *qh, *ql, *kh, *kl;
+  float* qnorm;
+  uint32_t* kmax;
+  float* logits;
+  int32_t* rlist;
+  int32_t* rc;
+};
+
+FastScratch fast_scratch(const Dims& d, void* scratch) {
   const int nbp = mask_fast_nbp(d.nb);
   const size_t split = align_up(static_cast<size_t>(d.BH) * nbp * d.D * 2, 256);
   char* base = static_cast<char*>(scratch);
-  __half* qh = reinterpret_cast<__half*>(base);
-  __half* ql = reinterpret_cast<__half*>(base + split);
-  __half* kh = reinterpret_cast<__half*>(base + 2 * split);
-  __half* kl = reinterpret_cast<__half*>(base + 3 * split);
+  FastScratch f;
+  f.qh = reinterpret_cast<__half*>(base);
+  f.ql = reinterpret_cast<__half*>(base + split);
+  f.kh = reinterpret_cast<__half*>(base + 2 * split);
+  f.kl = reinterpret_cast<__half*>(base + 3 * split);
   char* c = base + 4 * split;
-  float* qnorm = reinterpret_cast<float*>(c);
+  f.qnorm = reinterpret_cast<float*>(c);
   c += align_up(static_cast<size_t>(d.BH) * d.nb * 4, 256);
-  uint32_t* kmax = reinterpret_cast<uint32_t*>(c);
+  f.kmax = reinterpret_cast<uint32_t*>(c);
   c += align_up(static_cast<size_t>(d.BH) * 4, 256);
-  float* logits = reinterpret_cast<float*>(c);
+  f.logits = reinterpret_cast<float*>(c);
   c += align_up(static_cast<size_t>(d.BH) * nbp * nbp * 4, 256);
-  int32_t* rlist = reinterpret_cast<int32_t*>(c);
+  f.rlist = reinterpret_cast<int32_t*>(c);
   c += align_up(static_cast<size_t>(d.BH) * d.nb * 4, 256);
-  int32_t* rc = reinterpret_cast<int32_t*>(c);
+  f.rc = reinterpret_cast<int32_t*>(c);
+  return f;
+}
 
-  cudaError_t e = cudaMemsetAsync(kmax, 0, static_cast<size_t>(d.BH) * 4, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(rc, 0, static_cast<size_t>(d.BH) * 4, st);
+}  // namespace
+
+// Tiers 1-2a: split of the pooled means and the pooled logits (independent of thr).
+cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d, double scale,
+                              void* scratch, uint32_t* status, cudaStream_t st) {
+  const int nbp = mask_fast_nbp(d.nb);
+  const FastScratch f = fast_scratch(d, scratch);
+  cudaError_t e = cudaMemsetAsync(f.kmax, 0, static_cast<size_t>(d.BH) * 4, st);
   if (e != cudaSuccess) return e;
   const long long rows_pad = static_cast<long long>(d.BH) * nbp;
   if (d.D == 64)
     split_pools_kernel<64><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, st>>>(
-        qp, kp, d.nb, nbp, rows_pad, qh, ql, kh, kl, qnorm, kmax);
+        qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax);
   else
     split_pools_kernel<128><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, st>>>(
-        qp, kp, d.nb, nbp, rows_pad, qh, ql, kh, kl, qnorm, kmax);
+        qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   CUtensorMap mqh, mql, mkh, mkl;
-  if (!(make_map_16(&mqh, qh, rows_pad, d.D, 128, true) && make_map_16(&mql, ql, rows_pad, d.D, 128, true) &&
-        make_map_16(&mkh, kh, rows_pad, d.D, 256, true) && make_map_16(&mkl, kl, rows_pad, d.D, 256, true)))
+  if (!(make_map_16(&mqh, f.qh, rows_pad, d.D, 128, true) && make_map_16(&mql, f.ql, rows_pad, d.D, 128, true) &&
+        make_map_16(&mkh, f.kh, rows_pad, d.D, 256, true) && make_map_16(&mkl, f.kl, rows_pad, d.D, 256, true)))
     return cudaErrorInvalidValue;
   dim3 grid(nbp / 128, nbp / 256, d.BH);
   if (d.D == 64) {
@@ -524,25 +540,36 @@ cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, dou
                              LogitCfg<64>::kSmemBytes);
     if (e != cudaSuccess) return e;
     pooled_logits_kernel<64><<<grid, 128, LogitCfg<64>::kSmemBytes, st>>>(
-        mqh, mql, mkh, mkl, logits, nbp, static_cast<float>(scale), status);
+        mqh, mql, mkh, mkl, f.logits, nbp, static_cast<float>(scale), status);
   } else {
     e = cudaFuncSetAttribute(pooled_logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              LogitCfg<128>::kSmemBytes);
     if (e != cudaSuccess) return e;
     pooled_logits_kernel<128><<<grid, 128, LogitCfg<128>::kSmemBytes, st>>>(
-        mqh, mql, mkh, mkl, logits, nbp, static_cast<float>(scale), status);
+        mqh, mql, mkh, mkl, f.logits, nbp, static_cast<float>(scale), status);
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
+// Tier 2b: the certified cut for one thr from the logits mask_fast_prepare wrote.  Rows
+// that are not certified are listed per head in rescue_list / rescue_cnt (returned) for
+// the fp64 kernel; the lists are rebuilt by every call.
+cudaError_t mask_fast_select(const Dims& d, double scale, double thr, const nabla_window& w,
+                             uint32_t* bits, int32_t* ridx, int32_t* rcnt, void* scratch,
+                             int32_t** rescue_list, int32_t** rescue_cnt, cudaStream_t st) {
+  const int nbp = mask_fast_nbp(d.nb);
+  const FastScratch f = fast_scratch(d, scratch);
+  cudaError_t e = cudaMemsetAsync(f.rc, 0, static_cast<size_t>(d.BH) * 4, st);
+  if (e != cudaSuccess) return e;
   SelectParams p;
-  p.logits = logits;
-  p.qnorm = qnorm;
-  p.kmax_bits = kmax;
+  p.logits = f.logits;
+  p.qnorm = f.qnorm;
+  p.kmax_bits = f.kmax;
   p.bits = bits;
   p.row_idx = ridx;
   p.row_cnt = rcnt;
-  p.rescue_list = rlist;
-  p.rescue_cnt = rc;
+  p.rescue_list = f.rlist;
+  p.rescue_cnt = f.rc;
   p.nb = d.nb;
   p.nbp = nbp;
   p.nw = d.nw;
@@ -567,9 +594,19 @@ cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, dou
     case 56: e = launch_select<56>(p, rows, st); break;
     default: e = launch_select<64>(p, rows, st); break;
   }
-  *rescue_list = rlist;
-  *rescue_cnt = rc;
+  *rescue_list = f.rlist;
+  *rescue_cnt = f.rc;
   return e;
+}
+
+// Runs tiers 1-2 (split, logits, certified select) for one thr.
+cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, double scale, double thr,
+                          const nabla_window& w, uint32_t* bits, int32_t* ridx, int32_t* rcnt,
+                          void* scratch, uint32_t* status, int32_t** rescue_list,
+                          int32_t** rescue_cnt, cudaStream_t st) {
+  cudaError_t e = mask_fast_prepare(qp, kp, d, scale, scratch, status, st);
+  if (e != cudaSuccess) return e;
+  return mask_fast_select(d, scale, thr, w, bits, ridx, rcnt, scratch, rescue_list, rescue_cnt, st);
 }
 
 }  // namespace nabla

@@ -466,6 +466,24 @@ def main():
                                row_idx=path.ridx, row_cnt=path.rcnt, workspace=path.mask_ws)
     mask_ms = time_call(mask_from_qk, 5)
     mask_bytes = 2 * BH * wl.S * wl.D * 2 + BH * nb * sh.nw * 4
+    # several thresholds from one pooled map (the pools of the step), against one mask
+    # call per threshold; the masks are the same bit for bit
+    sweep_thrs = (0.5, 0.7, 0.8, 0.9, 0.95)
+    sw_bits = torch.empty(len(sweep_thrs), wl.B, wl.H, nb, sh.nw, dtype=torch.int32, device=dev)
+    sw_cnt = torch.empty(len(sweep_thrs), wl.B, wl.H, nb, dtype=torch.int32, device=dev)
+    sweep_call = lambda: m.nabla_build_mask_sweep(None, None, sh, sweep_thrs, wl.window,
+                                                  mask_bits=sw_bits, row_cnt=sw_cnt, q_pool=path.qp,
+                                                  k_pool=path.kp, workspace=path.mask_ws)
+
+    def separate_calls():
+        for t, thr in enumerate(sweep_thrs):
+            m.nabla_build_mask(None, None, sh, thr, wl.window, mask_bits=sw_bits[t], row_cnt=sw_cnt[t],
+                               q_pool=path.qp, k_pool=path.kp, workspace=path.mask_ws)
+    sweep_ms = time_call(sweep_call, 3)
+    separate_ms = time_call(separate_calls, 3)
+    sweep = {"thrs": list(sweep_thrs), "ms": sweep_ms, "ms_separate_calls": separate_ms,
+             "sparsity": m.sparsity_curve(sw_cnt, sh)}
+    del sw_bits, sw_cnt
     # bytes of the pass before the mask: pooling of Q, K (natural path) or reorder of Q,
     # K, V with pooling (training path)
     reorder_bytes = (2 * BH * wl.S * wl.D * 2 if path.natural else 3 * 2 * BH * wl.S * wl.D * 2) \
@@ -542,7 +560,7 @@ def main():
         "dense_fwd_ms": dense_ms, "dense_tflops": dense_tflops, "speedup_vs_dense": dense_ms / fwd_ms,
         "mask_ms": mask_ms, "mask_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
         "mask_frac_hbm": mask_bytes / (mask_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-        "mask_ms_from_pools": mask_ms_fused, "reorder_ms": reorder_ms,
+        "mask_ms_from_pools": mask_ms_fused, "mask_sweep_from_pools": sweep, "reorder_ms": reorder_ms,
         "reorder_gbs": reorder_bytes / (reorder_ms * 1e-3) / 1e9,
         "bwd_ms": bwd_ms, "bwd_tflops_kept": bwd_tflops,
         "kept_tiles": kept, "sparsity": sparsity,

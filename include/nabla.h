@@ -134,6 +134,34 @@ nabla_status nabla_build_mask(const void *q, const void *k, const double *q_pool
                               int32_t *col_cnt, void *workspace, size_t workspace_bytes,
                               nabla_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Several thresholds on one pooled map ("mask reuse").
+ * The pages tune thr per model (lsdiaocha.cn article, section 3: thr 0.2-0.9 swept
+ * against quality and speed; gist.science, Chinese edition, "Experimental results":
+ * sparsity and quality per thr); this call builds the masks of n_thr thresholds from one
+ * computation of the pooled means and the pooled logits, the per-row cut (and its fp64
+ * check) running once per threshold.  Each mask is identical, bit for bit, to the one
+ * nabla_build_mask returns for that thr with the same inputs.
+ *
+ * q, k, q_pool,
+ * k_pool, sta,
+ * scale      : as nabla_build_mask (q, k and the pools may all be NULL when every thr is
+ *              <= 0 or >= 1).
+ * thrs       : host array of n_thr values in [0, 1]; 1 <= n_thr <= 64.
+ * mask_bits  : out uint32 [n_thr][B,H,nb,ceil(nb/32)]: mask t at offset
+ *              t * B*H*nb*ceil(nb/32) words.
+ * row_cnt    : out, nullable, int32 [n_thr][B,H,nb]: kept blocks per row of each mask
+ *              (row lists: nabla_mask_lists on a mask).
+ * workspace  : >= nabla_mask_workspace_bytes(s) bytes, 256-byte aligned (reused by the
+ *              thresholds one after another).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * --------------------------------------------------------------------------------- */
+nabla_status nabla_build_mask_sweep(const void *q, const void *k, const double *q_pool,
+                                    const double *k_pool, nabla_shape s, const double *thrs,
+                                    int n_thr, nabla_window sta, double scale,
+                                    uint32_t *mask_bits, int32_t *row_cnt, void *workspace,
+                                    size_t workspace_bytes, nabla_stream_t stream);
+
 /* Row and column lists of an arbitrary block mask (e.g. a dense all-ones mask for the
  * dense comparator, or a caller-made mask).  Same layouts as nabla_build_mask; any of
  * the two list pairs may be NULL.  Padding bits of mask_bits are ignored. */

@@ -96,6 +96,21 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert bm(wsb=ws_need - 1) == WS
     assert bm(ws=None) == WS
     assert bm(ws=ctypes.c_void_p(0x20000010)) == WS                       # misaligned workspace
+    thr3 = (ctypes.c_double * 3)(0.5, 0.8, 0.95)
+
+    def sw(thrs=thr3, n=3, window=win, bits=A, ws=Bp, wsb=ws_need, qp=A):
+        return lib.nabla_build_mask_sweep(None, None, qp, qp, good, ctypes.cast(thrs, ctypes.c_void_p)
+                                          if thrs is not None else None, n, window, 0.125, bits, None,
+                                          ws, wsb, st)
+    assert sw(n=0) == INV
+    assert sw(n=65) == INV
+    assert sw(thrs=None) == INV
+    assert sw(thrs=(ctypes.c_double * 3)(0.5, 1.5, 0.8)) == INV              # thr out of range
+    assert sw(thrs=(ctypes.c_double * 3)(0.5, float("nan"), 0.8)) == INV
+    assert sw(window=nb._Window(2, 3, 3)) == INV
+    assert sw(bits=None) == INV
+    assert sw(qp=None) == INV                                                  # no Q, K, nor pools
+    assert sw(wsb=ws_need - 1) == WS
     fws = lib.nabla_fwd_workspace_bytes(good)
 
     def fwd(q=A, o=Bp, scale=0.125, odt=0, ws=Bp, wsb=fws, ridx=A, vdt=0, layout=0):

@@ -104,6 +104,44 @@ def test_mask_without_data():
         assert np.array_equal(rcnt.cpu().numpy(), gm.sum(-1))
 
 
+@pytest.mark.parametrize("name,window", [("small", (0, 0, 0)), ("small", (3, 1, 3)), ("odd", (0, 0, 0)),
+                                         ("wide", (0, 0, 0))])
+def test_mask_sweep(data, name, window):
+    """Several thresholds from one pooled map: each mask equals the single-threshold call
+    bit for bit, matches the oracle outside the 1e-6 band, and the masks nest in thr."""
+    m = nbl()
+    wl = _wl(name)
+    shape = shape_of(wl)
+    q, k, _ = data(wl)
+    _, qp = gpu_reorder(q, shape, pool=True)
+    _, kp = gpu_reorder(k, shape, pool=True)
+    thrs = (0.0, 0.3, 0.5, 0.8, 0.95, 1.0)
+    bits, cnt = m.nabla_build_mask_sweep(None, None, shape, thrs, window, q_pool=qp, k_pool=kp)
+    torch.cuda.synchronize()
+    assert bits.shape[0] == len(thrs) and cnt.shape[0] == len(thrs)
+    prev = None
+    curve = m.sparsity_curve(cnt, shape)
+    for t, thr in enumerate(thrs):
+        one, *_ = gpu_mask(None, None, shape, thr, window, cols=False, q_pool=qp, k_pool=kp)
+        assert torch.equal(bits[t], one), thr
+        gm = bits_to_mask(bits[t], wl.nb)
+        assert np.array_equal(cnt[t].cpu().numpy(), gm.sum(-1))
+        assert abs(curve[t] - (1 - gm.mean())) < 1e-12
+        if 0.0 < thr < 1.0:
+            om, E = oracle_mask_per_head(q.cpu(), k.cpu(), wl, thr, window)
+            check_mask(gm, om, E, thr)
+        if prev is not None:
+            assert not np.any(prev & ~gm), thr          # a larger thr keeps a superset
+        prev = gm
+    print(f"{name} sta={window}: sparsity per thr {[round(c, 4) for c in curve]}")
+    # the sweep from bf16 Q, K (pooled inside) gives the same masks
+    qf, _ = gpu_reorder(q, shape)
+    kf, _ = gpu_reorder(k, shape)
+    bits2, _ = m.nabla_build_mask_sweep(qf, kf, shape, thrs, window)
+    torch.cuda.synchronize()
+    assert torch.equal(bits2, bits)
+
+
 @pytest.mark.parametrize("name,thr,window", MASK_CASES)
 def test_mask_parity(data, name, thr, window):
     wl = _wl(name)
