@@ -70,3 +70,75 @@ def test_reference_arm_torchrun_world2():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+
+
+# ---- head-sharded attention for sequence-sharded callers (two gloo ranks) -------------------
+
+def _oracle_heads(q, k, v, shape, thr, window, scale):
+    """The hot path on a rank's heads, computed by the oracle (fp64, natural order in/out)."""
+    import numpy as np
+    import oracle
+    T, Hg, W, P = shape.T, shape.Hg, shape.W, shape.P
+    out = torch.empty(q.shape, dtype=torch.float64)
+    for b in range(q.shape[0]):
+        for h in range(q.shape[1]):
+            qf, kf, vf = (oracle.reorder(x[b, h].double().numpy()[None, None], T, Hg, W, P)
+                          for x in (q, k, v))
+            mk, _, _ = oracle.nabla_mask(qf, kf, T, Hg, W, P, thr, window, scale=scale)
+            o, _ = oracle.block_sparse_attention(qf, kf, vf, mk, P * P, scale)
+            out[b, h] = torch.from_numpy(oracle.inverse_reorder(o, T, Hg, W, P)[0, 0])
+    return out
+
+
+def _sharded_worker(rank, world, port, wl_args, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from adaptive_block_sparse_b200 import sharding
+    from synth import Workload, make_qkv
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    wl = Workload(**wl_args)
+    q, k, v = make_qkv(wl)
+    s = wl.S // world
+    mine = slice(rank * s, (rank + 1) * s)       # this rank's contiguous token range
+    x = [t[:, :, mine].contiguous() for t in (q, k, v)]
+    # the two exchanges alone: a round trip returns the input, and the head shard holds
+    # every token of the rank's heads
+    heads = sharding.seq_to_heads(x[0])
+    hpr = wl.H // world
+    assert torch.equal(heads, q[:, rank * hpr:(rank + 1) * hpr])
+    assert torch.equal(sharding.heads_to_seq(heads), x[0])
+    o = sharding.sharded_nabla_attention(*x, wl.T, wl.Hg, wl.W, wl.thrs[0], wl.window,
+                                         compute=_oracle_heads)
+    out.put((rank, o))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("wl_args", [
+    dict(name="sh_a", B=1, H=2, T=2, Hg=16, W=16, D=64, thrs=(0.8,), seed=1101),
+    dict(name="sh_b", B=2, H=4, T=2, Hg=16, W=8, D=64, thrs=(0.6,), window=(1, 1, 1), seed=1102),
+])
+def test_sharded_attention_gloo_world2(wl_args):
+    """Sequence-sharded inputs -> all-to-all to head shards -> per-head path -> all-to-all
+    back: equals the unsharded computation exactly."""
+    import math
+    from adaptive_block_sparse_b200 import Shape
+    from synth import Workload, make_qkv
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, 2, port, wl_args, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(out.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    wl = Workload(**wl_args)
+    q, k, v = make_qkv(wl)
+    shape = Shape(wl.B, wl.H, wl.T, wl.Hg, wl.W, wl.D)
+    ref = _oracle_heads(q, k, v, shape, wl.thrs[0], wl.window, 1 / math.sqrt(wl.D))
+    got = torch.cat([res[0], res[1]], dim=2)
+    assert torch.equal(got, ref)
