@@ -54,7 +54,11 @@ struct FwdCfg {
   static constexpr int kSlotBytes = 3 * kTileBytes;       // Q, K pair, V pair
   static constexpr int kOffMeta = 2 * kSlotBytes;         // [2 slots][kMetaRing][kMetaInts]
   static constexpr int kOffBar = kOffMeta + 2 * kMetaRing * kMetaInts * 4;
-  static constexpr int kSmemBytes = kOffBar + 512 + 1024;
+  // bf16 O staging for the epilogue's tiled stores: per softmax warp 32 rows x 128 bytes
+  // (64 dims), 1 KB aligned for the 128-byte swizzle
+  static constexpr int kOffOStage = (kOffBar + 512 + 1023) / 1024 * 1024;
+  static constexpr int kOStageWarpBytes = 32 * 128;
+  static constexpr int kSmemBytes = kOffOStage + 8 * kOStageWarpBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   // slot s: score buffer at column 128 s, accumulator at column 256 + 128 s
   static __device__ __forceinline__ uint32_t col_s(int s) { return static_cast<uint32_t>(s) * 128u; }
@@ -155,7 +159,8 @@ template <int D, bool VF16, bool NAT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k,
-                    const __grid_constant__ CUtensorMap map_v, const FwdParams prm) {
+                    const __grid_constant__ CUtensorMap map_v,
+                    const __grid_constant__ CUtensorMap map_o, const FwdParams prm) {
   using C = FwdCfg<D>;
   constexpr int R = kMetaRing;
   extern __shared__ unsigned char smem_raw[];
@@ -623,17 +628,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&B.o_free);
-        if (valid_row) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.o) + tok * D);
+        // Each warp stages its 32 rows, 64 dims at a time, in the 128-byte-swizzled layout
+        // of a tiled copy and one lane stores them with TMA (32 rows x 128 bytes per copy:
+        // a 4 x 8 token part of the patch, or 32 consecutive reordered rows), instead of
+        // 16-byte stores scattered over 32 rows.
+        const int wq = (warp - kSoftmaxWarp0) & 3;
+        unsigned char* stage = smem + C::kOffOStage + ((warp - kSoftmaxWarp0) >> 2) * 4 * C::kOStageWarpBytes +
+                               wq * C::kOStageWarpBytes;
+        const int r32 = row & 31;
 #pragma unroll
-          for (int cc = 0; cc < D / 8; ++cc)
-            dst[cc] = make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2], packed[4 * cc + 3]);
+        for (int half = 0; half < D / 64; ++half) {
+          if (lane == 0) bulk_wait_read_all();     // the previous copy has read the staging
+          __syncwarp();
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(stage + r32 * 128 + ((ch ^ (r32 & 7)) << 4)) =
+                make_uint4(packed[32 * half + 4 * ch], packed[32 * half + 4 * ch + 1],
+                           packed[32 * half + 4 * ch + 2], packed[32 * half + 4 * ch + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && valid_row) {             // warp-uniform: a warp's rows are one block
+            if constexpr (NAT) {
+              const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+              tma_store_4d(&map_o, stage, 64 * half, wb * 8, hb * 8 + 4 * (wq & 1), t.bh * prm.T + tf);
+            } else {
+              tma_store_2d(&map_o, stage, 64 * half,
+                           static_cast<int>(static_cast<long long>(t.bh) * prm.S + static_cast<long long>(blk) * 64 +
+                                            32 * (wq & 1)));
+            }
+            bulk_commit_group();
+          }
         }
       }
       if (valid_row && prm.lse != nullptr)
         prm.lse[tok] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       mbar_arrive(&B.meta_empty[c % R]);
     }
+    if (lane == 0) bulk_wait_all();   // the epilogue's O copies have landed
+    __syncwarp();
   }
   // ------------------------------------------------------------------ teardown
   tc_fence_before();
@@ -682,14 +714,17 @@ bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int 
 // box = 64 channels x 8 columns x 8 rows x 1 frame (one P x P patch = one block),
 // 128-byte swizzle: the box lands as 64 rows of 128 bytes in the patch's row-major order,
 // the order of the reordered layout.
-bool make_map_nat(CUtensorMap* map, const void* base, long long frames, int Hg, int W, int D, bool fp16) {
+bool make_map_nat(CUtensorMap* map, const void* base, long long frames, int Hg, int W, int D, bool fp16,
+                  int box_h = 8);
+bool make_map_nat(CUtensorMap* map, const void* base, long long frames, int Hg, int W, int D, bool fp16,
+                  int box_h) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(W),
                         static_cast<cuuint64_t>(Hg), static_cast<cuuint64_t>(frames)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(W) * D * 2,
                            static_cast<cuuint64_t>(Hg) * W * D * 2};
-  cuuint32_t box[4] = {64u, 8u, 8u, 1u};
+  cuuint32_t box[4] = {64u, 8u, static_cast<cuuint32_t>(box_h), 1u};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   CUresult r = enc(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -702,7 +737,7 @@ namespace {
 template <int D, bool VF16, bool NAT>
 cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& d,
                        const FwdParams& prm, cudaStream_t st, bool* map_ok, bool* regs_ok) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const long long rows = static_cast<long long>(d.BH) * d.S;
   const long long frames = static_cast<long long>(d.BH) * d.T;
   if constexpr (NAT) {
@@ -713,6 +748,12 @@ cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& 
     *map_ok = make_map_16(&mq, q, rows, D, 64, false) && make_map_16(&mk, k, rows, D, 64, false) &&
               make_map_16(&mv, v, rows, D, 64, VF16);   // one 64-row block per copy
   }
+  // bf16 O: tiled stores of 32-row parts (an f32 O is stored directly; the map is unused)
+  if (*map_ok && !prm.o_f32)
+    *map_ok = NAT ? make_map_nat(&mo, prm.o, frames, d.Hg, d.W, D, false, 4)
+                  : make_map_16(&mo, prm.o, rows, D, 32, false);
+  else
+    mo = mq;
   if (!*map_ok) return cudaErrorInvalidValue;
   using C = FwdCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, VF16, NAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -730,7 +771,7 @@ cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& 
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = prm.items < sms ? prm.items : sms;
-  attn_fwd_kernel<D, VF16, NAT><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, prm);
+  attn_fwd_kernel<D, VF16, NAT><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mo, prm);
   return cudaGetLastError();
 }
 }  // namespace
