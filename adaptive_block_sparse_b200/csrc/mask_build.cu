@@ -45,7 +45,6 @@ namespace {
 constexpr int kThreads = 256;   // 8 warps; one pooled row per warp during selection
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
-constexpr int kRescueCtasPerHead = 64;
 constexpr int kCand = 16;       // the cut's bisection stops at this many candidates
 
 template <int D>
@@ -53,9 +52,11 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
     const double* __restrict__ qpool, const double* __restrict__ kpool, int nb, int nw, int R,
     double scale, double thr, int sta_on, int wt2, int wh2, int ww2, int Hb, int Wb,
     uint32_t* __restrict__ bits, int32_t* __restrict__ row_idx, int32_t* __restrict__ row_cnt,
-    const int32_t* __restrict__ rlist, const int32_t* __restrict__ rlist_cnt) {
-  // Rows: R consecutive rows from blockIdx.x * R, or (rlist != nullptr) the head's listed
-  // rows rlist[bh*nb + ...], taken R at a time by the CTAs of the head in turn.
+    const int32_t* __restrict__ rlist, const int32_t* __restrict__ rlist_cnt, int BH) {
+  // Rows: R consecutive rows from blockIdx.x * R of head blockIdx.y, or (rlist != nullptr)
+  // the listed rows: group g of head h = rows rlist[h*nb + gR ...], R at a time; the
+  // groups of all heads are numbered head after head and CTA c takes every gridDim.x-th
+  // one from c, so a few heads with many listed rows spread over every SM.
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int rows_s[8];
   __shared__ unsigned long long cand_key[kWarps * kCand];   // per warp: cut candidates
@@ -67,15 +68,27 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const long long bh = blockIdx.y;
-  const int listed = rlist != nullptr ? min(max(rlist_cnt[bh], 0), nb) : 0;
-  for (int g = rlist != nullptr ? blockIdx.x : 0;; g += gridDim.x) {
-  int nrows;
+  long long bh = blockIdx.y;
+  int listed = 0;
+  int hh = -1;                    // rescue mode: head of the current group,
+  long long hbase = 0, hnext = 0; // whose groups are [hbase, hnext) in the global numbering
+  for (long long u = rlist != nullptr ? blockIdx.x : 0;; u += gridDim.x) {
+  int nrows, g;
   if (rlist != nullptr) {
-    if (g * R >= listed) break;
+    while (u >= hnext && hh < BH) {
+      ++hh;
+      if (hh >= BH) break;
+      listed = min(max(rlist_cnt[hh], 0), nb);
+      hbase = hnext;
+      hnext += (listed + R - 1) / R;
+    }
+    if (hh >= BH) break;
+    bh = hh;
+    g = static_cast<int>(u - hbase);
     nrows = min(R, listed - g * R);
   } else {
-    if (g > 0) break;
+    if (u > 0) break;
+    g = 0;
     nrows = min(R, nb - static_cast<int>(blockIdx.x) * R);
   }
   __syncthreads();
@@ -405,11 +418,14 @@ cudaError_t launch_mask_rows(const double* qp, const double* kp, const Dims& d, 
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int sta_on = (w.t | w.h | w.w) != 0;
-  // Listed rows: a few CTAs per head take the head's rows R at a time.
-  dim3 grid(rlist != nullptr ? kRescueCtasPerHead : (d.nb + R - 1) / R, d.BH);
+  // Listed rows: one CTA per SM walks the groups of every head (the counts are on the
+  // device); all rows: one CTA per group of R rows of each head.
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  dim3 grid(rlist != nullptr ? sms : (d.nb + R - 1) / R, rlist != nullptr ? 1 : d.BH);
   mask_rows_kernel<D><<<grid, kThreads, smem, st>>>(qp, kp, d.nb, d.nw, R, scale, thr, sta_on,
                                                    w.t / 2, w.h / 2, w.w / 2, d.Hb, d.Wb, bits,
-                                                   ridx, rcnt, rlist, rlist_cnt);
+                                                   ridx, rcnt, rlist, rlist_cnt, d.BH);
   return cudaGetLastError();
 }
 

@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm
   } else {
     // Fast path: take maxima in descending order (ties: lower block index first) while
     // the running mass is below thr; most rows keep only a few blocks.
-    constexpr int kMaxExtract = 8;
+    constexpr int kMaxExtract = 16;
     uint64_t taken = 0;                 // bit t: p[t] of this lane already taken
     float acc = 0.f, acc_prev = 0.f;
     bool found = false;
