@@ -585,7 +585,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         tok = static_cast<long long>(t.bh) * prm.S + static_cast<long long>(valid_row ? blk : 0) * 64 + (row & 63);
       }
+      // Each warp stages its 32 rows, 128 bytes of each at a time (64 bf16 or 32 f32 dims),
+      // in the 128-byte-swizzled layout of a tiled copy, and one lane stores them with TMA
+      // (a 4 x 8 token part of the patch, or 32 consecutive reordered rows), instead of
+      // 16-byte stores scattered over 32 rows.
+      const int wq = (warp - kSoftmaxWarp0) & 3;
+      unsigned char* stage = smem + C::kOffOStage + ((warp - kSoftmaxWarp0) >> 2) * 4 * C::kOStageWarpBytes +
+                             wq * C::kOStageWarpBytes;
+      const int r32 = row & 31;
+      // stage 8 x 16 bytes of this row, then one lane copies the warp's 32 rows to
+      // columns [x0, x0 + 128 bytes) of O
+      auto stage_and_store = [&](const uint4 (&ch8)[8], int x0) {
+        if (lane == 0) bulk_wait_read_all();       // the previous copy has read the staging
+        __syncwarp();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(stage + r32 * 128 + ((ch ^ (r32 & 7)) << 4)) = ch8[ch];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && valid_row) {               // warp-uniform: a warp's rows are one block
+          if constexpr (NAT) {
+            const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+            tma_store_4d(&map_o, stage, x0, wb * 8, hb * 8 + 4 * (wq & 1), t.bh * prm.T + tf);
+          } else {
+            tma_store_2d(&map_o, stage, x0,
+                         static_cast<int>(static_cast<long long>(t.bh) * prm.S + static_cast<long long>(blk) * 64 +
+                                          32 * (wq & 1)));
+          }
+          bulk_commit_group();
+        }
+      };
       if (prm.o_f32) {
+        // 32 dims per copy; the accumulator is released after its last columns are read
 #pragma unroll 1
         for (int d0 = 0; d0 < D; d0 += 32) {
           uint32_t a0[32];
@@ -597,16 +628,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int cc = 0; cc < 32; ++cc) a0[cc] = 0u;
           }
-          if (valid_row) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(prm.o) + tok * D + d0);
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-              dst[cc] = make_float4(__uint_as_float(a0[4 * cc]) * inv, __uint_as_float(a0[4 * cc + 1]) * inv,
-                                    __uint_as_float(a0[4 * cc + 2]) * inv, __uint_as_float(a0[4 * cc + 3]) * inv);
+          if (d0 + 32 == D) {
+            tc_fence_before();
+            mbar_arrive(&B.o_free);
           }
+          uint4 ch8[8];
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc)
+            ch8[cc] = make_uint4(__float_as_uint(__uint_as_float(a0[4 * cc]) * inv),
+                                 __float_as_uint(__uint_as_float(a0[4 * cc + 1]) * inv),
+                                 __float_as_uint(__uint_as_float(a0[4 * cc + 2]) * inv),
+                                 __float_as_uint(__uint_as_float(a0[4 * cc + 3]) * inv));
+          stage_and_store(ch8, d0);
         }
-        tc_fence_before();
-        mbar_arrive(&B.o_free);
       } else {
         // bf16 output: the whole row is read and packed first (D / 2 registers), so that the
         // next tile's P V may overwrite the accumulator while the row is being stored.
@@ -628,36 +662,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&B.o_free);
-        // Each warp stages its 32 rows, 64 dims at a time, in the 128-byte-swizzled layout
-        // of a tiled copy and one lane stores them with TMA (32 rows x 128 bytes per copy:
-        // a 4 x 8 token part of the patch, or 32 consecutive reordered rows), instead of
-        // 16-byte stores scattered over 32 rows.
-        const int wq = (warp - kSoftmaxWarp0) & 3;
-        unsigned char* stage = smem + C::kOffOStage + ((warp - kSoftmaxWarp0) >> 2) * 4 * C::kOStageWarpBytes +
-                               wq * C::kOStageWarpBytes;
-        const int r32 = row & 31;
 #pragma unroll
         for (int half = 0; half < D / 64; ++half) {
-          if (lane == 0) bulk_wait_read_all();     // the previous copy has read the staging
-          __syncwarp();
+          uint4 ch8[8];
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4*>(stage + r32 * 128 + ((ch ^ (r32 & 7)) << 4)) =
-                make_uint4(packed[32 * half + 4 * ch], packed[32 * half + 4 * ch + 1],
-                           packed[32 * half + 4 * ch + 2], packed[32 * half + 4 * ch + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && valid_row) {             // warp-uniform: a warp's rows are one block
-            if constexpr (NAT) {
-              const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
-              tma_store_4d(&map_o, stage, 64 * half, wb * 8, hb * 8 + 4 * (wq & 1), t.bh * prm.T + tf);
-            } else {
-              tma_store_2d(&map_o, stage, 64 * half,
-                           static_cast<int>(static_cast<long long>(t.bh) * prm.S + static_cast<long long>(blk) * 64 +
-                                            32 * (wq & 1)));
-            }
-            bulk_commit_group();
-          }
+            ch8[ch] = make_uint4(packed[32 * half + 4 * ch], packed[32 * half + 4 * ch + 1],
+                                 packed[32 * half + 4 * ch + 2], packed[32 * half + 4 * ch + 3]);
+          stage_and_store(ch8, 64 * half);
         }
       }
       if (valid_row && prm.lse != nullptr)
@@ -733,6 +745,34 @@ bool make_map_nat(CUtensorMap* map, const void* base, long long frames, int Hg, 
   return r == CUDA_SUCCESS;
 }
 
+// f32 O maps for the epilogue's stores: box = 32 floats (128 bytes) x 32 rows, or x 8
+// columns x 4 rows x 1 frame of a natural-order tensor; 128-byte swizzle.
+bool make_map_f32(CUtensorMap* map, const void* base, long long rows, int D) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 4};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_nat_f32(CUtensorMap* map, const void* base, long long frames, int Hg, int W, int D) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(W),
+                        static_cast<cuuint64_t>(Hg), static_cast<cuuint64_t>(frames)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(W) * D * 4,
+                           static_cast<cuuint64_t>(Hg) * W * D * 4};
+  cuuint32_t box[4] = {32u, 8u, 4u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 template <int D, bool VF16, bool NAT>
 cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& d,
@@ -748,12 +788,12 @@ cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& 
     *map_ok = make_map_16(&mq, q, rows, D, 64, false) && make_map_16(&mk, k, rows, D, 64, false) &&
               make_map_16(&mv, v, rows, D, 64, VF16);   // one 64-row block per copy
   }
-  // bf16 O: tiled stores of 32-row parts (an f32 O is stored directly; the map is unused)
-  if (*map_ok && !prm.o_f32)
-    *map_ok = NAT ? make_map_nat(&mo, prm.o, frames, d.Hg, d.W, D, false, 4)
-                  : make_map_16(&mo, prm.o, rows, D, 32, false);
-  else
-    mo = mq;
+  // O: tiled stores of 32-row parts, 128 bytes of each row per copy
+  if (*map_ok)
+    *map_ok = prm.o_f32 ? (NAT ? make_map_nat_f32(&mo, prm.o, frames, d.Hg, d.W, D)
+                               : make_map_f32(&mo, prm.o, rows, D))
+                        : (NAT ? make_map_nat(&mo, prm.o, frames, d.Hg, d.W, D, false, 4)
+                               : make_map_16(&mo, prm.o, rows, D, 32, false));
   if (!*map_ok) return cudaErrorInvalidValue;
   using C = FwdCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, VF16, NAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -206,7 +206,8 @@ def test_fwd_parity(data, name, thr, window, o_dtype, v_dtype):
                                              ("small", 0.5, (1, 3, 3)), ("odd", 0.8, (0, 0, 0)),
                                              ("odd64", 0.6, (0, 0, 0))])
 @pytest.mark.parametrize("v_dtype", ["f16", "bf16"])
-def test_fwd_natural_layout(data, name, thr, window, v_dtype):
+@pytest.mark.parametrize("o_dtype", ["f32", "bf16"])
+def test_fwd_natural_layout(data, name, thr, window, v_dtype, o_dtype):
     """Natural-order q, k, v in, natural-order O and LSE out (the reorder done by the
     kernel's loads); same mask, compared with the oracle's output in natural order."""
     m = nbl()
@@ -220,17 +221,17 @@ def test_fwd_natural_layout(data, name, thr, window, v_dtype):
     vn = v.half() if v_dtype == "f16" else v
     lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
     ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
-    o, _ = m.nabla_attn_fwd(q, k, vn, bits, shape, o_dtype=m.NABLA_F32, lse=lse, workspace=ws,
-                            layout=m.NABLA_LAYOUT_NATURAL)
+    o, _ = m.nabla_attn_fwd(q, k, vn, bits, shape, o_dtype=m.NABLA_F32 if o_dtype == "f32" else m.NABLA_BF16,
+                            lse=lse, workspace=ws, layout=m.NABLA_LAYOUT_NATURAL)
     torch.cuda.synchronize()
     assert m.nabla_read_device_status(ws) == 0
     gm = bits_to_mask(bits, wl.nb)
     O, L = oracle.block_sparse_attention(to64(qf), to64(kf), to64(vf), gm, wl.N, 1 / math.sqrt(wl.D))
     On = oracle.inverse_reorder(O, wl.T, wl.Hg, wl.W, wl.P)
     Ln = oracle.inverse_reorder(L[..., None], wl.T, wl.Hg, wl.W, wl.P)[..., 0]
-    mx, mean = check_close(to64(o), On, f"O natural {name}")
+    mx, mean = check_close(to64(o), On, f"O natural {name}", storage_bf16=o_dtype == "bf16")
     check_lse(lse.cpu().numpy().astype(np.float64), Ln)
-    print(f"natural {name} thr={thr} V {v_dtype}: max err {mx:.2e} mean err {mean:.2e}")
+    print(f"natural {name} thr={thr} V {v_dtype} O {o_dtype}: max err {mx:.2e} mean err {mean:.2e}")
 
 
 def test_fwd_dense_and_empty_rows(data):
