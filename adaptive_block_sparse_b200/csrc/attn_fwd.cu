@@ -11,7 +11,8 @@
 //    step (N = 128 keys per MMA); a half of the rows whose block does not keep a key
 //    block is masked (-inf);
 //  * persistent: one CTA per SM runs two independent pipelines ("slots"), each taking
-//    tiles in a head-major, longest-first order through an atomic counter.  A slot owns
+//    tiles through an atomic counter in the schedule's order (heads by their longest
+//    tile, tiles longest first inside a head).  A slot owns
 //    a Q buffer, one K and one V stage, a TMEM score buffer and a TMEM accumulator; per
 //    step its chain is S = Q K^T (tcgen05.mma) -> softmax -> O += P V with P read from
 //    TMEM.  The two chains share the tensor core: while one slot runs its softmax, the
@@ -22,7 +23,8 @@
 //    a softmax warpgroup (one query row per thread, TMEM lane = row) holds a whole row
 //    of 128 scores in registers, rescales O only when a row maximum grows by more than
 //    2^8, rounds P to the V operand's 16-bit type (the row sum takes the rounded
-//    weights), and at the end of the tile normalises and stores O and the LSE;
+//    weights), and at the end of the tile normalises O, releases the accumulator and
+//    writes O through a shared-memory staging area with tiled TMA stores, and the LSE;
 //  * the producer warps give registers to the softmax warpgroups (setmaxnreg);
 //  * every barrier wait is bounded; on a timeout a kernel records a status code, stops,
 //    drains its own copies and MMAs and frees TMEM.
