@@ -42,7 +42,7 @@ EXPORTED = (
     "nabla_status_string", "nabla_reorder", "nabla_mask_workspace_bytes", "nabla_build_mask",
     "nabla_mask_lists", "nabla_fwd_workspace_bytes", "nabla_attn_fwd",
     "nabla_bwd_workspace_bytes", "nabla_attn_bwd", "nabla_read_device_status",
-    "nabla_attn_fwd_noalloc", "nabla_build_mask_sweep",
+    "nabla_attn_fwd_noalloc", "nabla_build_mask_sweep", "nabla_selftest_bounded_wait",
 )
 
 
@@ -75,6 +75,7 @@ _sigs = {
                                       _vp, _vp, _vp, _Shape, ctypes.c_float, _vp, _vp, _vp, _vp,
                                       _sz, _vp]),
     "nabla_read_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
+    "nabla_selftest_bounded_wait": (ctypes.c_int, [_vp, _sz, _vp]),
     "nabla_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape,
                                               ctypes.c_float, _vp, ctypes.c_int, _vp, ctypes.c_int,
                                               _vp]),
@@ -311,6 +312,16 @@ def nabla_read_device_status(workspace, stream=None) -> int:
     if rc not in (NABLA_OK, NABLA_ERR_DEVICE_CHECK):
         raise NablaError(rc, "nabla_read_device_status")
     return int(code.value)
+
+
+def nabla_selftest_bounded_wait(workspace, stream=None):
+    """Enqueue the failure-path self-test (a bounded wait that must give up); read the
+    outcome with nabla_read_device_status (expected code: DEVICE_TIMEOUT_SELFTEST)."""
+    _check(load_library().nabla_selftest_bounded_wait(_ptr(workspace), workspace.numel(), _stream(stream)),
+           "nabla_selftest_bounded_wait")
+
+
+DEVICE_TIMEOUT_SELFTEST = 0x10A
 
 
 # ---------------------------------------------------------------------------------------

@@ -63,3 +63,32 @@ extern "C" nabla_status nabla_read_device_status(void* workspace, uint32_t* code
   }
   return NABLA_OK;
 }
+
+namespace {
+
+// One warp waits, through the bounded wait every kernel uses, for a barrier phase that
+// nothing completes (the barrier expects one arrival and none is made): the wait gives up
+// after its time limit, records kDevTimeoutSelftest and the kernel returns normally.
+__global__ void __launch_bounds__(32) selftest_bounded_wait_kernel(uint32_t* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncwarp();
+  const bool done = __all_sync(0xffffffffu, mbar_wait(&bar, 0, status, kDevTimeoutSelftest));
+  if (done && threadIdx.x == 0) record_status(status, kDevSelftestUnexpected);
+}
+
+}  // namespace
+
+extern "C" nabla_status nabla_selftest_bounded_wait(void* workspace, size_t workspace_bytes,
+                                                    nabla_stream_t stream) {
+  if (!workspace || workspace_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return NABLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  selftest_bounded_wait_kernel<<<1, 32, 0, st>>>(static_cast<uint32_t*>(workspace));
+  return cuda_status(cudaGetLastError());
+}

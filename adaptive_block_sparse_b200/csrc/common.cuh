@@ -50,6 +50,8 @@ enum : uint32_t {
   kDevTimeoutDrain = 0x107,
   kDevTimeoutBwd = 0x108,
   kDevTimeoutMeta = 0x109,
+  kDevTimeoutSelftest = 0x10A,   // nabla_selftest_bounded_wait: the expected outcome
+  kDevSelftestUnexpected = 0x10B,
   kDevFp16Range = 0x201,   // backward: an input exceeds the fp16 range (|x| > 65504)
 };
 

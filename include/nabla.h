@@ -244,6 +244,16 @@ nabla_status nabla_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                                     float scale, void *o, nabla_dtype o_dtype, float *lse,
                                     nabla_layout layout, nabla_stream_t stream);
 
+/* Failure-path self-test (no counterpart in the pages).  Enqueues one warp that waits,
+ * through the same bounded barrier wait as every kernel of the library, for a barrier
+ * phase that nothing completes.  The wait gives up after its limit (about 2 s), records
+ * the code 0x10A in the status word of `workspace` (>= 256 bytes, 256-byte aligned) and
+ * the kernel returns: nabla_read_device_status() then reports NABLA_ERR_DEVICE_CHECK
+ * with code 0x10A, and the stream and context stay usable.  No trap, fault or hang.
+ * Errors: WORKSPACE, CUDA. */
+nabla_status nabla_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
+                                         nabla_stream_t stream);
+
 /* Reads (synchronously on `stream`) the device status word that the kernels of the
  * last call on `workspace` recorded: 0 = fine, otherwise a code naming the barrier
  * wait that gave up.  Returns NABLA_ERR_DEVICE_CHECK when the word is non-zero, and

@@ -126,3 +126,6 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert fwd(layout=2) == INV                                            # unknown layout
     assert lib.nabla_fwd_workspace_bytes(_shape(nb, D=96)) == 0
     assert lib.nabla_status_string(3) == b"NABLA_ERR_WORKSPACE"
+    assert lib.nabla_selftest_bounded_wait(None, 256, st) == WS
+    assert lib.nabla_selftest_bounded_wait(Bp, 255, st) == WS
+    assert lib.nabla_selftest_bounded_wait(ctypes.c_void_p(0x20000010), 256, st) == WS   # misaligned
