@@ -52,8 +52,9 @@ static_assert(128 * kRegProducer + 256 * kRegSoftmax <= kThreads * kLaunchRegs,
 template <int D>
 struct FwdCfg {
   static constexpr int kPanels = D / 64;                  // 128-byte swizzle panels
-  static constexpr int kTileBytes = 128 * D * 2;          // 128 rows of Q, K or V
-  static constexpr int kSlotBytes = 3 * kTileBytes;       // Q, K pair, V pair
+  static constexpr int kTileBytes = 128 * D * 2;          // 128 rows of Q
+  static constexpr int kStageBytes = 64 * D * 2;          // one key block of K or V
+  static constexpr int kSlotBytes = kTileBytes + 4 * kStageBytes;   // Q, 2 K stages, 2 V stages
   static constexpr int kOffMeta = 2 * kSlotBytes;         // [2 slots][kMetaRing][kMetaInts]
   static constexpr int kOffBar = kOffMeta + 2 * kMetaRing * kMetaInts * 4;
   // bf16 O staging for the epilogue's tiled stores: per softmax warp 32 rows x 128 bytes
@@ -62,8 +63,10 @@ struct FwdCfg {
   static constexpr int kOStageWarpBytes = 32 * 128;
   static constexpr int kSmemBytes = kOffOStage + 8 * kOStageWarpBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  // slot s: score buffer at column 128 s, accumulator at column 256 + 128 s
-  static __device__ __forceinline__ uint32_t col_s(int s) { return static_cast<uint32_t>(s) * 128u; }
+  // slot s: score buffers b = 0, 1 at column 128 s + 64 b, accumulator at 256 + 128 s
+  static __device__ __forceinline__ uint32_t col_s(int s, int b) {
+    return static_cast<uint32_t>(s) * 128u + static_cast<uint32_t>(b) * 64u;
+  }
   static __device__ __forceinline__ uint32_t col_o(int s) { return 256u + static_cast<uint32_t>(s) * 128u; }
 };
 
@@ -140,11 +143,12 @@ __device__ __forceinline__ TileMeta read_meta(const int32_t* m) {
 
 // Per-slot barriers (all in shared memory).
 struct SlotBars {
-  uint64_t q_full, q_empty;      // Q landed / the tile's last S has read Q
-  uint64_t k_full, k_empty;      // K pair landed / S has read it
-  uint64_t v_full, v_empty;      // V pair landed / P V has read it
-  uint64_t s_full, p_full;       // S landed in TMEM / the softmax wrote P
-  uint64_t tile_done, o_free;    // the tile's last P V landed / the epilogue read O
+  uint64_t q_full, q_empty;          // Q landed / the tile's last S has read Q
+  uint64_t k_full[2], k_empty[2];    // K stage landed / S has read it
+  uint64_t v_full[2], v_empty[2];    // V stage landed / P V has read it
+  uint64_t s_full[2], p_full[2];     // score buffer: S landed / the softmax wrote P
+  uint64_t pv_done;                  // completes once per P V (O may then be rescaled)
+  uint64_t tile_done, o_free;        // the tile's last P V landed / the epilogue read O
   uint64_t meta_full[kMetaRing], meta_empty[kMetaRing];
   uint64_t drain;
 };
@@ -182,12 +186,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       SlotBars& B = bars[s];
       mbar_init(&B.q_full, 1);
       mbar_init(&B.q_empty, 1);
-      mbar_init(&B.k_full, 1);
-      mbar_init(&B.k_empty, 1);
-      mbar_init(&B.v_full, 1);
-      mbar_init(&B.v_empty, 1);
-      mbar_init(&B.s_full, 1);
-      mbar_init(&B.p_full, 128);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&B.k_full[b], 1);
+        mbar_init(&B.k_empty[b], 1);
+        mbar_init(&B.v_full[b], 1);
+        mbar_init(&B.v_empty[b], 1);
+        mbar_init(&B.s_full[b], 1);
+        mbar_init(&B.p_full[b], 128);
+      }
+      mbar_init(&B.pv_done, 1);
       mbar_init(&B.tile_done, 1);
       mbar_init(&B.o_free, 128);
       for (int r = 0; r < R; ++r) {
@@ -212,14 +219,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int slot = warp >> 1;
     SlotBars& B = bars[slot];
     unsigned char* sQ = smem + slot * C::kSlotBytes;
-    unsigned char* sK = sQ + C::kTileBytes;
-    unsigned char* sV = sK + C::kTileBytes;
+    unsigned char* sK = sQ + C::kTileBytes;             // stage b at sK + b * kStageBytes
+    unsigned char* sV = sK + 2 * C::kStageBytes;
     int32_t* meta = reinterpret_cast<int32_t*>(smem + C::kOffMeta) + slot * R * kMetaInts;
     if ((warp & 1) == 0) {
       // ---------------------------------------------------------------- streamer of the slot
-      // The whole warp fetches and walks; lane 0 issues the copies.  Everything per slot is
-      // one chain, so one K and one V stage suffice: K of step g + 1 loads while the
-      // softmax of step g runs, V of step g + 1 once P V of step g has read the stage.
+      // The whole warp fetches and walks; lane 0 issues the copies.  A step is one key
+      // block; K and V each have two stages, K running a step ahead of V: K of step g + 1
+      // once S of step g - 1 has read its stage, V of step g once P V of step g - 2 has.
       if (lane == 0) {
         tma_prefetch_desc(&map_q);
         tma_prefetch_desc(&map_k);
@@ -292,13 +299,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mt[1] = bh;
           mt[2] = ab.x;
           mt[3] = ab.y;
-          mt[4] = (cnt + 1) >> 1;
+          mt[4] = cnt;
           mbar_arrive(&B.meta_full[r]);
         }
         __syncwarp();
         return 1;
       };
-      long long gk = 0, gv = 0;   // K and V pairs issued
+      long long gk = 0, gv = 0;   // K and V blocks issued
       int nq = 0;                 // Q tiles issued
       int fetched = 0;            // descriptors published
       bool end = false, ok = true;
@@ -337,57 +344,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         WarpBitWalk wk;
         wk.init(prm.bits + (static_cast<long long>(t.bh) * nb + t.ia) * nw,
                 t.ib >= 0 ? prm.bits + (static_cast<long long>(t.bh) * nb + t.ib) * nw : nullptr, nw, nb);
-        for (int k = 0; k < t.n; ++k) {
-          uint32_t fa = 0, fb = 0;
-          const int ja = wk.next(&fa);
-          int jb = wk.next(&fb);
-          if (jb < 0) jb = ja;                      // odd tail: a masked duplicate
-          if (gk > 0 && !wait_all(&B.k_empty, (gk - 1) & 1, kDevTimeoutKvEmpty)) { ok = false; break; }
+        auto load_k = [&](int j) -> bool {
+          const int st = static_cast<int>(gk & 1);
+          if (gk >= 2 && !wait_all(&B.k_empty[st], ((gk >> 1) - 1) & 1, kDevTimeoutKvEmpty)) return false;
           if (lane == 0) {
-            mbar_arrive_expect_tx(&B.k_full, C::kTileBytes);
+            mbar_arrive_expect_tx(&B.k_full[st], C::kStageBytes);
 #pragma unroll
-            for (int pn = 0; pn < C::kPanels; ++pn) {
-              load_block(sK + pn * 16384, &map_k, &B.k_full, pn, t.bh, ja);
-              load_block(sK + pn * 16384 + 8192, &map_k, &B.k_full, pn, t.bh, jb);
-            }
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              load_block(sK + st * C::kStageBytes + pn * 8192, &map_k, &B.k_full[st], pn, t.bh, j);
           }
           __syncwarp();
           ++gk;
-          if (gv > 0 && !wait_all(&B.v_empty, (gv - 1) & 1, kDevTimeoutKvEmpty)) { ok = false; break; }
+          return true;
+        };
+        auto load_v = [&](int j) -> bool {
+          const int st = static_cast<int>(gv & 1);
+          if (gv >= 2 && !wait_all(&B.v_empty[st], ((gv >> 1) - 1) & 1, kDevTimeoutKvEmpty)) return false;
           if (lane == 0) {
-            mbar_arrive_expect_tx(&B.v_full, C::kTileBytes);
+            mbar_arrive_expect_tx(&B.v_full[st], C::kStageBytes);
 #pragma unroll
-            for (int pn = 0; pn < C::kPanels; ++pn) {
-              load_block(sV + pn * 16384, &map_v, &B.v_full, pn, t.bh, ja);
-              load_block(sV + pn * 16384 + 8192, &map_v, &B.v_full, pn, t.bh, jb);
-            }
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              load_block(sV + st * C::kStageBytes + pn * 8192, &map_v, &B.v_full[st], pn, t.bh, j);
           }
           __syncwarp();
           ++gv;
+          return true;
+        };
+        uint32_t f = 0;
+        int j_next = t.n > 0 ? wk.next(&f) : -1;
+        if (t.n > 0 && !load_k(j_next)) { ok = false; break; }
+        for (int k = 0; k < t.n; ++k) {
+          const int j = j_next;
+          if (k + 1 < t.n) {
+            j_next = wk.next(&f);
+            if (!load_k(j_next)) { ok = false; break; }
+          }
+          if (!load_v(j)) { ok = false; break; }
         }
+        if (!ok) break;
       }
       // Drain: copies still in flight must land before the CTA exits.
       if (nq > 0) mbar_wait(&B.q_full, (nq - 1) & 1, status, kDevTimeoutDrain);
-      if (gk > 0) mbar_wait(&B.k_full, (gk - 1) & 1, status, kDevTimeoutDrain);
-      if (gv > 0) mbar_wait(&B.v_full, (gv - 1) & 1, status, kDevTimeoutDrain);
+      for (long long x = gk > 2 ? gk - 2 : 0; x < gk; ++x)
+        mbar_wait(&B.k_full[x & 1], (x >> 1) & 1, status, kDevTimeoutDrain);
+      for (long long x = gv > 2 ? gv - 2 : 0; x < gv; ++x)
+        mbar_wait(&B.v_full[x & 1], (x >> 1) & 1, status, kDevTimeoutDrain);
       __syncwarp();
     } else {
       // ---------------------------------------------------------------- MMA issuer of the slot
-      // Per step: S = Q K^T into the score buffer (the previous step's P V, which read P
-      // from that buffer, was issued before: tcgen05 MMAs of one thread run in order), then
-      // O += P V once the softmax has written P.  s_full also tells the softmax that every
-      // earlier P V of the slot has landed, so it may rescale O.
+      // Step g (one key block): S_g = Q K_g^T into score buffer g & 1, issued before
+      // O += P_{g-1} V_{g-1}, so that S of the next step runs while the softmax of this
+      // one does.  The buffer S_g overwrites held P_{g-2}, read by the P V issued before
+      // (tcgen05 MMAs of one thread run in order).  Every P V commits pv_done, which the
+      // softmax waits for before it rescales O.
       if (lane == 0) {
-        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t idesc_o = VF16 ? idesc_f16_f32(128, D, false, true)
                                           : idesc_bf16_f32(128, D, false, true);
         const uint32_t q_addr = smem_u32(sQ);
         const uint32_t k_addr = smem_u32(sK);
         const uint32_t v_addr = smem_u32(sV);
-        const uint32_t s_tmem = tmem + C::col_s(slot);
         const uint32_t o_tmem = tmem + C::col_o(slot);
-        long long g = 0;   // steps issued
+        long long g = 0;   // steps whose S has been issued
         bool ok = true;
+        auto issue_s = [&](bool last_of_tile) -> bool {
+          const int b = static_cast<int>(g & 1);
+          if (!mbar_wait(&B.k_full[b], (g >> 1) & 1, status, kDevTimeoutTmaFull)) return false;
+          tc_fence_after();
+          const uint32_t ks = k_addr + b * C::kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int pn = kk >> 2, w = kk & 3;
+            const uint64_t ad = sdesc_sw128(q_addr + pn * 16384 + w * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(ks + pn * 8192 + w * 32, 16, 1024);
+            mma_bf16_ss(tmem + C::col_s(slot, b), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&B.s_full[b]);
+          mma_commit(&B.k_empty[b]);
+          if (last_of_tile) mma_commit(&B.q_empty);   // the tile's last S has read Q
+          ++g;
+          return true;
+        };
         for (int c = 0; ok; ++c) {
           if (!mbar_wait(&B.meta_full[c % R], (c / R) & 1, status, kDevTimeoutMeta)) break;
           const TileMeta t = read_meta(meta + (c % R) * kMetaInts);
@@ -401,34 +438,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&B.tile_done);
             continue;
           }
-          for (int k = 0; k < t.n; ++k, ++g) {
-            if (!mbar_wait(&B.k_full, g & 1, status, kDevTimeoutTmaFull)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int pn = kk >> 2, w = kk & 3;
-              const uint64_t ad = sdesc_sw128(q_addr + pn * 16384 + w * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(k_addr + pn * 16384 + w * 32, 16, 1024);
-              mma_bf16_ss(s_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&B.s_full);
-            mma_commit(&B.k_empty);
-            if (k == t.n - 1) mma_commit(&B.q_empty);   // the tile's last S has read Q
-            if (!mbar_wait(&B.p_full, g & 1, status, kDevTimeoutPFull)) { ok = false; break; }
+          if (!issue_s(t.n == 1)) break;
+          for (int k = 0; k < t.n; ++k) {
+            if (k + 1 < t.n && !issue_s(k + 2 == t.n)) { ok = false; break; }
+            // P V of step k of the tile (global step gs: S of the next step, if any, is
+            // already issued)
+            const long long gs = (k + 1 < t.n) ? g - 2 : g - 1;
+            const int b = static_cast<int>(gs & 1);
+            if (!mbar_wait(&B.p_full[b], (gs >> 1) & 1, status, kDevTimeoutPFull)) { ok = false; break; }
             if (k == 0 && c > 0) {
               // The accumulator holds the previous tile until its epilogue has read it.
               if (!mbar_wait(&B.o_free, (c - 1) & 1, status, kDevTimeoutOBar)) { ok = false; break; }
             }
-            if (!mbar_wait(&B.v_full, g & 1, status, kDevTimeoutTmaFull)) { ok = false; break; }
+            if (!mbar_wait(&B.v_full[b], (gs >> 1) & 1, status, kDevTimeoutTmaFull)) { ok = false; break; }
             tc_fence_after();
-            // O += P V: P (16-bit, 128 keys) in the first 64 columns of the score buffer,
-            // V pair MN-major (panel stride 16 KB along D, 8-row groups 1 KB apart).
+            // O += P V: P (16-bit, 64 keys) in the first 32 columns of score buffer b, V stage
+            // b MN-major (panel stride 8 KB along D, 8-row groups 1 KB apart).
+            const uint32_t vs = v_addr + b * C::kStageBytes;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, 16384, 1024);
-              mma_bf16_ts(o_tmem, s_tmem + kk * 8, bd, idesc_o, (k > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = sdesc_sw128(vs + kk * 2048, 8192, 1024);
+              mma_bf16_ts(o_tmem, tmem + C::col_s(slot, b) + kk * 8, bd, idesc_o, (k > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&B.v_empty);
+            mma_commit(&B.v_empty[b]);
+            mma_commit(&B.pv_done);
           }
           if (!ok) break;
           mma_commit(&B.tile_done);
@@ -449,7 +482,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool upper = row >= 64;
     const float sl2 = prm.scale_log2;
     const float2 sl2v = make_float2(sl2, sl2);
-    const uint32_t s_col = tmem + lane_base + C::col_s(slot);
     const uint32_t o_col = tmem + lane_base + C::col_o(slot);
     long long g = 0;   // steps processed
     bool ok = true;
@@ -461,55 +493,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = t.n;
       float m_ref = -INFINITY;
       float l = 0.f;
-      // The step's key blocks and flags come from the tile's bitmask rows, walked the same
+      // The step's key block and flags come from the tile's bitmask rows, walked the same
       // way as the streamer does.
       WarpBitWalk wk;
       wk.init(prm.bits + (static_cast<long long>(t.bh) * nb + t.ia) * nw,
               t.ib >= 0 ? prm.bits + (static_cast<long long>(t.bh) * nb + t.ib) * nw : nullptr, nw, nb);
       for (int k = 0; k < n; ++k, ++g) {
-        uint32_t fa = 0, fb = 0;
-        wk.next(&fa);
-        if (wk.next(&fb) < 0) fb = 0;
+        uint32_t f = 0;
+        wk.next(&f);
         // warp-uniform: rows 0-63 (block a) and 64-127 (block b) sit in different warps
-        const bool keep_a = upper ? (fa >> 1) : (fa & 1u);
-        const bool keep_b = upper ? (fb >> 1) : (fb & 1u);
-        ok = __all_sync(0xffffffffu, mbar_wait(&B.s_full, g & 1, status, kDevTimeoutSFull));
+        const bool keep = upper ? (f >> 1) : (f & 1u);
+        const int b = static_cast<int>(g & 1);
+        const uint32_t s_col = tmem + lane_base + C::col_s(slot, b);
+        ok = __all_sync(0xffffffffu, mbar_wait(&B.s_full[b], (g >> 1) & 1, status, kDevTimeoutSFull));
         if (!ok) break;
         tc_fence_after();
-        // The whole row of 128 scores in registers: one TMEM round trip per step.
-        uint32_t sv[128];
+        // The row's 64 scores of the step in registers: one TMEM round trip.
+        uint32_t sv[64];
         uint32_t(&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
         uint32_t(&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-        uint32_t(&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[64]);
-        uint32_t(&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[96]);
-        if (keep_a) {
+        float mx = -INFINITY;
+        if (keep) {
           tmem_ld32(s_col, c0);
           tmem_ld32(s_col + 32, c1);
-        }
-        if (keep_b) {
-          tmem_ld32(s_col + 64, c2);
-          tmem_ld32(s_col + 96, c3);
-        }
-        tmem_wait_ld();
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
-        if (keep_a) {
+          tmem_wait_ld();
           reg_fence32(c0);
           reg_fence32(c1);
+          float m8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
 #pragma unroll
           for (int cc = 0; cc < 64; cc += 2)
             m8[(cc >> 1) & 7] = fmax3(m8[(cc >> 1) & 7], __uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1]));
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
-        if (keep_b) {
-          reg_fence32(c2);
-          reg_fence32(c3);
-#pragma unroll
-          for (int cc = 64; cc < 128; cc += 2)
-            m8[(cc >> 1) & 7] = fmax3(m8[(cc >> 1) & 7], __uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1]));
-        }
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         float factor = 1.f;
         bool rescale = false;
         if (mx != -INFINITY && mx * sl2 > m_ref + 8.0f) {
@@ -521,39 +539,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_ref = rm;
         }
         // P = 2^(s*scale*log2e - m) as 16-bit pairs (keys 2e, 2e+1 -> column e) into the
-        // first 64 columns of the score buffer (those scores are already in registers).
+        // first 32 columns of the score buffer (those scores are already in registers).
         const float2 negm = make_float2(-m_ref, -m_ref);
         float2 acc = make_float2(0.f, 0.f);
+        if (keep) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h == 0 ? keep_a : keep_b) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int i = h * 64 + 2 * e;
-              const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), sl2v, negm);
-              const float2 pr = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
-              // The row sum takes the rounded weights that enter the PV product, so the
-              // output is an exact convex combination of them.
-              uint32_t pk;
-              if constexpr (VF16) {
-                pk = pack_f16x2(pr.x, pr.y);
-                acc = __fadd2_rn(acc, make_float2(f16lo(pk), f16hi(pk)));
-              } else {
-                pk = pack_bf16x2(pr.x, pr.y);
-                acc = __fadd2_rn(acc, make_float2(bf16lo(pk), bf16hi(pk)));
-              }
-              sv[h * 32 + e] = pk;
+          for (int e = 0; e < 32; ++e) {
+            const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2v, negm);
+            const float2 pr = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
+            // The row sum takes the rounded weights that enter the PV product, so the
+            // output is an exact convex combination of them.
+            uint32_t pk;
+            if constexpr (VF16) {
+              pk = pack_f16x2(pr.x, pr.y);
+              acc = __fadd2_rn(acc, make_float2(f16lo(pk), f16hi(pk)));
+            } else {
+              pk = pack_bf16x2(pr.x, pr.y);
+              acc = __fadd2_rn(acc, make_float2(bf16lo(pk), bf16hi(pk)));
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sv[h * 32 + e] = 0u;
+            sv[e] = pk;
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sv[e] = 0u;
         }
         tmem_st32(s_col, c0);
-        tmem_st32(s_col + 32, c1);
-        // Every earlier P V of the slot has landed (s_full), so O may be rescaled in place
-        // before this step's P V (issued once p_full completes); warp-uniform.
+        // O may be rescaled in place once every earlier P V of the slot has landed (the
+        // previous step's, of this tile: a tile's first step never rescales), before this
+        // step's P V (issued once p_full completes); warp-uniform.
         if (__any_sync(0xffffffffu, rescale)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&B.pv_done, (g - 1) & 1, status, kDevTimeoutPFull));
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll 1
           for (int o0 = 0; o0 < D; o0 += 16) {
             uint32_t ov[16];
@@ -568,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = l * factor + (acc.x + acc.y);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&B.p_full);
+        mbar_arrive(&B.p_full[b]);
       }
       if (!ok) break;
       // ---- epilogue of the tile: O / l and the LSE, once its last P V has landed
