@@ -245,6 +245,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(dst, map, bar, pn * 64, static_cast<int>(bh * prm.S + static_cast<long long>(blk) * 64));
         }
       };
+      // K or V of block blk of head bh, all D columns in one copy: the map's outermost
+      // dimension walks the 64-column panels, so the copy lands as the panels one after
+      // the other (8 KB apart), as per-panel copies would
+      auto load_kv = [&](unsigned char* dst, const CUtensorMap* map, uint64_t* bar, int bh, int blk) {
+        if constexpr (NAT) {
+          const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+          tma_load_5d(dst, map, bar, 0, wb * 8, hb * 8, bh * prm.T + tf, 0);
+        } else {
+          tma_load_3d(dst, map, bar, 0, static_cast<int>(bh * prm.S + static_cast<long long>(blk) * 64), 0);
+        }
+      };
       // the rows of block blk of head bh into L2 (contiguous in the reordered order; eight
       // patch rows of 8 tokens in the natural one)
       auto prefetch_block = [&](int bh, int blk) {
@@ -349,9 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (gk >= 2 && !wait_all(&B.k_empty[st], ((gk >> 1) - 1) & 1, kDevTimeoutKvEmpty)) return false;
           if (lane == 0) {
             mbar_arrive_expect_tx(&B.k_full[st], C::kStageBytes);
-#pragma unroll
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              load_block(sK + st * C::kStageBytes + pn * 8192, &map_k, &B.k_full[st], pn, t.bh, j);
+            load_kv(sK + st * C::kStageBytes, &map_k, &B.k_full[st], t.bh, j);
           }
           __syncwarp();
           ++gk;
@@ -362,9 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (gv >= 2 && !wait_all(&B.v_empty[st], ((gv >> 1) - 1) & 1, kDevTimeoutKvEmpty)) return false;
           if (lane == 0) {
             mbar_arrive_expect_tx(&B.v_full[st], C::kStageBytes);
-#pragma unroll
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              load_block(sV + st * C::kStageBytes + pn * 8192, &map_v, &B.v_full[st], pn, t.bh, j);
+            load_kv(sV + st * C::kStageBytes, &map_v, &B.v_full[st], t.bh, j);
           }
           __syncwarp();
           ++gv;
@@ -764,6 +771,38 @@ bool make_map_nat(CUtensorMap* map, const void* base, long long frames, int Hg, 
   return r == CUDA_SUCCESS;
 }
 
+// K / V maps for one-copy block loads: the D columns split into 64-column panels as the
+// outermost dimension (stride 128 bytes), box = 64 columns x one block x all panels.
+// Natural order: [B*H*T, Hg, W, D] viewed as (64 ch, W, Hg, frames, D/64); reordered:
+// [rows, D] viewed as (64 ch, rows, D/64).
+bool make_map_kv(CUtensorMap* map, const void* base, long long rows, int D, bool fp16) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(D / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, 128u};
+  cuuint32_t box[3] = {64u, 64u, static_cast<cuuint32_t>(D / 64)};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_kv_nat(CUtensorMap* map, const void* base, long long frames, int Hg, int W, int D, bool fp16) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[5] = {64u, static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(Hg),
+                        static_cast<cuuint64_t>(frames), static_cast<cuuint64_t>(D / 64)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(W) * D * 2,
+                           static_cast<cuuint64_t>(Hg) * W * D * 2, 128u};
+  cuuint32_t box[5] = {64u, 8u, 8u, 1u, static_cast<cuuint32_t>(D / 64)};
+  cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  return enc(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // f32 O maps for the epilogue's stores: box = 32 floats (128 bytes) x 32 rows, or x 8
 // columns x 4 rows x 1 frame of a natural-order tensor; 128-byte swizzle.
 bool make_map_f32(CUtensorMap* map, const void* base, long long rows, int D) {
@@ -801,11 +840,11 @@ cudaError_t launch_fwd(const void* q, const void* k, const void* v, const Dims& 
   const long long frames = static_cast<long long>(d.BH) * d.T;
   if constexpr (NAT) {
     *map_ok = make_map_nat(&mq, q, frames, d.Hg, d.W, D, false) &&
-              make_map_nat(&mk, k, frames, d.Hg, d.W, D, false) &&
-              make_map_nat(&mv, v, frames, d.Hg, d.W, D, VF16);
+              make_map_kv_nat(&mk, k, frames, d.Hg, d.W, D, false) &&
+              make_map_kv_nat(&mv, v, frames, d.Hg, d.W, D, VF16);
   } else {
-    *map_ok = make_map_16(&mq, q, rows, D, 64, false) && make_map_16(&mk, k, rows, D, 64, false) &&
-              make_map_16(&mv, v, rows, D, 64, VF16);   // one 64-row block per copy
+    *map_ok = make_map_16(&mq, q, rows, D, 64, false) && make_map_kv(&mk, k, rows, D, false) &&
+              make_map_kv(&mv, v, rows, D, VF16);
   }
   // O: tiled stores of 32-row parts, 128 bytes of each row per copy
   if (*map_ok)
