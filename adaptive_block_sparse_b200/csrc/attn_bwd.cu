@@ -36,6 +36,7 @@ namespace nabla {
 
 bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows,
                  bool fp16);
+bool make_map_kv(CUtensorMap* map, const void* base, long long rows, int D, bool fp16);
 
 namespace {
 
@@ -297,11 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         unsigned char* st = sStage + s * L::kStageStride;
         mbar_arrive_expect_tx(&full[s], 2 * C::kTileBytes + 512);
         const long long qrow = bh * prm.S + static_cast<long long>(i) * 64;
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_2d(st + pn * 8192, &map_q64, &full[s], pn * 64, static_cast<int>(qrow));
-          tma_load_2d(st + C::kTileBytes + pn * 8192, &map_do64, &full[s], pn * 64, static_cast<int>(qrow));
-        }
+        // one copy per operand: all D columns of the 64 rows (panels 8 KB apart)
+        tma_load_3d(st, &map_q64, &full[s], 0, static_cast<int>(qrow), 0);
+        tma_load_3d(st + C::kTileBytes, &map_do64, &full[s], 0, static_cast<int>(qrow), 0);
         bulk_load(st + 2 * C::kTileBytes, prm.lse2 + qrow, 256, &full[s]);
         bulk_load(st + 2 * C::kTileBytes + 256, prm.delta + qrow, 256, &full[s]);
         ++it;
@@ -582,11 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         unsigned char* st = sStage + s * L::kStageBytes;
         mbar_arrive_expect_tx(&full[s], 2 * C::kTileBytes);
         const int krow = static_cast<int>(bh * prm.S + static_cast<long long>(j) * 64);
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_2d(st + pn * 8192, &map_k64, &full[s], pn * 64, krow);
-          tma_load_2d(st + C::kTileBytes + pn * 8192, &map_v64, &full[s], pn * 64, krow);
-        }
+        // one copy per operand: all D columns of the 64 rows (panels 8 KB apart)
+        tma_load_3d(st, &map_k64, &full[s], 0, krow, 0);
+        tma_load_3d(st + C::kTileBytes, &map_v64, &full[s], 0, krow, 0);
         ++it;
       }
       // Copies still in flight (as in the dK/dV pass).
@@ -767,9 +764,13 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
       do16, delta, lse2, rows, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  CUtensorMap mq64, mdo64, mk64, mv64;
+  // per-panel maps for the resident 128-row operands (two 64-row blocks per panel), and
+  // one-copy maps (panels as the outermost dimension) for the streamed 64-row stages
+  CUtensorMap mq64, mdo64, mk64, mv64, mq3, mdo3, mk3, mv3;
   *map_ok = make_map_16(&mq64, q16, rows, D, 64, true) && make_map_16(&mdo64, do16, rows, D, 64, true) &&
-            make_map_16(&mk64, k16, rows, D, 64, true) && make_map_16(&mv64, v16, rows, D, 64, true);
+            make_map_16(&mk64, k16, rows, D, 64, true) && make_map_16(&mv64, v16, rows, D, 64, true) &&
+            make_map_kv(&mq3, q16, rows, D, true) && make_map_kv(&mdo3, do16, rows, D, true) &&
+            make_map_kv(&mk3, k16, rows, D, true) && make_map_kv(&mv3, v16, rows, D, true);
   if (!*map_ok) return cudaErrorInvalidValue;
 
   BwdParams p;
@@ -793,7 +794,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DkdvLayout<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk64, mv64, p);
+  attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq3, mdo3, mk64, mv64, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   p.order = order_rows;
@@ -804,7 +805,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DqLayout<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk64, mv64, p);
+  attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk3, mv3, p);
   return cudaGetLastError();
 }
 
