@@ -235,11 +235,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t code) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
       };
+      // Block index -> (frame, patch row, patch column) without integer division: the
+      // quotients come from float reciprocals, exact here (blk < 2^14, so (blk + 0.5) / n
+      // stays more than 0.5 / n from an integer while its float error is below 2^-9 / n).
+      const float inv_hw = 1.0f / static_cast<float>(prm.HW);
+      const float inv_wb = 1.0f / static_cast<float>(prm.Wb);
+      auto decode = [&](int blk) {
+        const int tf = static_cast<int>((static_cast<float>(blk) + 0.5f) * inv_hw);
+        const int r = blk - tf * prm.HW;
+        const int hb = static_cast<int>((static_cast<float>(r) + 0.5f) * inv_wb);
+        return make_int3(tf, hb, r - hb * prm.Wb);
+      };
       // one 64-column panel of block blk of head bh: 64 rows of 128 bytes
       auto load_block = [&](unsigned char* dst, const CUtensorMap* map, uint64_t* bar, int pn, int bh,
                             int blk) {
         if constexpr (NAT) {
-          const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+          const int3 c3 = decode(blk);
+          const int tf = c3.x, hb = c3.y, wb = c3.z;
           tma_load_4d(dst, map, bar, pn * 64, wb * 8, hb * 8, bh * prm.T + tf);
         } else {
           tma_load_2d(dst, map, bar, pn * 64, static_cast<int>(bh * prm.S + static_cast<long long>(blk) * 64));
@@ -250,7 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the other (8 KB apart), as per-panel copies would
       auto load_kv = [&](unsigned char* dst, const CUtensorMap* map, uint64_t* bar, int bh, int blk) {
         if constexpr (NAT) {
-          const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+          const int3 c3 = decode(blk);
+          const int tf = c3.x, hb = c3.y, wb = c3.z;
           tma_load_5d(dst, map, bar, 0, wb * 8, hb * 8, bh * prm.T + tf, 0);
         } else {
           tma_load_3d(dst, map, bar, 0, static_cast<int>(bh * prm.S + static_cast<long long>(blk) * 64), 0);
@@ -261,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto prefetch_block = [&](int bh, int blk) {
         const char* qg = static_cast<const char*>(prm.q);
         if constexpr (NAT) {
-          const int tf = blk / prm.HW, hb = (blk / prm.Wb) % prm.Hb, wb = blk % prm.Wb;
+          const int3 c3 = decode(blk);
+          const int tf = c3.x, hb = c3.y, wb = c3.z;
 #pragma unroll 1
           for (int hh = 0; hh < 8; ++hh)
             l2_prefetch(qg + ((static_cast<long long>(bh * prm.T + tf) * prm.Hg + hb * 8 + hh) * prm.W + wb * 8) * D * 2,
