@@ -16,10 +16,10 @@
 //
 // Selection without a sort: block j is kept iff E_j < thr, where E_j is the mass ranked
 // strictly before j (probability descending, ties by lower index).  The kept set is a
-// prefix of that ranking, so it is found by bisecting over the fp64 bit patterns of the
-// probabilities (non-negative doubles order like their bit patterns) until the interval
-// of keys where the "mass at or above" crosses thr holds at most a few blocks; those are
-// ranked (probability descending, index ascending) and walked in order.  The logits are
+// prefix of that ranking, so it is found by narrowing an interval of fp64 bit patterns
+// of the probabilities (non-negative doubles order like their bit patterns) where the
+// "mass at or above" crosses thr until it holds at most a few blocks; those are ranked
+// (probability descending, index ascending) and walked in order.  The logits are
 // computed with fp64 tensor-core MMA (m8n8k4), two key tiles per warp at a time.
 #include <math.h>
 
@@ -45,7 +45,7 @@ namespace {
 constexpr int kThreads = 256;   // 8 warps; one pooled row per warp during selection
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
-constexpr int kCand = 16;       // the cut's bisection stops at this many candidates
+constexpr int kCand = 16;       // the cut's search stops at this many candidates
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
@@ -168,11 +168,11 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
     for (int j = lane; j < nb; j += 32) row[j] = row[j] / ssum;
     __syncwarp();
 
-    // ---- the cut: bisection over the fp64 bit patterns, then the last few candidates -----
+    // ---- the cut: a bracket of fp64 bit patterns, then the last few candidates ----------
     // Non-negative doubles order like their bit patterns.  The keep rule (keep j iff the
     // mass ranked strictly above it is < thr; rank by P descending, index ascending) keeps
     // every block with key >= hi and drops every block with key < lo, for any lo < hi with
-    // mass(P >= lo) >= thr > mass(P >= hi).  The bisection narrows [lo, hi) until it holds
+    // mass(P >= lo) >= thr > mass(P >= hi).  The search narrows [lo, hi) until it holds
     // at most kCand blocks (or a single key, all ties); those candidates are ranked and
     // walked in order from mass(P >= hi).  Masses are summed per lane in index order, then
     // by a fixed butterfly: deterministic, fp64-accurate.
@@ -198,23 +198,60 @@ __global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
         *cnt = __reduce_add_sync(0xffffffffu, c);
         return acc;
       };
+      // Bracket: first guess one sixteenth of the row maximum; below it, the lower end
+      // from mass(P >= x) >= 1 - nb x; then probes interpolated linearly in the key, each
+      // kept within the middle half of the bracket.  The computed mass is monotone in
+      // the key, so every bracket that satisfies the invariant leads to the same walk.
+      double pm = 0.0;
+      for (int j = lane; j < nb; j += 32) pm = fmax(pm, row[j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) pm = fmax(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+      constexpr unsigned long long kSixteenth = 4ull << 52;   // 2^-4 in the exponent field
+      const unsigned long long kpm = static_cast<unsigned long long>(__double_as_longlong(pm));
+      const unsigned long long guess = kpm > kSixteenth ? kpm - kSixteenth : 0ull;
       int clo = 0, chi = 0;
-      if (mass_cnt_ge(0ull, &clo) >= thr) {
-        unsigned long long lo = 0ull, hi = 0x3FF0000000000001ull;   // just above 1.0
-        double mass_hi = 0.0;
+      unsigned long long lo, hi;
+      double mlo, mhi;
+      bool bracket = true;
+      const double mg = mass_cnt_ge(guess, &clo);
+      if (mg >= thr) {
+        lo = guess;
+        mlo = mg;
+        hi = 0x3FF0000000000001ull;                 // just above 1.0
+        mhi = 0.0;
+        chi = 0;
+      } else {
+        hi = guess;
+        mhi = mg;
+        chi = clo;
+        lo = static_cast<unsigned long long>(__double_as_longlong(0.5 * (1.0 - thr) / nb));
+        mlo = mass_cnt_ge(lo, &clo);
+        if (!(mlo >= thr)) {
+          lo = 0ull;
+          mlo = mass_cnt_ge(0ull, &clo);
+          bracket = mlo >= thr;
+        }
+      }
+      if (bracket) {
         while (clo - chi > kCand && hi - lo > 1ull) {
-          const unsigned long long mid = lo + ((hi - lo) >> 1);
+          const unsigned long long w = hi - lo;
+          const double f = fmin(fmax((mlo - thr) / (mlo - mhi), 0.25), 0.75);
+          unsigned long long step = static_cast<unsigned long long>(static_cast<double>(w) * f);
+          step = step < 1ull ? 1ull : (step > w - 1ull ? w - 1ull : step);
+          const unsigned long long mid = lo + step;
           int cm = 0;
           const double mm = mass_cnt_ge(mid, &cm);
           if (mm >= thr) {
             lo = mid;
             clo = cm;
+            mlo = mm;
           } else {
             hi = mid;
             chi = cm;
-            mass_hi = mm;
+            mhi = mm;
           }
         }
+        const double mass_hi = mhi;
         klo = lo;
         khi = hi;
         if (clo - chi <= kCand) {

@@ -17,17 +17,19 @@
 //     tcgen05 (M = 128, N = 256, K = 16 per instruction, fp32 accumulate in TMEM; the
 //     dominant q_hi k_hi^T term has its own accumulator), written to an fp32 scratch.
 //  3. mask_select_kernel: one warp per row: softmax in fp32; the cut value P_c (the
-//     smallest kept probability) by extracting maxima while the running mass is below
-//     thr (rows keeping a few blocks), else by bisection over the fp32 bit patterns until
-//     the interval where the mass at or above crosses thr holds at most 16 blocks, which
-//     are then ranked and walked; then the certificate: with rho the proven relative
-//     error of every P_j,
+//     smallest kept probability) from a bracket of fp32 bit patterns where the mass at
+//     or above crosses thr -- first guess one sixteenth of the row maximum, else a lower
+//     end from mass(P >= x) >= 1 - nb x and probes interpolated in the key -- narrowed
+//     until it holds at most 16 blocks, which are then ranked and walked; then the
+//     certificate: with rho the proven relative error of every P_j,
 //        thr - E_above > eta,  E_at_or_above - thr > eta,  P_c unique,
 //        P_c - P_next > 2 rho P_c,
 //     where eta = rho + 3e-6 bounds the error of the ranked masses.  A certified row
 //     keeps exactly the blocks with P_j >= P_c (the same set the exact ranking keeps);
 //     the others are appended to a per-head list that the fp64 kernel recomputes.
 #include <math.h>
+
+#include <type_traits>
 
 #include <cudaTypedefs.h>
 
@@ -44,7 +46,7 @@ namespace {
 // (3 x 2^-22), eight fp32 accumulations of the leading product (8 x 2^-22, allowing
 // truncating adds), the correction products and the final add / scale (~2^-22).
 constexpr float kLogitErr = 4.0e-6f;
-constexpr int kSelCand = 16;   // the cut's bisection stops at this many candidates
+constexpr int kSelCand = 16;   // the cut's search stops at this many candidates
 
 // ------------------------------------------------------------------------------------
 // 1. fp16 split of the pooled means + norms
@@ -53,28 +55,63 @@ template <int D>
 __global__ void __launch_bounds__(256) split_pools_kernel(
     const double* __restrict__ qpool, const double* __restrict__ kpool, int nb, int nbp,
     long long rows_pad, __half* __restrict__ qh, __half* __restrict__ ql, __half* __restrict__ kh,
-    __half* __restrict__ kl, float* __restrict__ qnorm, uint32_t* __restrict__ kmax_bits) {
+    __half* __restrict__ kl, float* __restrict__ qnorm, uint32_t* __restrict__ kmax_bits,
+    int vec16) {
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);   // padded
   const int lane = threadIdx.x & 31;
   if (row >= rows_pad) return;
   const long long bh = row / nbp;
   const int i = static_cast<int>(row - bh * nbp);
   const bool valid = i < nb;
+  // lane l takes the E = D / 32 consecutive columns from l * E: 16-byte loads of the
+  // fp64 means (8-byte loads when a pool base is only 8-byte aligned) and one 8- (or 4-)
+  // byte store per split tensor
   constexpr int E = D / 32;
+  static_assert(E == 2 || E == 4, "D must be 64 or 128");
+  double q[E], k[E];
+  if (valid && !vec16) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      q[e] = qpool[(bh * nb + i) * D + lane * E + e];
+      k[e] = kpool[(bh * nb + i) * D + lane * E + e];
+    }
+  } else if (valid) {
+    const double2* q2 = reinterpret_cast<const double2*>(qpool + (bh * nb + i) * D + lane * E);
+    const double2* k2 = reinterpret_cast<const double2*>(kpool + (bh * nb + i) * D + lane * E);
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      const double2 a = q2[e], b = k2[e];
+      q[2 * e] = a.x;
+      q[2 * e + 1] = a.y;
+      k[2 * e] = b.x;
+      k[2 * e + 1] = b.y;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) q[e] = k[e] = 0.0;
+  }
   double nq = 0.0, nk = 0.0;
+  __half qh1[E], ql1[E], kh1[E], kl1[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    const int d = lane * E + e;
-    const double q = valid ? qpool[(bh * nb + i) * D + d] : 0.0;
-    const double k = valid ? kpool[(bh * nb + i) * D + d] : 0.0;
-    const __half q1 = __double2half(q);
-    const __half k1 = __double2half(k);
-    qh[row * D + d] = q1;
-    kh[row * D + d] = k1;
-    ql[row * D + d] = __double2half(q - static_cast<double>(__half2float(q1)));
-    kl[row * D + d] = __double2half(k - static_cast<double>(__half2float(k1)));
-    nq = fma(q, q, nq);
-    nk = fma(k, k, nk);
+    qh1[e] = __double2half(q[e]);
+    kh1[e] = __double2half(k[e]);
+    ql1[e] = __double2half(q[e] - static_cast<double>(__half2float(qh1[e])));
+    kl1[e] = __double2half(k[e] - static_cast<double>(__half2float(kh1[e])));
+    nq = fma(q[e], q[e], nq);
+    nk = fma(k[e], k[e], nk);
+  }
+  const long long off = row * D + lane * E;
+  if constexpr (E == 4) {
+    *reinterpret_cast<uint2*>(qh + off) = *reinterpret_cast<const uint2*>(qh1);
+    *reinterpret_cast<uint2*>(ql + off) = *reinterpret_cast<const uint2*>(ql1);
+    *reinterpret_cast<uint2*>(kh + off) = *reinterpret_cast<const uint2*>(kh1);
+    *reinterpret_cast<uint2*>(kl + off) = *reinterpret_cast<const uint2*>(kl1);
+  } else {
+    *reinterpret_cast<uint32_t*>(qh + off) = *reinterpret_cast<const uint32_t*>(qh1);
+    *reinterpret_cast<uint32_t*>(ql + off) = *reinterpret_cast<const uint32_t*>(ql1);
+    *reinterpret_cast<uint32_t*>(kh + off) = *reinterpret_cast<const uint32_t*>(kh1);
+    *reinterpret_cast<uint32_t*>(kl + off) = *reinterpret_cast<const uint32_t*>(kl1);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -230,44 +267,61 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-template <int TPL>
+constexpr int kSelWarps = 8;   // rows (warps) per CTA of the select kernel
+
+// One warp per row.  The row's probabilities live in this warp's slice of shared memory
+// and every pass over them is a plain loop, so the kernel's code stays small (the passes
+// of a register-resident version, unrolled over the row, overflowed the instruction
+// cache) and its register count low.  Block j = lane + 32 t; lane l keeps t = 4 g + c
+// in ps4[32 g + l].c, so each access is one conflict-free 16-byte load or store per lane.
+// Sums are taken per lane in t order, then by a fixed butterfly.
 __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm, long long rows) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  extern __shared__ float4 psm4[];                     // [kSelWarps][T / 4][32]
+  __shared__ uint32_t cand_key[kSelWarps][kSelCand];   // per warp: the cut's candidates
+  __shared__ int cand_idx[kSelWarps][kSelCand];
+  __shared__ __align__(16) uint32_t words[kSelWarps][64];   // per warp: the row's bitmask
+  const long long row = static_cast<long long>(blockIdx.x) * kSelWarps + (threadIdx.x >> 5);
+  const int wslot = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   const int nb = prm.nb;
+  const int G = prm.nbp / 128;                         // float4 groups per lane
   const long long bh = row / nb;
   const int i = static_cast<int>(row - bh * nb);
   const float* a = prm.logits + (bh * prm.nbp + i) * static_cast<long long>(prm.nbp);
+  float4* ps4 = psm4 + static_cast<size_t>(wslot) * G * 32 + lane;   // ps4[32 g]
 
-  float p[TPL];
+  // ---- softmax (fp32): P_j = exp(A_j - max) / sum ------------------------------------
   float m = -INFINITY;
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    const int j = lane + 32 * t;
-    p[t] = (j < nb) ? a[j] : -INFINITY;
-    m = fmaxf(m, p[t]);
+#pragma unroll 2
+  for (int g = 0; g < G; ++g) {
+    const int j = lane + 128 * g;
+    float4 x;
+    x.x = j < nb ? a[j] : -INFINITY;
+    x.y = j + 32 < nb ? a[j + 32] : -INFINITY;
+    x.z = j + 64 < nb ? a[j + 64] : -INFINITY;
+    x.w = j + 96 < nb ? a[j + 96] : -INFINITY;
+    ps4[32 * g] = x;
+    m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
   }
   m = warp_max(m);
   float s = 0.f;
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    p[t] = __expf(p[t] - m);
-    s += p[t];
+  for (int g = 0; g < G; ++g) {
+    float4 x = ps4[32 * g];
+    x.x = __expf(x.x - m);
+    x.y = __expf(x.y - m);
+    x.z = __expf(x.z - m);
+    x.w = __expf(x.w - m);
+    ps4[32 * g] = x;
+    s += x.x;
+    s += x.y;
+    s += x.z;
+    s += x.w;
   }
   s = warp_sum(s);
   const float inv = 1.0f / s;
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) p[t] *= inv;
 
-  // Largest key k (fp32 bit pattern of a probability) with mass(P >= k) >= thr.
   const float thr = prm.thr;
-  auto mass_ge = [&](uint32_t k) {
-    float acc = 0.f;
-#pragma unroll
-    for (int t = 0; t < TPL; ++t) acc += (__float_as_uint(p[t]) >= k) ? p[t] : 0.f;
-    return warp_sum(acc);
-  };
   bool certified = false;
   uint32_t kcut = 0;
   // rho: relative error of every probability (two logits' errors, exp, division);
@@ -275,149 +329,158 @@ __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm
   const float eps = prm.scale * prm.qnorm[bh * nb + i] * __uint_as_float(prm.kmax_bits[bh]) * kLogitErr;
   const float rho = 2.f * eps + 1e-5f;
   const float eta = rho + 3.5e-6f;
-  // Certificate for a cut at value p_cut with ranked masses e_above (strictly above) and
-  // e_at (at or above), the next smaller value p_next and n_at values equal to p_cut.
-  // The kept set {P >= p_cut} must have exact mass > thr, and without its (exactly)
-  // smallest member -- at most e_above + eta + rho p_cut -- exact mass < thr.
-  auto certify = [&](float e_above, float e_at, float p_cut, float p_next, int n_at) {
-    return (thr - e_above > eta + rho * p_cut) && (e_at - thr > eta) && n_at == 1 &&
-           (p_cut - p_next > 2.f * rho * p_cut);
-  };
-  if (prm.thr_mode != 0) {            // thr >= 1: keep every block; thr <= 0: none
-    certified = true;
-    kcut = prm.thr_mode > 0 ? 0u : 0xFFFFFFFFu;
-  } else {
-    // Fast path: take maxima in descending order (ties: lower block index first) while
-    // the running mass is below thr; most rows keep only a few blocks.
-    constexpr int kMaxExtract = 16;
-    uint64_t taken = 0;                 // bit t: p[t] of this lane already taken
-    float acc = 0.f, acc_prev = 0.f;
-    bool found = false;
-    float p_cut = 0.f;
-    for (int e = 0; e <= kMaxExtract; ++e) {
-      float best = -1.f;
-      int bj = 0x7FFFFFFF;
-#pragma unroll
-      for (int t = 0; t < TPL; ++t)
-        if (!((taken >> t) & 1ull) && p[t] > best) { best = p[t]; bj = lane + 32 * t; }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-        if (ov > best || (ov == best && oj < bj)) { best = ov; bj = oj; }
+  // Bracket [lo, hi) of fp32 keys (bit patterns of probabilities) with
+  // mass(P >= lo) >= thr > mass(P >= hi); every block with key >= hi is kept and every
+  // block with key < lo dropped.  Probes, in order: one sixteenth of the row maximum
+  // (1 / sum; most rows keep a few large blocks, and then [guess, 1] already holds at
+  // most kSelCand of them); below it, the lower end from mass(P >= x) >= 1 - nb x (every
+  // block below x holds less than x), then 0; then points interpolated linearly in the
+  // key between the ends, kept within the middle half of the bracket.  The computed mass
+  // is monotone in the key (sums of a subset in a fixed order), so any bracket that
+  // satisfies the invariant leads to the same decision.  The first probe's pass also
+  // scales the exponentials into probabilities.
+  uint32_t lo = 0u, hi = 0x3F800001u;              // 0x3F800001: above 1.0
+  float mlo = 0.f, mhi = 0.f;
+  int clo = 0, chi = 0;
+  int phase = 0;                                   // 0 guess, 1 lower bound, 2 zero, 3 narrow
+  bool bracket = false;
+  uint32_t probe = max(__float_as_uint(inv), 4u << 23) - (4u << 23);
+  for (int it = 0; it < 128; ++it) {
+    float mm = 0.f;
+    int cm = 0;
+    auto acc = [&](float v) {
+      const bool ge = __float_as_uint(v) >= probe;
+      mm += ge ? v : 0.f;
+      cm += ge ? 1 : 0;
+    };
+    if (it == 0) {
+      for (int g = 0; g < G; ++g) {
+        float4 x = ps4[32 * g];
+        x.x *= inv;
+        x.y *= inv;
+        x.z *= inv;
+        x.w *= inv;
+        ps4[32 * g] = x;
+        acc(x.x);
+        acc(x.y);
+        acc(x.z);
+        acc(x.w);
       }
-      if (found) {                      // one more maximum: the first value below the cut
-        certified = certify(acc_prev, acc, p_cut, fmaxf(best, 0.f), best == p_cut ? 2 : 1);
-        break;
-      }
-      if (bj == 0x7FFFFFFF || e == kMaxExtract) break;
-      if ((bj & 31) == lane) taken |= 1ull << (bj >> 5);
-      acc_prev = acc;
-      acc += best;
-      if (acc >= thr) {
-        found = true;
-        p_cut = best;
-        kcut = __float_as_uint(best);
+    } else {
+      for (int g = 0; g < G; ++g) {
+        const float4 x = ps4[32 * g];
+        acc(x.x);
+        acc(x.y);
+        acc(x.z);
+        acc(x.w);
       }
     }
-    if (!found) {
-      // General path: bisection over the fp32 bit patterns until the interval [lo, hi)
-      // where the mass at or above crosses thr holds at most kSelCand blocks, then the
-      // candidates are ranked (value descending, index ascending) and walked from
-      // mass(P >= hi); the last kept candidate is the cut.
-      auto mass_cnt_ge = [&](uint32_t k, int* cnt) {
-        float acc = 0.f;
-        int c = 0;
+    if (prm.thr_mode != 0) break;                  // thr >= 1: keep all; thr <= 0: none
+    cm = __reduce_add_sync(0xffffffffu, cm);
+    mm = warp_sum(mm);
+    if (mm >= thr) {
+      lo = probe;
+      mlo = mm;
+      clo = cm;
+      phase = 3;
+    } else if (phase == 0) {
+      hi = probe;
+      mhi = mm;
+      chi = cm;
+      phase = 1;
+      probe = __float_as_uint(0.5f * (1.f - thr) / static_cast<float>(nb));
+      continue;
+    } else if (phase == 1) {
+      phase = 2;
+      probe = 0u;
+      continue;
+    } else if (phase == 2) {
+      break;                                       // total mass below thr: no bracket
+    } else {
+      hi = probe;
+      mhi = mm;
+      chi = cm;
+    }
+    if (clo - chi <= kSelCand || hi - lo <= 1u) {
+      bracket = clo - chi <= kSelCand;
+      break;
+    }
+    const uint32_t w = hi - lo;
+    const float f = fminf(fmaxf((mlo - thr) / (mlo - mhi), 0.25f), 0.75f);
+    probe = lo + min(max(static_cast<uint32_t>(static_cast<float>(w) * f), 1u), w - 1u);
+  }
+  if (prm.thr_mode != 0) {
+    certified = true;
+    kcut = prm.thr_mode > 0 ? 0u : 0xFFFFFFFFu;
+  } else if (bracket) {
+    // gather the candidates in index order into this warp's slots; the largest value
+    // below the bracket is the next value after the last candidate
+    uint32_t* ck = cand_key[wslot];
+    int* ci = cand_idx[wslot];
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int ncand = 0;
+    float below = 0.f;
+    for (int g = 0; g < G; ++g) {
+      const float4 x = ps4[32 * g];
+      const float v[4] = {x.x, x.y, x.z, x.w};
+      bool in[4];
+      bool any = false;
 #pragma unroll
-        for (int t = 0; t < TPL; ++t) {
-          const bool ge = __float_as_uint(p[t]) >= k;
-          acc += ge ? p[t] : 0.f;
-          c += ge ? 1 : 0;
-        }
-        *cnt = __reduce_add_sync(0xffffffffu, c);
-        return warp_sum(acc);
-      };
-      int clo = 0, chi = 0;
-      if (mass_cnt_ge(0u, &clo) >= thr) {
-        uint32_t lo = 0u, hi = 0x3F800001u;      // mass_ge(lo) >= thr > mass_ge(hi)
-        float mass_hi = 0.f;
-        while (clo - chi > kSelCand && hi - lo > 1u) {
-          const uint32_t mid = lo + ((hi - lo) >> 1);
-          int cm = 0;
-          const float mm = mass_cnt_ge(mid, &cm);
-          if (mm >= thr) {
-            lo = mid;
-            clo = cm;
-          } else {
-            hi = mid;
-            chi = cm;
-            mass_hi = mm;
-          }
-        }
-        if (clo - chi <= kSelCand) {
-          // gather the candidates in index order: candidate n goes to lane n (each lane
-          // holds the blocks lane + 32 t)
-          uint32_t ck = 0u;
-          int ci = 0x7FFFFFFF;
-          int ncand = 0;
-          float below = 0.f;                      // largest value below the interval
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t key = __float_as_uint(v[c]);
+        const bool valid = lane + 32 * (4 * g + c) < nb;
+        in[c] = valid && key >= lo && key < hi;
+        if (valid && key < lo) below = fmaxf(below, v[c]);
+        any = any || in[c];
+      }
+      if (__any_sync(0xffffffffu, any)) {
 #pragma unroll
-          for (int t = 0; t < TPL; ++t) {
-            const uint32_t key = __float_as_uint(p[t]);
-            const bool valid = lane + 32 * t < nb;
-            const bool in = valid && key >= lo && key < hi;
-            if (valid && key < lo) below = fmaxf(below, p[t]);
-            uint32_t bal = __ballot_sync(0xffffffffu, in);
-            while (bal != 0u) {                   // warp-uniform
-              const int src = __ffs(bal) - 1;
-              bal &= bal - 1u;
-              const uint32_t kv = __shfl_sync(0xffffffffu, key, src);
-              if (lane == ncand) {
-                ck = kv;
-                ci = src + 32 * t;
-              }
-              ++ncand;
-            }
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t bal = __ballot_sync(0xffffffffu, in[c]);
+          if (in[c]) {
+            const int pos = ncand + __popc(bal & lt_mask);
+            ck[pos] = __float_as_uint(v[c]);
+            ci[pos] = lane + 32 * (4 * g + c);
           }
-          below = warp_max(below);
-          // rank and exclusive mass of each candidate (lanes 0..ncand-1)
-          int rank = 0;
-          for (int d = 0; d < ncand; ++d) {
-            const uint32_t kd = __shfl_sync(0xffffffffu, ck, d);
-            const int id = __shfl_sync(0xffffffffu, ci, d);
-            rank += (lane < ncand && (kd > ck || (kd == ck && id < ci))) ? 1 : 0;
-          }
-          float e = mass_hi;
-          for (int d = 0; d < ncand; ++d) {
-            const int rd = __shfl_sync(0xffffffffu, rank, d);
-            const float pd = __uint_as_float(__shfl_sync(0xffffffffu, ck, d));
-            if (lane < ncand && rd < rank) e += pd;
-          }
-          // the cut: the candidate whose exclusive mass is below thr and inclusive mass
-          // reaches it
-          const float pc = __uint_as_float(ck);
-          const bool is_cut = lane < ncand && e < thr && e + pc >= thr;
-          const uint32_t cb = __ballot_sync(0xffffffffu, is_cut);
-          if (cb != 0u) {
-            const int cl = __ffs(cb) - 1;
-            const int crank = __shfl_sync(0xffffffffu, rank, cl);
-            const float e_above = __shfl_sync(0xffffffffu, e, cl);
-            const float p_cut = __uint_as_float(__shfl_sync(0xffffffffu, ck, cl));
-            // next value below the cut: the candidate ranked right after it, else the
-            // largest value below the interval
-            float p_next = below;
-            int n_at = 0;
-            for (int d = 0; d < ncand; ++d) {
-              const int rd = __shfl_sync(0xffffffffu, rank, d);
-              const float pd = __uint_as_float(__shfl_sync(0xffffffffu, ck, d));
-              if (rd == crank + 1) p_next = pd;
-              n_at += pd == p_cut ? 1 : 0;
-            }
-            kcut = __float_as_uint(p_cut);
-            certified = certify(e_above, e_above + p_cut, p_cut, p_next, n_at);
-          }
+          ncand += __popc(bal);
         }
       }
+    }
+    below = warp_max(below);
+    __syncwarp();
+    // lane n < ncand: rank of candidate n (value descending, index ascending) and its
+    // exclusive ranked mass, mass(P >= hi) plus the candidates ranked before it (added in
+    // index order)
+    const uint32_t kn = lane < ncand ? ck[lane] : 0u;
+    const int in_ = lane < ncand ? ci[lane] : 0x7FFFFFFF;
+    int rank = 0;
+    float e = mhi;
+    for (int d = 0; d < ncand; ++d) {
+      const uint32_t kd = ck[d];
+      const bool before = kd > kn || (kd == kn && ci[d] < in_);
+      rank += before ? 1 : 0;
+      e += before ? __uint_as_float(kd) : 0.f;
+    }
+    __syncwarp();
+    // the cut: the candidate whose exclusive mass is below thr and inclusive mass reaches it
+    const float pc = __uint_as_float(kn);
+    const uint32_t cb = __ballot_sync(0xffffffffu, lane < ncand && e < thr && e + pc >= thr);
+    if (cb != 0u) {
+      const int cl = __ffs(cb) - 1;
+      const int crank = __shfl_sync(0xffffffffu, rank, cl);
+      const float e_above = __shfl_sync(0xffffffffu, e, cl);
+      const float p_cut = __shfl_sync(0xffffffffu, pc, cl);
+      // next value below the cut: the candidate ranked right after it, else the largest
+      // value below the bracket; n_at: candidates equal to the cut value
+      const uint32_t nxt = __ballot_sync(0xffffffffu, lane < ncand && rank == crank + 1);
+      const float p_next = nxt != 0u ? __shfl_sync(0xffffffffu, pc, __ffs(nxt) - 1) : below;
+      const int n_at = __popc(__ballot_sync(0xffffffffu, lane < ncand && pc == p_cut));
+      kcut = __float_as_uint(p_cut);
+      // Certificate for the cut: the kept set {P >= p_cut} must have exact mass > thr, and
+      // without its (exactly) smallest member -- at most e_above + eta + rho p_cut --
+      // exact mass < thr.
+      certified = (thr - e_above > eta + rho * p_cut) && (e_above + p_cut - thr > eta) &&
+                  n_at == 1 && (p_cut - p_next > 2.f * rho * p_cut);
     }
   }
   if (!certified) {
@@ -427,38 +490,77 @@ __global__ void __launch_bounds__(256) mask_select_kernel(const SelectParams prm
     }
     return;
   }
-  // Emit: keep P >= P_c, OR the static window.
-  const int ti = i / (prm.Hb * prm.Wb), hi_ = (i / prm.Wb) % prm.Hb, wi = i % prm.Wb;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int run = 0;
-  uint32_t word[(TPL + 31) / 32];                     // lane l keeps bitmask word l + 32 w
-#pragma unroll
-  for (int w = 0; w < (TPL + 31) / 32; ++w) word[w] = 0u;
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    if (t >= prm.nw) break;
-    const int j = lane + 32 * t;
-    bool k = (j < nb) && (__float_as_uint(p[t]) >= kcut);
-    if (prm.sta_on && j < nb) {
-      const int tj = j / (prm.Hb * prm.Wb), hj = (j / prm.Wb) % prm.Hb, wj = j % prm.Wb;
-      k = k || (abs(ti - tj) <= prm.wt2 && abs(hi_ - hj) <= prm.wh2 && abs(wi - wj) <= prm.ww2);
-    }
-    const uint32_t kb = __ballot_sync(0xffffffffu, k);
-    if (lane == (t & 31)) word[t >> 5] = kb;
-    if (prm.row_idx != nullptr && k) prm.row_idx[(bh * nb + i) * static_cast<long long>(nb) + run + __popc(kb & lt_mask)] = j;
-    run += __popc(kb);
+  // ---- emit: keep P >= P_c, OR the static window ------------------------------------
+  // The window test follows block j = lane + 32 t through its (frame, row, column)
+  // coordinates by adding those of 32 with carries (no division per block).
+  const int nw = prm.nw;
+  const bool win = prm.sta_on != 0;
+  int ti = 0, hi_ = 0, wi = 0, tj = 0, hj = 0, wj = 0, dt = 0, dh = 0, dw = 0;
+  if (win) {
+    const int HW = prm.Hb * prm.Wb;
+    ti = i / HW;
+    hi_ = (i / prm.Wb) % prm.Hb;
+    wi = i % prm.Wb;
+    tj = lane / HW;
+    hj = (lane / prm.Wb) % prm.Hb;
+    wj = lane % prm.Wb;
+    dt = 32 / HW;
+    dh = (32 / prm.Wb) % prm.Hb;
+    dw = 32 % prm.Wb;
   }
-  // the row's bitmask words in one coalesced store
-  uint32_t* brow = prm.bits + (bh * nb + i) * prm.nw;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int32_t* ridx = prm.row_idx != nullptr ? prm.row_idx + (bh * nb + i) * static_cast<long long>(nb) : nullptr;
+  int run = 0;
+  for (int g = 0; 4 * g < nw; ++g) {
+    const float4 x = ps4[32 * g];
+    const float v[4] = {x.x, x.y, x.z, x.w};
+    uint32_t kb[4];
 #pragma unroll
-  for (int w = 0; w < (TPL + 31) / 32; ++w)
-    if (lane + 32 * w < prm.nw) brow[lane + 32 * w] = word[w];
-  if (prm.row_cnt != nullptr && lane == 0) prm.row_cnt[bh * nb + i] = run;
+    for (int c = 0; c < 4; ++c) {
+      const int j = lane + 32 * (4 * g + c);
+      bool k = j < nb && __float_as_uint(v[c]) >= kcut;
+      if (win) {
+        k = k || (j < nb && abs(ti - tj) <= prm.wt2 && abs(hi_ - hj) <= prm.wh2 && abs(wi - wj) <= prm.ww2);
+        wj += dw;
+        const int cw = wj >= prm.Wb ? 1 : 0;
+        wj -= cw * prm.Wb;
+        hj += dh + cw;
+        const int ch = hj >= prm.Hb ? 1 : 0;
+        hj -= ch * prm.Hb;
+        tj += dt + ch;
+      }
+      kb[c] = __ballot_sync(0xffffffffu, k);
+      if (ridx != nullptr) {
+        if (k) ridx[run + __popc(kb[c] & lt_mask)] = j;
+        run += __popc(kb[c]);
+      }
+    }
+    if (lane == 0) *reinterpret_cast<uint4*>(&words[wslot][4 * g]) = make_uint4(kb[0], kb[1], kb[2], kb[3]);
+  }
+  __syncwarp();
+  // the row's bitmask words in one coalesced store, and the kept count
+  uint32_t* brow = prm.bits + (bh * nb + i) * nw;
+  int cnt = 0;
+  for (int w = lane; w < nw; w += 32) {
+    const uint32_t wv = words[wslot][w];
+    brow[w] = wv;
+    cnt += __popc(wv);
+  }
+  if (prm.row_cnt != nullptr) {
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (lane == 0) prm.row_cnt[bh * nb + i] = cnt;
+  }
 }
 
-template <int TPL>
+size_t select_smem_bytes(int nbp) { return static_cast<size_t>(kSelWarps) * nbp * sizeof(float); }
+
 cudaError_t launch_select(const SelectParams& p, long long rows, cudaStream_t st) {
-  mask_select_kernel<TPL><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p, rows);
+  const size_t smem = select_smem_bytes(p.nbp);
+  cudaError_t e = cudaFuncSetAttribute(mask_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  mask_select_kernel<<<static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps), kSelWarps * 32, smem, st>>>(
+      p, rows);
   return cudaGetLastError();
 }
 
@@ -522,12 +624,13 @@ cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d,
   cudaError_t e = cudaMemsetAsync(f.kmax, 0, static_cast<size_t>(d.BH) * 4, st);
   if (e != cudaSuccess) return e;
   const long long rows_pad = static_cast<long long>(d.BH) * nbp;
+  const int vec16 = ((reinterpret_cast<uintptr_t>(qp) | reinterpret_cast<uintptr_t>(kp)) & 15) == 0;
   if (d.D == 64)
     split_pools_kernel<64><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, st>>>(
-        qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax);
+        qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax, vec16);
   else
     split_pools_kernel<128><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, st>>>(
-        qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax);
+        qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax, vec16);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   CUtensorMap mqh, mql, mkh, mkl;
@@ -583,17 +686,7 @@ cudaError_t mask_fast_select(const Dims& d, double scale, double thr, const nabl
   p.thr_mode = thr >= 1.0 ? 1 : (thr <= 0.0 ? -1 : 0);
   p.scale = static_cast<float>(scale);
   const long long rows = static_cast<long long>(d.BH) * d.nb;
-  const int tpl = nbp / 32;
-  switch (tpl) {
-    case 8: e = launch_select<8>(p, rows, st); break;
-    case 16: e = launch_select<16>(p, rows, st); break;
-    case 24: e = launch_select<24>(p, rows, st); break;
-    case 32: e = launch_select<32>(p, rows, st); break;
-    case 40: e = launch_select<40>(p, rows, st); break;
-    case 48: e = launch_select<48>(p, rows, st); break;
-    case 56: e = launch_select<56>(p, rows, st); break;
-    default: e = launch_select<64>(p, rows, st); break;
-  }
+  e = launch_select(p, rows, st);
   *rescue_list = f.rlist;
   *rescue_cnt = f.rc;
   return e;
