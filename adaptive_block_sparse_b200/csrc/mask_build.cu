@@ -43,12 +43,13 @@ cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, dou
 namespace {
 
 constexpr int kThreads = 256;   // 8 warps; one pooled row per warp during selection
+                                // (two CTAs per SM where shared memory allows)
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowBudget = 163840;  // bytes of shared memory for the fp64 score rows
 constexpr int kCand = 16;       // the cut's search stops at this many candidates
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) mask_rows_kernel(
+__global__ void __launch_bounds__(kThreads, 2) mask_rows_kernel(
     const double* __restrict__ qpool, const double* __restrict__ kpool, int nb, int nw, int R,
     double scale, double thr, int sta_on, int wt2, int wh2, int ww2, int Hb, int Wb,
     uint32_t* __restrict__ bits, int32_t* __restrict__ row_idx, int32_t* __restrict__ row_cnt,
@@ -455,11 +456,15 @@ cudaError_t launch_mask_rows(const double* qp, const double* kp, const Dims& d, 
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int sta_on = (w.t | w.h | w.w) != 0;
-  // Listed rows: one CTA per SM walks the groups of every head (the counts are on the
-  // device); all rows: one CTA per group of R rows of each head.
-  int dev = 0, sms = 148;
+  // Listed rows: as many CTAs as fit on the GPU at once walk the groups of every head
+  // (the counts are on the device); all rows: one CTA per group of R rows of each head.
+  int dev = 0, sms = 148, per_sm = 1;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  dim3 grid(rlist != nullptr ? sms : (d.nb + R - 1) / R, rlist != nullptr ? 1 : d.BH);
+  if (rlist != nullptr &&
+      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mask_rows_kernel<D>, kThreads, smem) != cudaSuccess ||
+       per_sm < 1))
+    per_sm = 1;
+  dim3 grid(rlist != nullptr ? sms * per_sm : (d.nb + R - 1) / R, rlist != nullptr ? 1 : d.BH);
   mask_rows_kernel<D><<<grid, kThreads, smem, st>>>(qp, kp, d.nb, d.nw, R, scale, thr, sta_on,
                                                    w.t / 2, w.h / 2, w.w / 2, d.Hb, d.Wb, bits,
                                                    ridx, rcnt, rlist, rlist_cnt, d.BH);

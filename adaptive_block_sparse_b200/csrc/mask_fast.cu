@@ -14,8 +14,9 @@
 //     q = q_hi + q_lo + r (|r| <= 2^-22 |q|), padded to a multiple of 256 rows; row
 //     norms |q_i| and the per-head maximum |k_j| are kept for the error bound.
 //  2. pooled_logits_kernel: A = scale * (q_hi k_hi^T + (q_hi k_lo^T + q_lo k_hi^T)) with
-//     tcgen05 (M = 128, N = 256, K = 16 per instruction, fp32 accumulate in TMEM; the
-//     dominant q_hi k_hi^T term has its own accumulator), written to an fp32 scratch.
+//     tcgen05 (M = 128, N = 128, K = 16 per instruction, fp32 accumulate in TMEM; the
+//     dominant q_hi k_hi^T term has its own accumulator), written to an fp32 scratch by
+//     a persistent kernel that overlaps the key tiles' copies, the MMAs and the stores.
 //  3. mask_select_kernel: one warp per row: softmax in fp32; the cut value P_c (the
 //     smallest kept probability) from a bracket of fp32 bit patterns where the mass at
 //     or above crosses thr -- first guess one sixteenth of the row maximum, else a lower
@@ -39,6 +40,7 @@ namespace nabla {
 
 bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows,
                  bool fp16);
+bool make_map_f32(CUtensorMap* map, const void* base, long long rows, int D);
 
 namespace {
 
@@ -127,42 +129,68 @@ __global__ void __launch_bounds__(256) split_pools_kernel(
 // ------------------------------------------------------------------------------------
 // 2. pooled logits on the tensor cores
 // ------------------------------------------------------------------------------------
+// Persistent and pipelined: the (head, 128-row query tile, 128-column key tile) units
+// are split into equal contiguous ranges, one per CTA.  Warp 0 streams the key tiles
+// (fp16 hi and lo) through a two-stage TMA ring and reloads the query tile only when it
+// changes; warp 1 issues the MMAs into one of two TMEM accumulator pairs; warps 2-5
+// (one TMEM lane quadrant each) add the pair, scale, and store 32 x 32 fp32 boxes with
+// tiled TMA stores through swizzled staging, while the next unit's MMAs run.
 template <int D>
 struct LogitCfg {
   static constexpr int kPanels = D / 64;
-  static constexpr int kABytes = 128 * D * 2;    // one 128-row fp16 operand
-  static constexpr int kBBytes = 256 * D * 2;    // one 256-row fp16 operand
+  static constexpr int kTileBytes = 128 * D * 2;   // one 128-row fp16 operand (hi or lo)
   static constexpr int kOffQh = 0;
-  static constexpr int kOffQl = kOffQh + kABytes;
-  static constexpr int kOffKh = kOffQl + kABytes;
-  static constexpr int kOffKl = kOffKh + kBBytes;
-  static constexpr int kOffBar = kOffKl + kBBytes;
-  static constexpr int kSmemBytes = kOffBar + 64 + 1024;
+  static constexpr int kOffQl = kOffQh + kTileBytes;
+  static constexpr int kOffK = kOffQl + kTileBytes;        // 2 stages x (hi, lo)
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kOffStage = kOffK + 2 * kStageBytes; // 4 warps x 2 x 4 KB
+  static constexpr int kOffBar = kOffStage + 4 * 2 * 4096;
+  static constexpr int kSmemBytes = kOffBar + 128 + 1024;
 };
+constexpr int kLogitThreads = 192;
+
+__device__ __forceinline__ void bulk_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 
 template <int D>
-__global__ void __launch_bounds__(128, 1) pooled_logits_kernel(
+__global__ void __launch_bounds__(kLogitThreads, 1) pooled_logits_kernel(
     const __grid_constant__ CUtensorMap map_qh, const __grid_constant__ CUtensorMap map_ql,
     const __grid_constant__ CUtensorMap map_kh, const __grid_constant__ CUtensorMap map_kl,
-    float* __restrict__ logits, int nbp, float scale, uint32_t* status) {
+    const __grid_constant__ CUtensorMap map_out, int nbp, long long units, float scale,
+    uint32_t* status) {
   using C = LogitCfg<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* done = full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* k_full = bars;          // [2]
+  uint64_t* k_empty = bars + 2;     // [2]
+  uint64_t* acc_full = bars + 4;    // [2]
+  uint64_t* acc_empty = bars + 6;   // [2]
+  uint64_t* q_full = bars + 8;
+  uint64_t* q_empty = bars + 9;
+  uint64_t* mma_done = bars + 10;   // the MMA thread's last commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int it = blockIdx.x, jt = blockIdx.y;
-  const long long bh = blockIdx.z;
+  const int nt = nbp / 128;                        // query tiles = key tiles per head
+  const long long u0 = units * blockIdx.x / gridDim.x;
+  const long long u1 = units * (blockIdx.x + 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
-    mbar_init(full, 1);
-    mbar_init(done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 4);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(mma_done, 1);
     fence_mbarrier_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -172,66 +200,154 @@ __global__ void __launch_bounds__(128, 1) pooled_logits_kernel(
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // ---------------- producer ----------------
     if (lane == 0) {
-      const int arow = static_cast<int>(bh * nbp + it * 128);
-      const int brow = static_cast<int>(bh * nbp + jt * 256);
-      mbar_arrive_expect_tx(full, 2 * C::kABytes + 2 * C::kBBytes);
+      long long cur_q = -1;
+      int nq = 0;
+      long long k = 0;
+      bool ok = true;
+      for (long long u = u0; u < u1 && ok; ++u, ++k) {
+        const long long qt = u / nt;               // (head, query tile)
+        const int jt = static_cast<int>(u - qt * nt);
+        const long long bh = qt / nt;
+        const int it = static_cast<int>(qt - bh * nt);
+        if (qt != cur_q) {
+          if (nq > 0) ok = mbar_wait(q_empty, (nq - 1) & 1, status, kDevTimeoutTmaFull);
+          if (!ok) break;
+          mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
+          const int arow = static_cast<int>(bh * nbp + it * 128);
 #pragma unroll
-      for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_2d(smem + C::kOffQh + pn * 16384, &map_qh, full, pn * 64, arow);
-        tma_load_2d(smem + C::kOffQl + pn * 16384, &map_ql, full, pn * 64, arow);
-        tma_load_2d(smem + C::kOffKh + pn * 32768, &map_kh, full, pn * 64, brow);
-        tma_load_2d(smem + C::kOffKl + pn * 32768, &map_kl, full, pn * 64, brow);
-      }
-      const bool ok = mbar_wait(full, 0, status, kDevTimeoutTmaFull);
-      tc_fence_after();
-      if (ok) {
-        constexpr uint32_t idesc = idesc_f16_f32(128, 256, false, false);
-        const uint32_t qh = smem_u32(smem + C::kOffQh), ql = smem_u32(smem + C::kOffQl);
-        const uint32_t kh = smem_u32(smem + C::kOffKh), kl = smem_u32(smem + C::kOffKl);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int pn = kk >> 2, w = kk & 3;
-          mma_bf16_ss(tmem, sdesc_sw128(qh + pn * 16384 + w * 32, 16, 1024),
-                      sdesc_sw128(kh + pn * 32768 + w * 32, 16, 1024), idesc, kk > 0);
+          for (int pn = 0; pn < C::kPanels; ++pn) {
+            tma_load_2d(smem + C::kOffQh + pn * 16384, &map_qh, q_full, pn * 64, arow);
+            tma_load_2d(smem + C::kOffQl + pn * 16384, &map_ql, q_full, pn * 64, arow);
+          }
+          cur_q = qt;
+          ++nq;
         }
+        const int st = static_cast<int>(k & 1);
+        const long long use = k >> 1;
+        if (use > 0) ok = mbar_wait(&k_empty[st], static_cast<uint32_t>((use - 1) & 1), status, kDevTimeoutKvEmpty);
+        if (!ok) break;
+        unsigned char* kb = smem + C::kOffK + st * C::kStageBytes;
+        mbar_arrive_expect_tx(&k_full[st], 2 * C::kTileBytes);
+        const int brow = static_cast<int>(bh * nbp + jt * 128);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int pn = kk >> 2, w = kk & 3;
-          mma_bf16_ss(tmem + 256, sdesc_sw128(qh + pn * 16384 + w * 32, 16, 1024),
-                      sdesc_sw128(kl + pn * 32768 + w * 32, 16, 1024), idesc, kk > 0);
-          mma_bf16_ss(tmem + 256, sdesc_sw128(ql + pn * 16384 + w * 32, 16, 1024),
-                      sdesc_sw128(kh + pn * 32768 + w * 32, 16, 1024), idesc, 1u);
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_2d(kb + pn * 16384, &map_kh, &k_full[st], pn * 64, brow);
+          tma_load_2d(kb + C::kTileBytes + pn * 16384, &map_kl, &k_full[st], pn * 64, brow);
         }
       }
-      mma_commit(done);
+      // drain: every copy issued has landed before the CTA may exit (the MMA warp waits
+      // for them on the normal path; after an error it may have stopped early)
+      for (long long kk = k > 2 ? k - 2 : 0; kk < k; ++kk)
+        mbar_wait(&k_full[kk & 1], static_cast<uint32_t>((kk >> 1) & 1), nullptr, kDevTimeoutDrain);
+      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, nullptr, kDevTimeoutDrain);
     }
     __syncwarp();
-  }
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, status, kDevTimeoutSFull));
-  tc_fence_after();
-  if (ok) {
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int row = warp * 32 + lane;
-    float* dst = logits + (bh * nbp + it * 128 + row) * static_cast<long long>(nbp) + jt * 256;
-#pragma unroll 1
-    for (int c0 = 0; c0 < 256; c0 += 32) {
-      uint32_t a0[32], a1[32];
-      tmem_ld32(tmem + lane_base + c0, a0);
-      tmem_ld32(tmem + lane_base + 256 + c0, a1);
-      tmem_wait_ld();
-      float4* d4 = reinterpret_cast<float4*>(dst + c0);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(128, 128, false, false);
+      const uint32_t qh = smem_u32(smem + C::kOffQh), ql = smem_u32(smem + C::kOffQl);
+      long long cur_q = -1;
+      int nq = 0;
+      long long k = 0;
+      bool ok = true;
+      for (long long u = u0; u < u1 && ok; ++u, ++k) {
+        const long long qt = u / nt;
+        if (qt != cur_q) {
+          ok = mbar_wait(q_full, nq & 1, status, kDevTimeoutQFull);
+          if (!ok) break;
+          cur_q = qt;
+          ++nq;
+        }
+        const int st = static_cast<int>(k & 1);
+        const long long use = k >> 1;
+        ok = mbar_wait(&k_full[st], static_cast<uint32_t>(use & 1), status, kDevTimeoutTmaFull);
+        if (ok && use > 0) ok = mbar_wait(&acc_empty[st], static_cast<uint32_t>((use - 1) & 1), status, kDevTimeoutOBar);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kh = smem_u32(smem + C::kOffK + st * C::kStageBytes);
+        const uint32_t kl = kh + C::kTileBytes;
+        const uint32_t acc = tmem + static_cast<uint32_t>(st * 256);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        d4[c] = make_float4((__uint_as_float(a0[4 * c]) + __uint_as_float(a1[4 * c])) * scale,
-                            (__uint_as_float(a0[4 * c + 1]) + __uint_as_float(a1[4 * c + 1])) * scale,
-                            (__uint_as_float(a0[4 * c + 2]) + __uint_as_float(a1[4 * c + 2])) * scale,
-                            (__uint_as_float(a0[4 * c + 3]) + __uint_as_float(a1[4 * c + 3])) * scale);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int pn = kk >> 2, w = kk & 3;
+          mma_bf16_ss(acc, sdesc_sw128(qh + pn * 16384 + w * 32, 16, 1024),
+                      sdesc_sw128(kh + pn * 16384 + w * 32, 16, 1024), idesc, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int pn = kk >> 2, w = kk & 3;
+          mma_bf16_ss(acc + 128, sdesc_sw128(qh + pn * 16384 + w * 32, 16, 1024),
+                      sdesc_sw128(kl + pn * 16384 + w * 32, 16, 1024), idesc, kk > 0);
+          mma_bf16_ss(acc + 128, sdesc_sw128(ql + pn * 16384 + w * 32, 16, 1024),
+                      sdesc_sw128(kh + pn * 16384 + w * 32, 16, 1024), idesc, 1u);
+        }
+        mma_commit(&k_empty[st]);
+        mma_commit(&acc_full[st]);
+        if (u + 1 == u1 || (u + 1) / nt != qt) mma_commit(q_empty);
+      }
+      // every MMA issued (and every commit before this one) has completed before the
+      // accumulators are freed and the CTA exits
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, nullptr, kDevTimeoutDrain);
     }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2-5: TMEM lane quadrant warp % 4) ----------------
+    const int q4 = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    unsigned char* stage0 = smem + C::kOffStage + (warp - 2) * 8192;
+    long long k = 0;
+    int nstore = 0;
+    for (long long u = u0; u < u1; ++u, ++k) {
+      const long long qt = u / nt;
+      const int jt = static_cast<int>(u - qt * nt);
+      const long long bh = qt / nt;
+      const int it = static_cast<int>(qt - bh * nt);
+      const int st = static_cast<int>(k & 1);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[st], static_cast<uint32_t>((k >> 1) & 1), status,
+                                                        kDevTimeoutSFull));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + lane_base + static_cast<uint32_t>(st * 256);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t a0[32], a1[32];
+        tmem_ld32(acc + 32 * c, a0);
+        tmem_ld32(acc + 128 + 32 * c, a1);
+        tmem_wait_ld();
+        if (c == 3) {                              // the pair is read: release it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[st]);
+        }
+        unsigned char* stage = stage0 + (nstore & 1) * 4096;
+        if (lane == 0) bulk_wait_read_le1();       // the copy from this buffer has read it
+        __syncwarp();
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<float4*>(stage + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+              make_float4((__uint_as_float(a0[4 * ch]) + __uint_as_float(a1[4 * ch])) * scale,
+                          (__uint_as_float(a0[4 * ch + 1]) + __uint_as_float(a1[4 * ch + 1])) * scale,
+                          (__uint_as_float(a0[4 * ch + 2]) + __uint_as_float(a1[4 * ch + 2])) * scale,
+                          (__uint_as_float(a0[4 * ch + 3]) + __uint_as_float(a1[4 * ch + 3])) * scale);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&map_out, stage, jt * 128 + 32 * c, static_cast<int>(bh * nbp + it * 128 + 32 * q4));
+          bulk_commit_group();
+        }
+        ++nstore;
+      }
+    }
+    if (lane == 0) bulk_wait_all();                // the stores have landed
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -633,23 +749,27 @@ cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d,
         qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax, vec16);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  CUtensorMap mqh, mql, mkh, mkl;
+  CUtensorMap mqh, mql, mkh, mkl, mout;
   if (!(make_map_16(&mqh, f.qh, rows_pad, d.D, 128, true) && make_map_16(&mql, f.ql, rows_pad, d.D, 128, true) &&
-        make_map_16(&mkh, f.kh, rows_pad, d.D, 256, true) && make_map_16(&mkl, f.kl, rows_pad, d.D, 256, true)))
+        make_map_16(&mkh, f.kh, rows_pad, d.D, 128, true) && make_map_16(&mkl, f.kl, rows_pad, d.D, 128, true) &&
+        make_map_f32(&mout, f.logits, rows_pad, nbp)))
     return cudaErrorInvalidValue;
-  dim3 grid(nbp / 128, nbp / 256, d.BH);
+  const long long units = static_cast<long long>(d.BH) * (nbp / 128) * (nbp / 128);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
   if (d.D == 64) {
     e = cudaFuncSetAttribute(pooled_logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              LogitCfg<64>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    pooled_logits_kernel<64><<<grid, 128, LogitCfg<64>::kSmemBytes, st>>>(
-        mqh, mql, mkh, mkl, f.logits, nbp, static_cast<float>(scale), status);
+    pooled_logits_kernel<64><<<grid, kLogitThreads, LogitCfg<64>::kSmemBytes, st>>>(
+        mqh, mql, mkh, mkl, mout, nbp, units, static_cast<float>(scale), status);
   } else {
     e = cudaFuncSetAttribute(pooled_logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              LogitCfg<128>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    pooled_logits_kernel<128><<<grid, 128, LogitCfg<128>::kSmemBytes, st>>>(
-        mqh, mql, mkh, mkl, f.logits, nbp, static_cast<float>(scale), status);
+    pooled_logits_kernel<128><<<grid, kLogitThreads, LogitCfg<128>::kSmemBytes, st>>>(
+        mqh, mql, mkh, mkl, mout, nbp, units, static_cast<float>(scale), status);
   }
   return cudaGetLastError();
 }
