@@ -167,6 +167,47 @@ def test_mask_parity(data, name, thr, window):
     assert torch.equal(bits2, bits)
 
 
+# Degenerate rows for the cut: head 0 has Q = K = 0 (every block of a row has the same
+# probability: all ties, decided by block index), head 1 repeats every even patch column
+# of K in the odd one (pooled keys equal in pairs: ties at every rank), head 2 has Q and K
+# scaled by 8 (very sharp rows).  nb = 4 x 8 x 8 = 256.
+DEGEN = Workload("degen", B=1, H=3, T=4, Hg=64, W=64, D=128, thrs=(0.8,), sigma=(1.5, 1.5), seed=81)
+
+
+def _degenerate_qk():
+    wl = DEGEN
+    q, k, _ = make_qkv(wl, device=DEV)
+    q[0, 0].zero_()
+    k[0, 0].zero_()
+    kv = k[0, 1].view(wl.T, wl.Hg, wl.W // 16, 2, 8, wl.D)
+    kv[:, :, :, 1] = kv[:, :, :, 0]
+    q[0, 2] = (q[0, 2].float() * 8).to(torch.bfloat16)
+    k[0, 2] = (k[0, 2].float() * 8).to(torch.bfloat16)
+    return q, k
+
+
+@pytest.mark.parametrize("thr", [0.3, 0.5, 0.8, 0.95])
+def test_mask_degenerate_rows(thr):
+    wl = DEGEN
+    shape = shape_of(wl)
+    q, k = _degenerate_qk()
+    qf, qp = gpu_reorder(q, shape, pool=True)
+    kf, kp = gpu_reorder(k, shape, pool=True)
+    bits, ridx, rcnt, cidx, ccnt = gpu_mask(qf, kf, shape, thr)
+    gm = bits_to_mask(bits, wl.nb)
+    om, E = oracle_mask_per_head(q.cpu(), k.cpu(), wl, thr, (0, 0, 0))
+    mism, amb = check_mask(gm, om, E, thr)
+    print(f"degenerate thr={thr}: kept per head {gm.sum(axis=(2, 3)).tolist()}, "
+          f"near-threshold {amb}, differing {mism}")
+    # all-tied rows keep the first blocks by index: E_j = j / nb < thr
+    nkeep = int(np.sum(np.arange(wl.nb) / wl.nb < thr))
+    assert np.array_equal(gm[0, 0], np.broadcast_to(np.arange(wl.nb) < nkeep, (wl.nb, wl.nb)))
+    check_lists(ridx, rcnt, gm)
+    check_lists(cidx, ccnt, np.swapaxes(gm, -1, -2))
+    bits2, *_ = gpu_mask(None, None, shape, thr, cols=False, q_pool=qp, k_pool=kp)
+    assert torch.equal(bits2, bits)
+
+
 def _fwd_case(data, wl, thr, window, o_dtype, v_dtype=torch.float16):
     m = nbl()
     shape = shape_of(wl)
