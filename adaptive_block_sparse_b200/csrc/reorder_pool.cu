@@ -81,6 +81,65 @@ __global__ void __launch_bounds__(kThreads) reorder_pool_kernel(
   }
 }
 
+// Pool only (no copy written): lane l of a warp owns the 16-byte column chunk c = l % C
+// (C = D / 8 chunks, 8 columns each) of block (l / C) of the warp's 32 / C blocks, reads
+// that chunk of the block's 64 tokens straight from memory (the C lanes of a block read
+// one token's whole row: 2 x 256-byte runs per load at D = 128) and keeps eight fp64
+// sums, each over its column in token order: the same sums, in the same order, as the
+// copy-and-pool kernel's, without staging through shared memory.
+template <int D, bool GATHER>
+__global__ void __launch_bounds__(kThreads) pool_only_kernel(
+    const uint4* __restrict__ src, double* __restrict__ pool_out, int Hg, int W, int Hb, int Wb,
+    int nb, long long n_blocks) {
+  constexpr int C = D / 8;                 // 16-byte chunks per token row
+  constexpr int BPW = 32 / C;              // blocks per warp
+  const int lane = threadIdx.x & 31;
+  const int c = lane % C;
+  const long long g = (static_cast<long long>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5)) * BPW + lane / C;
+  if (g >= n_blocks) return;               // whole block groups of lanes leave together
+  const long long bh = g / nb;
+  const int blk = static_cast<int>(g - bh * nb);
+  const long long S = static_cast<long long>(nb) * 64;
+  const int t = blk / (Hb * Wb);
+  const int rem = blk - t * (Hb * Wb);
+  const int hb = rem / Wb;
+  const int wb = rem - hb * Wb;
+  const uint4* base = src + bh * S * C + c;
+  double acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.0;
+#pragma unroll 2
+  for (int r = 0; r < 8; ++r) {            // patch row r: tokens 8 r .. 8 r + 7 of the block
+    const long long tok0 = GATHER ? (static_cast<long long>(t) * Hg + hb * 8 + r) * W + wb * 8
+                                  : static_cast<long long>(blk) * 64 + 8 * r;
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(base + (tok0 + u) * C);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[2 * k] += static_cast<double>(__uint_as_float(w[k] << 16));
+        acc[2 * k + 1] += static_cast<double>(__uint_as_float(w[k] & 0xFFFF0000u));
+      }
+    }
+  }
+  double* out = pool_out + g * D + c * 8;   // 8-byte stores: the pool may be 8-byte aligned
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out[k] = acc[k] / 64.0;
+}
+
+template <int D, bool GATHER>
+cudaError_t go_pool(const void* src, double* pool, const Dims& d, cudaStream_t st) {
+  const long long n_blocks = static_cast<long long>(d.BH) * d.nb;
+  constexpr int kBlocksPerCta = (kThreads / 32) * (32 / (D / 8));
+  const long long grid = (n_blocks + kBlocksPerCta - 1) / kBlocksPerCta;
+  pool_only_kernel<D, GATHER><<<static_cast<unsigned>(grid), kThreads, 0, st>>>(
+      static_cast<const uint4*>(src), pool, d.Hg, d.W, d.Hb, d.Wb, d.nb, n_blocks);
+  return cudaGetLastError();
+}
+
 template <int D, int ESZ, bool GATHER, bool SCATTER, bool WRITE, bool POOL, bool TO_F16>
 cudaError_t go(const void* src, void* dst, double* pool, const Dims& d, cudaStream_t st) {
   dim3 grid(d.nb, d.BH);
@@ -97,7 +156,7 @@ cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims&
                     : go<D, 2, false, true, true, false, false>(src, dst, nullptr, d, st);
   }
   if (dst == nullptr)   // pool only: the fp64 block means of a natural-order tensor
-    return go<D, 2, true, false, false, true, false>(src, nullptr, pool, d, st);
+    return go_pool<D, true>(src, pool, d, st);
   if (to_f16) {
     return pool ? go<D, 2, true, false, true, true, true>(src, dst, pool, d, st)
                 : go<D, 2, true, false, true, false, true>(src, dst, nullptr, d, st);
@@ -110,8 +169,7 @@ cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims&
 
 // Pools a reordered bf16 tensor into fp64 block means (used by the mask build).
 cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st) {
-  return d.D == 64 ? go<64, 2, false, false, false, true, false>(x, nullptr, pool, d, st)
-                   : go<128, 2, false, false, false, true, false>(x, nullptr, pool, d, st);
+  return d.D == 64 ? go_pool<64, false>(x, pool, d, st) : go_pool<128, false>(x, pool, d, st);
 }
 
 }  // namespace nabla
