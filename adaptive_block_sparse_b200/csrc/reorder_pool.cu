@@ -10,7 +10,9 @@
 // 8 * D * 2 bytes, so every warp issues 16-byte loads over 512-byte contiguous spans;
 // the reordered block is one contiguous 64 * D * 2-byte run.  The optional pool sums
 // the block's 64 rows column by column in fp64, in token order (exact for bf16), and
-// divides by 64.
+// divides by 64.  When no copy is written (the pool alone), pool_only_kernel skips the
+// shared-memory staging: each lane reads one 16-byte column chunk of its block's tokens
+// and keeps the eight column sums itself, in the same order.
 #include "common.cuh"
 
 namespace nabla {
