@@ -42,7 +42,8 @@ EXPORTED = (
     "nabla_status_string", "nabla_reorder", "nabla_mask_workspace_bytes", "nabla_build_mask",
     "nabla_mask_lists", "nabla_fwd_workspace_bytes", "nabla_attn_fwd",
     "nabla_bwd_workspace_bytes", "nabla_attn_bwd", "nabla_read_device_status",
-    "nabla_attn_fwd_noalloc", "nabla_build_mask_sweep", "nabla_selftest_bounded_wait",
+    "nabla_attn_fwd_noalloc", "nabla_attn_fwd_noalloc_status", "nabla_build_mask_sweep",
+    "nabla_selftest_bounded_wait",
 )
 
 
@@ -79,6 +80,7 @@ _sigs = {
     "nabla_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape,
                                               ctypes.c_float, _vp, ctypes.c_int, _vp, ctypes.c_int,
                                               _vp]),
+    "nabla_attn_fwd_noalloc_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _vp]),
 }
 
 
@@ -304,6 +306,16 @@ def nabla_attn_fwd_noalloc(q, k, v, mask_bits, shape: Shape, o, lse=None, scale=
         float(scale), _ptr(o), dtype_code(o), _ptr(lse), int(layout), _stream(stream)),
         "nabla_attn_fwd_noalloc")
     return o, lse
+
+
+def nabla_attn_fwd_noalloc_status(stream=None) -> int:
+    """Device status word of the last nabla_attn_fwd_noalloc call on the current device
+    (0 = fine); waits for the stream and clears the word."""
+    code = ctypes.c_uint32(0)
+    rc = load_library().nabla_attn_fwd_noalloc_status(ctypes.byref(code), _stream(stream))
+    if rc not in (NABLA_OK, NABLA_ERR_DEVICE_CHECK):
+        raise NablaError(rc, "nabla_attn_fwd_noalloc_status")
+    return int(code.value)
 
 
 def nabla_read_device_status(workspace, stream=None) -> int:

@@ -350,41 +350,89 @@ def oracle_sample(wl, q_nat, k_nat, v_nat, rcnt, budget_s=20.0):
 
 
 # --------------------------------------------------------------------------------------
+def workload_config(wl, thr, world, natural, scaling="weak"):
+    """The ``config`` object of a bench line; both arms print the same one."""
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.T, wl.Hg, wl.W],
+            "D": wl.D, "P": wl.P, "thr": thr, "sta": list(wl.window),
+            "step": ("pool Q/K, mask, attn fwd on natural-order Q/K/V" if natural
+                     else "reorder+pool, mask, attn fwd, attn bwd"),
+            "l2": "inputs larger than L2 (no flush)",
+            "parallelism": (f"heads-replicated x{world}" if scaling == "weak"
+                            else f"heads split over {world} ranks (LPT by kept tiles)")}
+
+
 def run_reference(args, wl, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the host cores.
+
+    Set-up (untimed): the inputs of the GPU arm (drawn on the GPU when there is one, so
+    that both arms see the same tensors; on the host otherwise) and the oracle mask of
+    every head, which gives the exact kept-tile count.  Each step is a bounded 1/(B*H)
+    slice of the workload, timed as it runs: the oracle mask of one head (heads in turn)
+    plus the oracle forward over query blocks drawn in a fixed shuffled order across all
+    heads until they hold (kept tiles) / (B*H) tiles; the attention time is scaled by the
+    small overshoot of the last block.  value = the slice's kept-tile FLOPs / its time.
+    """
     if rank != 0:
         return
-    torch.manual_seed(0)
-    q, k, v = make_qkv(wl, device="cpu", heads=list(range(min(4, wl.B * wl.H))))
     import oracle
+    BH = wl.B * wl.H
     thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
-    # kept tiles of the sampled heads, scaled to all heads
-    kept = 0
-    nh = min(4, wl.B * wl.H)
-    for bh in range(nh):
+    scale = 1 / math.sqrt(wl.D)
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    q, k, v = (t.cpu() for t in make_qkv(wl, device=gen_dev))
+    cores = len(os.sched_getaffinity(0))
+    heads = []
+    kept_all = 0
+    for bh in range(BH):
         b, h = divmod(bh, wl.H)
-        qf = oracle.reorder(q[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
-        kf = oracle.reorder(k[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)
-        mk, _, _ = oracle.nabla_mask(qf, kf, wl.T, wl.Hg, wl.W, wl.P, thr, wl.window)
-        kept += int(mk.sum())
-    kept_all = kept * (wl.B * wl.H) / nh
-    times = []
-    cb = None
+        qf, kf, vf = (oracle.reorder(t[b, h].double().numpy()[None, None], wl.T, wl.Hg, wl.W, wl.P)[0, 0]
+                      for t in (q, k, v))
+        heads.append((qf, kf, vf))
+    masks = []
+    for bh in range(BH):
+        qf, kf, _ = heads[bh]
+        mk, _, _ = oracle.nabla_mask(qf[None, None], kf[None, None], wl.T, wl.Hg, wl.W, wl.P, thr, wl.window)
+        masks.append(mk[0, 0])
+        kept_all += int(mk.sum())
+    budget = kept_all / BH
+    order = [(bh, i) for bh in range(BH) for i in range(wl.nb) if masks[bh][i].any()]
+    np.random.default_rng(0).shuffle(order)
+    fl = 4.0 * wl.N * wl.N * wl.D
+    cursor = 0
+    times, samples = [], []
     for s in range(args.warmup + args.steps):
+        bh_m = s % BH
+        qf, kf, _ = heads[bh_m]
         t0 = time.perf_counter()
-        cb = oracle_sample(wl, q, k, v, kept_all, budget_s=min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+        oracle.nabla_mask(qf[None, None], kf[None, None], wl.T, wl.Hg, wl.W, wl.P, thr, wl.window)
+        t_mask = time.perf_counter() - t0
+        done = 0
+        t1 = time.perf_counter()
+        while done < budget:
+            bh, i = order[cursor % len(order)]
+            cursor += 1
+            qh, kh, vh = heads[bh]
+            rows = np.arange(i * wl.N, (i + 1) * wl.N)
+            oracle.block_sparse_attention_rows(qh, kh, vh, masks[bh], wl.N, scale, rows)
+            done += int(masks[bh][i].sum())
+        t_attn = (time.perf_counter() - t1) * budget / done
         if s >= args.warmup:
-            times.append(cb["est_step_s"])
-        del t0
-    est = statistics.median(times)
-    flops = 4.0 * 64 * 64 * wl.D * kept_all
-    val = flops / est / 1e12
+            times.append(t_mask + t_attn)
+            samples.append((t_mask, t_attn))
+    step_s = statistics.median(times)
+    val = budget * fl / step_s / 1e12
+    sample = (f"1/{BH} of the workload per step: oracle mask of one head (median "
+              f"{statistics.median(t for t, _ in samples):.2f} s) + oracle forward over {budget:.0f} "
+              f"kept tiles (median {statistics.median(a for _, a in samples):.2f} s); kept tiles of all "
+              f"{BH} heads from the oracle masks: {kept_all}")
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": wl.name, "B": wl.B, "H": wl.H,
-                                             "grid": [wl.T, wl.Hg, wl.W], "D": wl.D,
-                                             "thr": thr, "sta": list(wl.window)},
-            "cpu_baseline": {k2: cb[k2] for k2 in ("kind", "cores", "sample")} | {"value": val, "unit": "TFLOP/s"},
+            "data": "synthetic",
+            "config": workload_config(wl, thr, world, not wl.backward),
+            "kept_tiles": kept_all,
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": val,
+                             "unit": "TFLOP/s"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -399,6 +447,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the side measurements (training step, forward vs sparsity)")
     args = ap.parse_args()
     wl = WORKLOADS[args.config]
     world, rank, local = init_dist() if args.impl == "ours" else (
@@ -501,8 +551,80 @@ def main():
     dense_ms = time_call(dense_call, dense_iters, warm=1)
     dense_tflops = BH * nb * nb * fl_fwd / (dense_ms * 1e-3) / 1e12
     path.check_status()
-    # restore the NABLA lists (the dense run reused the output buffers only)
     del dense_bits
+
+    # per-head sparsity (from the step's row counts) and the near-threshold blocks: blocks
+    # (outside the static window) whose ranked mass E lies within 1e-6 of thr, counted as
+    # kept(thr + 1e-6) - kept(thr - 1e-6) from two exact masks of the step's pooled map
+    head_kept = path.rcnt.to(torch.int64).reshape(BH, nb).sum(dim=1).cpu().tolist()
+    head_sp = sorted(1.0 - x / (nb * nb) for x in head_kept)
+    per_head = {"min": head_sp[0], "median": statistics.median(head_sp), "max": head_sp[-1]}
+    near = None
+    if 0.0 < path.thr < 1.0:
+        nt_bits = torch.empty(2, wl.B, wl.H, nb, sh.nw, dtype=torch.int32, device=dev)
+        nt_cnt = torch.empty(2, wl.B, wl.H, nb, dtype=torch.int32, device=dev)
+        m.nabla_build_mask_sweep(None, None, sh, (path.thr - 1e-6, path.thr + 1e-6), wl.window,
+                                 mask_bits=nt_bits, row_cnt=nt_cnt, q_pool=path.qp, k_pool=path.kp,
+                                 workspace=path.mask_ws)
+        c = nt_cnt.to(torch.int64).reshape(2, -1).sum(dim=1).tolist()
+        near = int(c[1] - c[0])
+        del nt_bits, nt_cnt
+
+    side = {}
+    if not args.no_side:
+        # forward throughput against sparsity: the same pooled map cut at several thresholds,
+        # up to the pages' operating range (80-92% sparsity) where the data reaches it
+        fvs = []
+        for thr_s in (0.5, 0.8, 0.9, 0.95, 0.99, 0.999):
+            b_s = torch.empty_like(path.bits)
+            c_s = torch.empty(wl.B, wl.H, nb, dtype=torch.int32, device=dev)
+            m.nabla_build_mask(None, None, sh, thr_s, wl.window, mask_bits=b_s, row_cnt=c_s,
+                               q_pool=path.qp, k_pool=path.kp, workspace=path.mask_ws)
+            kept_s = int(c_s.to(torch.int64).sum())
+            if path.natural:
+                call = lambda: m.nabla_attn_fwd(path.q, path.k, path.v, b_s, sh, o=path.o,  # noqa: E731
+                                                o_dtype=path.o_dtype, lse=path.lse,
+                                                workspace=path.fwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
+            else:
+                call = lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, b_s, sh, o=path.o,  # noqa: E731
+                                                o_dtype=path.o_dtype, lse=path.lse, workspace=path.fwd_ws)
+            ms_s = time_call(call, 3, warm=1)
+            tf = kept_s * fl_fwd / (ms_s * 1e-3) / 1e12
+            fvs.append({"thr": thr_s, "sparsity": 1.0 - kept_s / (BH * nb * nb), "kept_tiles": kept_s,
+                        "ms": ms_s, "tflops_kept": tf, "frac": tf / pk["bf16_tflops"]})
+            del b_s, c_s
+        path.check_status()
+        side["fwd_vs_sparsity"] = fvs
+        if not wl.backward:
+            # the training step (forward + backward) on the training-like workload, beside
+            # the headline inference step
+            twl = WORKLOADS["train_mid"]
+            tpath = Path(twl, dev)
+            for _ in range(3):
+                tpath.step()
+            torch.cuda.synchronize()
+            tpath.check_status()
+            tpath.ev = {}
+            for _ in range(10):
+                tpath.step(timing=True)
+            torch.cuda.synchronize()
+            tpath.check_status()
+            tk = tpath.kept_pairs()
+            t_bwd = statistics.mean(tpath.segment_ms("t_fwd", "t_bwd"))
+            t_fwd = statistics.mean(tpath.segment_ms("t_mask", "t_fwd"))
+            t_step = statistics.mean(tpath.segment_ms("t0", "t_bwd"))
+            fl_b = 10.0 * 64 * 64 * twl.D
+            btf = tk * fl_b / (t_bwd * 1e-3) / 1e12
+            side.update({
+                "train_workload": twl.name, "train_step_ms": t_step, "train_fwd_ms": t_fwd,
+                "train_kept_tiles": tk, "bwd_ms": t_bwd, "bwd_tflops_kept": btf,
+                "bwd_roofline": {"bound": "tensor", "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel "
+                                 "(+ preprocess)", "achieved": btf, "peak": pk["bf16_tflops"],
+                                 "unit": "TFLOP/s", "frac": btf / pk["bf16_tflops"],
+                                 "peak_kind": f"{pk_kind} burst bf16 dense",
+                                 "algorithmic_per_launch": f"{tk} kept 64x64 tiles x {int(fl_b)} FLOP"}})
+            del tpath
+            torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers --------------------------------
     hq, hk, hv = (t.cpu().pin_memory() for t in (path.q, path.k, path.v))
@@ -551,11 +673,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.T, wl.Hg, wl.W],
-                   "D": wl.D, "P": wl.P, "thr": path.thr, "sta": list(wl.window),
-                   "step": ("pool Q/K, mask, attn fwd on natural-order Q/K/V" if path.natural
-                            else "reorder+pool, mask, attn fwd, attn bwd"),
-                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"heads-replicated x{world}"},
+        "config": workload_config(wl, path.thr, world, path.natural),
         "fwd_ms": fwd_ms, "fwd_tflops_kept": fwd_tflops,
         "dense_fwd_ms": dense_ms, "dense_tflops": dense_tflops, "speedup_vs_dense": dense_ms / fwd_ms,
         "mask_ms": mask_ms, "mask_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
@@ -563,7 +681,8 @@ def main():
         "mask_ms_from_pools": mask_ms_fused, "mask_sweep_from_pools": sweep, "reorder_ms": reorder_ms,
         "reorder_gbs": reorder_bytes / (reorder_ms * 1e-3) / 1e9,
         "bwd_ms": bwd_ms, "bwd_tflops_kept": bwd_tflops,
-        "kept_tiles": kept, "sparsity": sparsity,
+        "kept_tiles": kept, "sparsity": sparsity, "sparsity_per_head": per_head,
+        "near_threshold_blocks": near,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
@@ -571,6 +690,9 @@ def main():
         "gpu_launches": path.launches_per_step() * args.steps,
         "clocks": clocks,
     }
+    for key, val in side.items():
+        if line.get(key) is None:
+            line[key] = val
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

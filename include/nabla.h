@@ -233,16 +233,25 @@ nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, nabla_d
  * exceeds 1 MiB are rejected with NABLA_ERR_UNSUPPORTED before anything is enqueued
  * (the 720p-like 40-head problem needs about 200 KB).  The first call on a device looks
  * up that array's device address (cudaGetSymbolAddress, with the device current); make
- * that first call before any stream capture.  The call allocates nothing.  All calls
- * share the one array, which keeps the last call's contents (each call clears what
- * must start at zero): calls that can overlap on the GPU (different streams, or several
- * host threads on one device) race on it and must be serialised by the caller.  The
- * device status word of the last call is not readable through this entry point.
+ * that first call before any stream capture.  A re-created context (cudaDeviceReset)
+ * is detected by its context id and the lookup is repeated on the next call.  The call
+ * allocates nothing.  All calls share the one array, which keeps the last call's
+ * contents (each call clears what must start at zero): calls that can overlap on the
+ * GPU (different streams, or several host threads on one device) race on it and must
+ * be serialised by the caller.  The device status word of the last call on the current
+ * device (a bounded wait that gave up leaves O incomplete) is read, and cleared, with
+ * nabla_attn_fwd_noalloc_status().
  * --------------------------------------------------------------------------------- */
 nabla_status nabla_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                                     nabla_dtype v_dtype, const uint32_t *mask_bits, nabla_shape s,
                                     float scale, void *o, nabla_dtype o_dtype, float *lse,
                                     nabla_layout layout, nabla_stream_t stream);
+
+/* Status of the last nabla_attn_fwd_noalloc call on the current device: waits for
+ * `stream`, then behaves as nabla_read_device_status on the fixed array (NABLA_OK, or
+ * NABLA_ERR_DEVICE_CHECK with the code in `code`, nullable; the word is then cleared).
+ * Allocates nothing.  Errors: CUDA. */
+nabla_status nabla_attn_fwd_noalloc_status(uint32_t *code, nabla_stream_t stream);
 
 /* Failure-path self-test (no counterpart in the pages).  Enqueues one warp that waits,
  * through the same bounded barrier wait as every kernel of the library, for a barrier

@@ -14,7 +14,7 @@ Notation follows the pages: Q, K, V; P = patch side (P x P spatial patch), N = P
 per block; thr = CDF threshold; M = M_nabla OR M_STA.  Tensors are [B, H, S, D] with
 S = T * Hg * W tokens; nb = S / N blocks.
 
-Readings taken where the pages are silent (all listed again in the design doc):
+Readings taken where the pages are silent (each restated at the function that uses it):
   * row-major patch order and row-major order inside a patch;
   * the pooled map is scaled by 1/sqrt(D) like token attention;
   * block j is kept iff the probability mass ranked strictly before it (ranking by

@@ -84,19 +84,52 @@ def check_lists(ridx, rcnt, gmask):
     assert np.array_equal(np.where(valid, ri, -1), idx)
 
 
-def bf16_half_ulp(x):
-    ax = np.maximum(np.abs(x), 1e-30)
-    return 0.5 * np.exp2(np.floor(np.log2(ax)) - 7)
+def bf16_round(x):
+    """x (float64) rounded to the nearest bfloat16, ties to even, returned as float64.
+
+    Done on the fp64 value directly (frexp, 8 significant bits, round half to even), so
+    there is no double rounding through fp32.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def bf16_ulp(y):
+    """Spacing of bfloat16 values at |y| (y itself a bf16 value); 0 maps to the smallest."""
+    ay = np.maximum(np.abs(y), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(ay)) - 7)
 
 
 def check_close(got, ref, what, storage_bf16=False):
-    """max-abs / mean-abs gates; bf16 storage adds half an ulp of the reference value."""
-    err = np.abs(got - ref)
-    slack = bf16_half_ulp(ref) if storage_bf16 else 0.0
-    max_gate = FWD_MAX_ABS + slack
-    assert np.all(err <= max_gate), f"{what}: max abs err {err.max():.3e} (worst excess {(err - max_gate).max():.3e})"
-    mean_gate = FWD_MEAN_ABS + (np.mean(slack) if storage_bf16 else 0.0)
-    assert err.mean() <= mean_gate, f"{what}: mean abs err {err.mean():.3e} > {mean_gate:.3e}"
+    """max-abs / mean-abs gates of the fp64 reference.
+
+    f32 outputs: |got - ref| <= FWD_MAX_ABS everywhere and mean <= FWD_MEAN_ABS.
+
+    bf16 outputs: the reference is rounded to bf16 first (the output format cannot hold
+    anything closer) and the same two gates apply to |got - bf16(ref)|, the mean gate
+    without any slack.  Where one bf16 step exceeds the max gate (|ref| >= 4, step
+    2^-5), a result that rounded to the neighbouring bf16 value (one step away) is a
+    storage effect, not an error of the kernel, and is accepted; nothing further is.
+    Returns (max, mean) of |got - bf16(ref)| (bf16) or |got - ref| (f32), and prints the
+    unrounded error beside it for bf16 outputs.
+    """
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if storage_bf16:
+        ref_r = bf16_round(ref)
+        err = np.abs(got - ref_r)
+        max_gate = np.maximum(FWD_MAX_ABS, bf16_ulp(ref_r))
+        raw = np.abs(got - ref)
+        print(f"{what}: vs bf16(ref) max {err.max():.3e} mean {err.mean():.3e}; "
+              f"vs ref max {raw.max():.3e} mean {raw.mean():.3e}; "
+              f"one-step bf16 flips above the max gate: {int((err > FWD_MAX_ABS).sum())}")
+    else:
+        err = np.abs(got - ref)
+        max_gate = FWD_MAX_ABS
+    assert np.all(err <= max_gate), \
+        f"{what}: max abs err {err.max():.3e} (worst excess {(err - max_gate).max():.3e})"
+    assert err.mean() <= FWD_MEAN_ABS, f"{what}: mean abs err {err.mean():.3e} > {FWD_MEAN_ABS:.3e}"
     return float(err.max()), float(err.mean())
 
 

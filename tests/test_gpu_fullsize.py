@@ -1,8 +1,9 @@
 """Parity at the benchmark's full sizes, in the launch configuration bench.py times.
 
-Masks: every head against the oracle (bit-exact outside the 1e-6 band).  Forward:
-sampled heads x sampled query blocks, computed row by row by the oracle on the GPU's
-mask.  Backward (training workload): two sampled heads in full.
+Masks: every head against the oracle (bit-exact outside the 1e-6 band).  Forward: every
+row of the head with the most kept tiles, plus six query blocks of each of four other
+distinct heads, computed by the oracle on the GPU's mask.  Backward (training workload):
+two sampled heads in full.
 """
 import math
 
@@ -66,21 +67,37 @@ def test_fullsize_mask_and_forward(name):
             mism += m1
             amb += a1
     print(f"{name}: sparsity {1 - gm.mean():.4f}, near-threshold blocks {amb}, differing {mism}")
-    # forward on sampled heads / query blocks (rows of whole blocks)
+    # Forward.  (1) Every query row of the head that keeps the most tiles: its tiles are
+    # the longest walks of the launch (hundreds of key blocks per tile on the 720p-like
+    # workload), which exercise long online-softmax runs and the rescaling of O.  (2) Six
+    # query blocks of each of four further distinct heads.
     rng = np.random.default_rng(7)
     bf16_out = path.o.dtype == torch.bfloat16
     scale = 1 / math.sqrt(wl.D)
-    heads = [(int(b), int(h)) for b, h in zip(rng.integers(0, wl.B, 4), rng.integers(0, wl.H, 4))]
     perm = oracle.fractal_permutation(wl.T, wl.Hg, wl.W, wl.P)
-    for b, h in heads:
+    kept_per_head = gm.reshape(wl.B * wl.H, -1).sum(axis=1)
+    heavy = int(np.argmax(kept_per_head))
+    others = [x for x in range(wl.B * wl.H) if x != heavy]
+    picks = [(heavy, None)] + [(int(x), rng.choice(wl.nb, size=6, replace=False))
+                               for x in rng.choice(others, size=min(4, len(others)), replace=False)]
+    for bh, blocks in picks:
+        b, h = divmod(bh, wl.H)
         q, k, v = (_head(t, b, h, wl, reorder=True) for t in (path.q, path.k, path.v))
-        blocks = rng.choice(wl.nb, size=6, replace=False)
-        rows = (blocks[:, None] * wl.N + np.arange(wl.N)[None, :]).reshape(-1)
-        O, L = oracle.block_sparse_attention_rows(q, k, v, gm[b, h], wl.N, scale, rows)
+        if blocks is None:
+            O, L = oracle.block_sparse_attention(q[None, None], k[None, None], v[None, None],
+                                                 gm[b:b + 1, h:h + 1], wl.N, scale)
+            O, L = O[0, 0], L[0, 0]
+            rows = np.arange(wl.S)
+            what = f"O {name} heaviest head {b},{h} ({int(kept_per_head[bh])} tiles), every row"
+        else:
+            rows = (blocks[:, None] * wl.N + np.arange(wl.N)[None, :]).reshape(-1)
+            O, L = oracle.block_sparse_attention_rows(q, k, v, gm[b, h], wl.N, scale, rows)
+            what = f"O {name} head {b},{h}"
         # outputs in natural order (the inference path) sit at the tokens' natural indices
         at = torch.from_numpy(perm[rows] if path.natural else rows).cuda()
         got = path.o[b, h, at].detach().cpu().double().numpy()
-        check_close(got, O, f"O {name} head {b},{h}", storage_bf16=bf16_out)
+        mx, mean = check_close(got, O, what, storage_bf16=bf16_out)
+        print(f"{what}: max err {mx:.2e} mean {mean:.2e}")
         lse = path.lse[b, h, at].cpu().double().numpy()
         check_lse(lse, L)
 
