@@ -110,7 +110,7 @@ def _sharded_worker(rank, world, port, wl_args, out):
     assert torch.equal(heads, q[:, rank * hpr:(rank + 1) * hpr])
     assert torch.equal(sharding.heads_to_seq(heads), x[0])
     o = sharding.sharded_nabla_attention(*x, wl.T, wl.Hg, wl.W, wl.thrs[0], wl.window,
-                                         compute=_oracle_heads)
+                                         compute=_oracle_heads, balance="contiguous")
     out.put((rank, o))
     dist.barrier()
     dist.destroy_process_group()
@@ -141,4 +141,75 @@ def test_sharded_attention_gloo_world2(wl_args):
     shape = Shape(wl.B, wl.H, wl.T, wl.Hg, wl.W, wl.D)
     ref = _oracle_heads(q, k, v, shape, wl.thrs[0], wl.window, 1 / math.sqrt(wl.D))
     got = torch.cat([res[0], res[1]], dim=2)
+    assert torch.equal(got, ref)
+
+
+# ---- head balance: units assigned to ranks by load (longest processing time first) ----------
+
+def test_lpt_assign_plan_and_bound():
+    from adaptive_block_sparse_b200.sharding import lpt_assign
+    # one heavy head and many light ones: the contiguous split would give 102 against 52
+    loads = [100, 1, 1, 1, 1, 50]
+    plan = lpt_assign(loads, 2)
+    assert plan == [[0], [1, 2, 3, 4, 5]]
+    rng = __import__("numpy").random.default_rng(3)
+    for n in (2, 3, 4, 8):
+        for _ in range(20):
+            loads = [int(x) for x in rng.integers(1, 1000, size=int(rng.integers(n, 50)))]
+            plan = lpt_assign(loads, n)
+            assert sorted(u for p in plan for u in p) == list(range(len(loads)))
+            span = max(sum(loads[u] for u in p) for p in plan)
+            lower = max(max(loads), sum(loads) / n)       # no split can do better than this
+            assert span <= 4.0 / 3.0 * lower + 1e-9
+
+
+def _lpt_worker(rank, world, port, wl_args, loads, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from adaptive_block_sparse_b200 import sharding
+    from synth import Workload, make_qkv
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    wl = Workload(**wl_args)
+    q, k, v = make_qkv(wl)
+    s = wl.S // world
+    mine = slice(rank * s, (rank + 1) * s)
+    x = [t[:, :, mine].contiguous() for t in (q, k, v)]
+    plan = sharding.lpt_assign(loads, world)
+    # the uneven exchanges alone: every token of this rank's units, and back
+    u = sharding.seq_to_units(x[0], plan)
+    assert torch.equal(u[0], q.reshape(wl.B * wl.H, wl.S, wl.D)[plan[rank]])
+    assert torch.equal(sharding.units_to_seq(u, plan, wl.B, wl.H), x[0])
+    o = sharding.sharded_nabla_attention(*x, wl.T, wl.Hg, wl.W, wl.thrs[0], wl.window,
+                                         compute=_oracle_heads, balance="lpt", loads=loads)
+    out.put((rank, o, len(plan[rank])))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_sharded_attention_lpt_gloo_world2():
+    """Deliberately skewed head loads: the heavy head gets a rank of its own, the light
+    ones share the other; the result equals the unsharded computation exactly."""
+    import math
+    from adaptive_block_sparse_b200 import Shape
+    from synth import Workload, make_qkv
+    wl_args = dict(name="sh_lpt", B=2, H=3, T=2, Hg=16, W=16, D=64, thrs=(0.7,), seed=1103)
+    loads = [900, 5, 7, 3, 400, 2]        # per (b, h): units 0 and 4 dominate
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_lpt_worker, args=(r, 2, port, wl_args, loads, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = {r: (o, nu) for r, o, nu in (out.get(timeout=300) for _ in procs)}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0][1] == 1 and res[1][1] == 5          # plan [[0], [1, 2, 3, 4, 5]]
+    wl = Workload(**wl_args)
+    q, k, v = make_qkv(wl)
+    shape = Shape(wl.B, wl.H, wl.T, wl.Hg, wl.W, wl.D)
+    ref = _oracle_heads(q, k, v, shape, wl.thrs[0], wl.window, 1 / math.sqrt(wl.D))
+    got = torch.cat([res[0][0], res[1][0]], dim=2)
     assert torch.equal(got, ref)
