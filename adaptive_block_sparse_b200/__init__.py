@@ -73,8 +73,8 @@ _sigs = {
                                       _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _sz, _vp]),
     "nabla_bwd_workspace_bytes": (_sz, [_Shape]),
     "nabla_attn_bwd": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp,
-                                      _vp, _vp, _vp, _Shape, ctypes.c_float, _vp, _vp, _vp, _vp,
-                                      _sz, _vp]),
+                                      _vp, _vp, _vp, _Shape, ctypes.c_float, _vp, _vp, _vp,
+                                      ctypes.c_int, _vp, _sz, _vp]),
     "nabla_read_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _vp]),
     "nabla_selftest_bounded_wait": (ctypes.c_int, [_vp, _sz, _vp]),
     "nabla_attn_fwd_noalloc": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _vp, _Shape,
@@ -165,15 +165,21 @@ def nabla_status_string(status: int) -> str:
     return load_library().nabla_status_string(status).decode()
 
 
+REORDER_FORWARD = 0      # natural -> reordered
+REORDER_INVERSE = 1      # reordered -> natural
+REORDER_KEEP = 2         # natural -> natural (dtype conversion, optional pools)
+
+
 def nabla_reorder(src, dst, shape: Shape, inverse=False, pool_out=None, stream=None):
     """Natural <-> reordered token order ([B,H,S,D]); optional fp64 block means.
 
     Forward: bf16 ``src`` into a bf16 or fp16 ``dst``.  Inverse: same dtype both sides.
-    Forward with ``dst=None`` and ``pool_out``: the block means only.
+    Forward with ``dst=None`` and ``pool_out``: the block means only.  ``inverse`` may
+    also be REORDER_KEEP: bf16 ``src`` into a bf16 or fp16 ``dst`` in the same order.
     """
     _check(load_library().nabla_reorder(_ptr(src), dtype_code(src), _ptr(dst),
                                         dtype_code(dst) if dst is not None else NABLA_BF16,
-                                        _ptr(pool_out), shape.c(), int(bool(inverse)),
+                                        _ptr(pool_out), shape.c(), int(inverse),
                                         _stream(stream)), "nabla_reorder")
     return dst
 
@@ -271,8 +277,10 @@ def nabla_attn_fwd(q, k, v, mask_bits, shape: Shape, scale=None, o=None,
 
 
 def nabla_attn_bwd(q, k, v, o, dout, lse, row_idx, row_cnt, col_idx, col_cnt, shape: Shape,
-                   scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """Block-sparse attention backward (mask constant).  Returns (dq, dk, dv), fp32."""
+                   scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None,
+                   layout=NABLA_LAYOUT_REORDERED):
+    """Block-sparse attention backward (mask constant).  Returns (dq, dk, dv), fp32.
+    ``layout``: token order of every tensor argument (reordered, or natural)."""
     if scale is None:
         scale = 1.0 / math.sqrt(shape.D)
     o_dtype = NABLA_F32 if o.dtype == torch.float32 else NABLA_BF16
@@ -284,7 +292,7 @@ def nabla_attn_bwd(q, k, v, o, dout, lse, row_idx, row_cnt, col_idx, col_cnt, sh
     _check(load_library().nabla_attn_bwd(_ptr(q), _ptr(k), _ptr(v), dtype_code(v), _ptr(o), o_dtype,
                                _ptr(dout), _ptr(lse),
                                _ptr(row_idx), _ptr(row_cnt), _ptr(col_idx), _ptr(col_cnt),
-                               shape.c(), float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                               shape.c(), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), int(layout),
                                _ptr(workspace), workspace.numel(), _stream(stream)),
            "nabla_attn_bwd")
     return dq, dk, dv

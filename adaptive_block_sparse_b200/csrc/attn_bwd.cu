@@ -55,6 +55,24 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
+// Reordered row -> natural token of the same head (NABLA_LAYOUT_NATURAL): block r / 64
+// is the 8 x 8 patch (frame, patch row, patch column) of the fractal order, token r % 64
+// the row-major position inside it.
+struct NatMap {
+  int on;
+  int HW, Wb, Hg, W;
+  long long S;
+  __device__ __forceinline__ long long token(long long bh, int blk, int r64) const {
+    const int tf = blk / HW, rr = blk - tf * HW, hb = rr / Wb, wb = rr - hb * Wb;
+    return bh * S + (static_cast<long long>(tf) * Hg + hb * 8 + (r64 >> 3)) * W + wb * 8 + (r64 & 7);
+  }
+  __device__ __forceinline__ long long token_of_row(long long row) const {
+    const long long bh = row / S;
+    const int r = static_cast<int>(row - bh * S);
+    return token(bh, r >> 6, r & 63);
+  }
+};
+
 // -------------------------------------------------------------------------------------
 // 1. preprocess: delta = rowsum(dO * O), lse2 = LSE * log2(e)
 // -------------------------------------------------------------------------------------
@@ -70,7 +88,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
     const __nv_bfloat16* __restrict__ k, const void* __restrict__ v, int v_f16,
     __half* __restrict__ q16, __half* __restrict__ k16, __half* __restrict__ v16,
     __half* __restrict__ do16, float* __restrict__ delta, float* __restrict__ lse2,
-    long long rows, uint32_t* status) {
+    long long rows, uint32_t* status, NatMap nat) {
   // D / 8 lanes per row, 8 contiguous elements (16 bytes of a 16-bit tensor) per lane.
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
@@ -78,7 +96,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
   const long long row = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kRowsPerWarp +
                         lane / kLanesPerRow;
   const bool active = row < rows;
+  // the outputs are written at the reordered row; with natural-order inputs the row's
+  // token is read from its natural index (the gather of the fractal flatten)
+  const long long src_row = nat.on && active ? nat.token_of_row(row) : row;
   const long long base = (active ? row : 0) * D + (lane % kLanesPerRow) * 8;
+  const long long sbase = (active ? src_row : 0) * D + (lane % kLanesPerRow) * 8;
   float acc = 0.f;
   bool range_ok = true;
   if (active) {
@@ -101,25 +123,27 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
       return make_uint4(w[0], w[1], w[2], w[3]);
     };
     float g[8], of[8], t[8];
-    widen(*reinterpret_cast<const uint4*>(dout + base), g);
+    widen(*reinterpret_cast<const uint4*>(dout + sbase), g);
     if (o_f32) {
-      const float4 o0 = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + base);
-      const float4 o1 = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + base + 4);
+      const float4 o0 = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + sbase);
+      const float4 o1 = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + sbase + 4);
       of[0] = o0.x; of[1] = o0.y; of[2] = o0.z; of[3] = o0.w;
       of[4] = o1.x; of[5] = o1.y; of[6] = o1.z; of[7] = o1.w;
     } else {
-      widen(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + base), of);
+      widen(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + sbase), of);
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc = fmaf(g[i], of[i], acc);
     *reinterpret_cast<uint4*>(do16 + base) = to_f16(g);
-    widen(*reinterpret_cast<const uint4*>(q + base), t);
+    widen(*reinterpret_cast<const uint4*>(q + sbase), t);
     *reinterpret_cast<uint4*>(q16 + base) = to_f16(t);
-    widen(*reinterpret_cast<const uint4*>(k + base), t);
+    widen(*reinterpret_cast<const uint4*>(k + sbase), t);
     *reinterpret_cast<uint4*>(k16 + base) = to_f16(t);
-    if (!v_f16) {   // an fp16 V is used as it is
-      widen(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(v) + base), t);
+    if (!v_f16) {
+      widen(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(v) + sbase), t);
       *reinterpret_cast<uint4*>(v16 + base) = to_f16(t);
+    } else if (nat.on) {   // an fp16 V in the natural order is gathered as it is
+      *reinterpret_cast<uint4*>(v16 + base) = *reinterpret_cast<const uint4*>(static_cast<const __half*>(v) + sbase);
     }
   }
 #pragma unroll
@@ -127,7 +151,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
   if (!__all_sync(0xffffffffu, range_ok) && lane == 0) record_status(status, kDevFp16Range);
   if (active && lane % kLanesPerRow == 0) {
     delta[row] = acc;
-    lse2[row] = lse[row] * kLog2e;
+    lse2[row] = lse[src_row] * kLog2e;
   }
 }
 
@@ -146,6 +170,7 @@ struct BwdParams {
   long long S;
   float scale_log2;
   float scale;
+  NatMap nat;                // outputs at natural token indices when nat.on
 };
 
 // Walks the ascending union of two sorted lists; returns -1 at the end.  f: bit0 = in
@@ -431,7 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue: dV and scale * dK (fp32), columns [64h, 64h + 64) of the row ----------
     const int blk = upper ? jab.y : jab.x;
     const bool valid = blk >= 0;
-    const long long tok = bh * prm.S + static_cast<long long>(valid ? blk : 0) * 64 + (row & 63);
+    const long long tok = prm.nat.on ? prm.nat.token(bh, valid ? blk : 0, row & 63)
+                                     : bh * prm.S + static_cast<long long>(valid ? blk : 0) * 64 + (row & 63);
     bool have = ok && it > 0;
     if (have) {
       have = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, prm.status, kDevTimeoutOBar));
@@ -662,7 +688,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool upper = row >= 64;
     const int blk = upper ? iab.y : iab.x;
     const bool valid = blk >= 0;
+    // tok: the row in the reordered order (lse2 and delta); otok: where dQ goes
     const long long tok = bh * prm.S + static_cast<long long>(valid ? blk : 0) * 64 + (row & 63);
+    const long long otok = prm.nat.on ? prm.nat.token(bh, valid ? blk : 0, row & 63) : tok;
     const float my_lse2 = valid ? prm.lse2[tok] : 0.f;
     const float my_delta = valid ? prm.delta[tok] : 0.f;
     const float sl2 = prm.scale_log2;
@@ -717,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 32; ++c) ov[c] = 0u;
       }
       if (valid) {
-        float4* dst = reinterpret_cast<float4*>(prm.out0 + tok * D + (D / 2) * h + c0);
+        float4* dst = reinterpret_cast<float4*>(prm.out0 + otok * D + (D / 2) * h + c0);
         const float mul = prm.scale;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -738,7 +766,15 @@ template <int D>
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, const void* o, int o_f32,
                        const void* dout, const float* lse, const int32_t* ridx, const int32_t* rcnt,
                        const int32_t* cidx, const int32_t* ccnt, const Dims& d, float scale,
-                       float* dq, float* dk, float* dv, void* ws, cudaStream_t st, bool* map_ok) {
+                       float* dq, float* dk, float* dv, void* ws, cudaStream_t st, bool* map_ok,
+                       bool natural) {
+  NatMap nat;
+  nat.on = natural ? 1 : 0;
+  nat.HW = d.Hb * d.Wb;
+  nat.Wb = d.Wb;
+  nat.Hg = d.Hg;
+  nat.W = d.W;
+  nat.S = d.S;
   const long long rows = static_cast<long long>(d.BH) * d.S;
   float* delta = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
   float* lse2 = delta + align_up(static_cast<size_t>(rows), 64);
@@ -757,11 +793,11 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
     e = build_schedule(rcnt, nullptr, d, sched + schedule_scratch_bytes(d), &order_rows, st, /*frame_pairs=*/true);
   if (e != cudaSuccess) return e;
   constexpr int kRowsPerCta = 8 * (256 / D);
-  if (v_f16) v16 = static_cast<__half*>(const_cast<void*>(v));   // used as it is
+  if (v_f16 && !natural) v16 = static_cast<__half*>(const_cast<void*>(v));   // used as it is
   bwd_preprocess_kernel<D><<<static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta), 256, 0, st>>>(
       o, o_f32, static_cast<const __nv_bfloat16*>(dout), lse, static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), v, v_f16, q16, k16, v16,
-      do16, delta, lse2, rows, status);
+      do16, delta, lse2, rows, status, nat);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   // per-panel maps for the resident 128-row operands (two 64-row blocks per panel), and
@@ -783,6 +819,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   p.S = d.S;
   p.scale_log2 = scale * kLog2e;
   p.scale = scale;
+  p.nat = nat;
   const unsigned grid = static_cast<unsigned>(d.BH) * static_cast<unsigned>((d.nb + 1) / 2);
   p.npairs = (d.nb + 1) / 2;
 
@@ -828,7 +865,7 @@ extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void*
                                        const int32_t* row_idx, const int32_t* row_cnt,
                                        const int32_t* col_idx, const int32_t* col_cnt,
                                        nabla_shape s, float scale, float* dq, float* dk, float* dv,
-                                       void* workspace, size_t workspace_bytes,
+                                       nabla_layout layout, void* workspace, size_t workspace_bytes,
                                        nabla_stream_t stream) {
   Dims d;
   nabla_status rc = check_shape(s, &d);
@@ -845,6 +882,7 @@ extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void*
   if (o_dtype != NABLA_BF16 && o_dtype != NABLA_F32) return NABLA_ERR_INVALID_ARG;
   if (v_dtype != NABLA_BF16 && v_dtype != NABLA_F16) return NABLA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
+  if (layout != NABLA_LAYOUT_REORDERED && layout != NABLA_LAYOUT_NATURAL) return NABLA_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < nabla_bwd_workspace_bytes(s) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255))
     return NABLA_ERR_WORKSPACE;
@@ -854,8 +892,10 @@ extern "C" nabla_status nabla_attn_bwd(const void* q, const void* k, const void*
   if (e != cudaSuccess) return cuda_status(e);
   bool map_ok = true;
   e = d.D == 64 ? launch_bwd<64>(q, k, v, v_dtype == NABLA_F16, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
-                                 col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok)
+                                 col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok,
+                                 layout == NABLA_LAYOUT_NATURAL)
                 : launch_bwd<128>(q, k, v, v_dtype == NABLA_F16, o, o_dtype == NABLA_F32, dout, lse, row_idx, row_cnt, col_idx,
-                                  col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok);
+                                  col_cnt, d, scale, dq, dk, dv, workspace, st, &map_ok,
+                                  layout == NABLA_LAYOUT_NATURAL);
   return cuda_status(e);
 }

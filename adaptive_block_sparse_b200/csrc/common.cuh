@@ -52,6 +52,7 @@ enum : uint32_t {
   kDevTimeoutMeta = 0x109,
   kDevTimeoutSelftest = 0x10A,   // nabla_selftest_bounded_wait: the expected outcome
   kDevSelftestUnexpected = 0x10B,
+  kDevSmemAlign = 0x10C,   // dynamic shared memory not 1024-byte aligned (launch refused work)
   kDevFp16Range = 0x201,   // backward: an input exceeds the fp16 range (|x| > 65504)
 };
 
@@ -135,6 +136,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)

@@ -153,6 +153,13 @@ cudaError_t go(const void* src, void* dst, double* pool, const Dims& d, cudaStre
 template <int D>
 cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims& d, int inverse,
                            int esz, bool to_f16, cudaStream_t st) {
+  if (inverse == 2) {   // natural order kept: the dtype conversion alone (+ the pools)
+    if (to_f16)
+      return pool ? go<D, 2, true, true, true, true, true>(src, dst, pool, d, st)
+                  : go<D, 2, true, true, true, false, true>(src, dst, nullptr, d, st);
+    return pool ? go<D, 2, true, true, true, true, false>(src, dst, pool, d, st)
+                : go<D, 2, true, true, true, false, false>(src, dst, nullptr, d, st);
+  }
   if (inverse) {
     return esz == 4 ? go<D, 4, false, true, true, false, false>(src, dst, nullptr, d, st)
                     : go<D, 2, false, true, true, false, false>(src, dst, nullptr, d, st);
@@ -184,21 +191,23 @@ extern "C" nabla_status nabla_reorder(const void* src, nabla_dtype src_dtype, vo
   Dims d;
   nabla_status rc = check_shape(s, &d);
   if (rc != NABLA_OK) return rc;
-  // dst may be NULL for the pool alone (forward direction, pool_out given)
+  // inverse: 0 natural -> reordered, 1 reordered -> natural, 2 natural -> natural (the
+  // conversion alone).  dst may be NULL for the pool alone (direction 0, pool_out given).
+  if (inverse < 0 || inverse > 2) return NABLA_ERR_INVALID_ARG;
   if (!src || (!dst && (inverse || !pool_out))) return NABLA_ERR_INVALID_ARG;
   if (!aligned16(src) || (dst && !aligned16(dst))) return NABLA_ERR_INVALID_ARG;
-  const bool dt_ok = inverse ? (src_dtype == dst_dtype &&
-                                (src_dtype == NABLA_BF16 || src_dtype == NABLA_F16 || src_dtype == NABLA_F32))
-                             : (src_dtype == NABLA_BF16 && (dst_dtype == NABLA_BF16 || dst_dtype == NABLA_F16));
+  const bool dt_ok = inverse == 1 ? (src_dtype == dst_dtype &&
+                                     (src_dtype == NABLA_BF16 || src_dtype == NABLA_F16 || src_dtype == NABLA_F32))
+                                  : (src_dtype == NABLA_BF16 && (dst_dtype == NABLA_BF16 || dst_dtype == NABLA_F16));
   if (!dt_ok) return NABLA_ERR_INVALID_ARG;
-  if (pool_out && (inverse || (reinterpret_cast<uintptr_t>(pool_out) & 7))) return NABLA_ERR_INVALID_ARG;
+  if (pool_out && (inverse == 1 || (reinterpret_cast<uintptr_t>(pool_out) & 7))) return NABLA_ERR_INVALID_ARG;
   const int esz = src_dtype == NABLA_F32 ? 4 : 2;
   const size_t bytes = static_cast<size_t>(d.BH) * d.S * d.D * esz;
   const char* a = static_cast<const char*>(src);
   const char* b = static_cast<const char*>(dst);
   if (b && a < b + bytes && b < a + bytes) return NABLA_ERR_INVALID_ARG;   // overlap
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool to_f16 = !inverse && dst_dtype == NABLA_F16;
+  const bool to_f16 = inverse != 1 && dst_dtype == NABLA_F16;
   cudaError_t e = d.D == 64 ? launch_reorder<64>(src, dst, pool_out, d, inverse, esz, to_f16, st)
                             : launch_reorder<128>(src, dst, pool_out, d, inverse, esz, to_f16, st);
   return cuda_status(e);

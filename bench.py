@@ -184,23 +184,31 @@ def sum_over_ranks(x, world, dev):
 class Path:
     """Buffers and the step of the hot path for one workload on one GPU."""
 
-    def __init__(self, wl, dev):
+    def __init__(self, wl, dev, units=None):
+        """``units``: optional list of flat (b*H + h) heads of ``wl`` to keep (the rank's
+        share of a strong-scaling run); they form a problem of B = 1, H = len(units)."""
+        import dataclasses
         import adaptive_block_sparse_b200 as m
         self.m = m
+        full_wl = wl
+        self.q, self.k, self.v = make_qkv(wl, device=dev)          # natural order
+        if units is not None:
+            pick = torch.tensor(units, dtype=torch.long, device=dev)
+            self.q, self.k, self.v = (t.reshape(wl.B * wl.H, wl.S, wl.D)[pick][None].contiguous()
+                                      for t in (self.q, self.k, self.v))
+            wl = dataclasses.replace(wl, B=1, H=len(units))
         self.wl = wl
         self.dev = dev
         self.shape = m.Shape(wl.B, wl.H, wl.T, wl.Hg, wl.W, wl.D, wl.P)
         sh = self.shape
         self.thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
-        self.q, self.k, self.v = make_qkv(wl, device=dev)          # natural order
-        # Inference (forward only): the forward reads Q, K, V in their natural order and
-        # writes O in it; only the pooled means are computed beforehand.  Training: the
-        # tensors are reordered once (fp16 V for the P V products) and the backward reads
-        # the reordered copies.
-        self.natural = not wl.backward
-        if not self.natural:
-            self.qf, self.kf = (torch.empty_like(self.q) for _ in range(2))
-            self.vf = torch.empty(self.q.shape, dtype=torch.float16, device=dev)
+        # Both steps read Q, K, V in their natural order (no reordered copy): only the
+        # pooled means are computed beforehand.  Training also converts V to fp16 in place
+        # order (the P V products and the backward take fp16 P and V), and the forward
+        # writes f32 O for the backward.
+        self.natural = True
+        if wl.backward:
+            self.vh = torch.empty(self.q.shape, dtype=torch.float16, device=dev)
         self.qp = torch.empty(wl.B, wl.H, sh.nb, wl.D, dtype=torch.float64, device=dev)
         self.kp = torch.empty_like(self.qp)
         # the forward reads the bitmask only; the lists serve the backward
@@ -213,7 +221,9 @@ class Path:
                              dtype=torch.float32 if wl.backward else torch.bfloat16)
         self.lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=dev)
         if wl.backward:
-            self.do = make_dout(wl, device=dev)
+            self.do = make_dout(full_wl, device=dev)
+            if units is not None:
+                self.do = self.do.reshape(full_wl.B * full_wl.H, wl.S, wl.D)[pick][None].contiguous()
             self.dq, self.dk, self.dv = (torch.empty(self.q.shape, dtype=torch.float32, device=dev)
                                          for _ in range(3))
             self.bwd_ws = torch.zeros(m.nabla_bwd_workspace_bytes(sh), dtype=torch.uint8, device=dev)
@@ -223,11 +233,11 @@ class Path:
         """Kernels of this library launched by one step (memsets not counted).
 
         Inference: pool Q, pool K; mask (split, logits, select, fp64 rescue); forward
-        (schedule: per-head sort + head placement; attention).  Training: reorder Q, K,
-        V; the mask as above + column lists; forward; backward (2 schedules of 2
+        (schedule: per-head sort + head placement; attention).  Training: pool Q, pool K,
+        V to fp16; the mask as above + column lists; forward; backward (2 schedules of 2
         launches, preprocess, dK/dV, dQ).
         """
-        if self.natural:
+        if not self.wl.backward:
             return 2 + 4 + 3
         return 3 + 4 + 1 + 3 + 7
 
@@ -240,31 +250,24 @@ class Path:
     def step(self, timing=False):
         m, sh, wl = self.m, self.shape, self.wl
         self._mark("t0", timing)
-        if self.natural:
-            m.nabla_reorder(self.q, None, sh, pool_out=self.qp)
-            m.nabla_reorder(self.k, None, sh, pool_out=self.kp)
-        else:
-            m.nabla_reorder(self.q, self.qf, sh, pool_out=self.qp)
-            m.nabla_reorder(self.k, self.kf, sh, pool_out=self.kp)
-            m.nabla_reorder(self.v, self.vf, sh)
+        m.nabla_reorder(self.q, None, sh, pool_out=self.qp)
+        m.nabla_reorder(self.k, None, sh, pool_out=self.kp)
+        if wl.backward:
+            m.nabla_reorder(self.v, self.vh, sh, inverse=m.REORDER_KEEP)
         self._mark("t_reorder", timing)
         m.nabla_build_mask(None, None, sh, self.thr, wl.window, mask_bits=self.bits,
                            row_idx=self.ridx, row_cnt=self.rcnt, col_idx=self.cidx,
                            col_cnt=self.ccnt, q_pool=self.qp, k_pool=self.kp,
                            workspace=self.mask_ws)
         self._mark("t_mask", timing)
-        if self.natural:
-            m.nabla_attn_fwd(self.q, self.k, self.v, self.bits, sh, o=self.o,
-                             o_dtype=self.o_dtype, lse=self.lse, workspace=self.fwd_ws,
-                             layout=m.NABLA_LAYOUT_NATURAL)
-        else:
-            m.nabla_attn_fwd(self.qf, self.kf, self.vf, self.bits, sh, o=self.o,
-                             o_dtype=self.o_dtype, lse=self.lse, workspace=self.fwd_ws)
+        v = self.vh if wl.backward else self.v
+        m.nabla_attn_fwd(self.q, self.k, v, self.bits, sh, o=self.o, o_dtype=self.o_dtype,
+                         lse=self.lse, workspace=self.fwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
         self._mark("t_fwd", timing)
         if wl.backward:
-            m.nabla_attn_bwd(self.qf, self.kf, self.vf, self.o, self.do, self.lse, self.ridx,
+            m.nabla_attn_bwd(self.q, self.k, self.vh, self.o, self.do, self.lse, self.ridx,
                              self.rcnt, self.cidx, self.ccnt, sh, dq=self.dq, dk=self.dk,
-                             dv=self.dv, workspace=self.bwd_ws)
+                             dv=self.dv, workspace=self.bwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
             self._mark("t_bwd", timing)
 
     def segment_ms(self, a, b):
@@ -278,6 +281,25 @@ class Path:
             code = self.m.nabla_read_device_status(ws)
             if code:
                 raise RuntimeError(f"device status 0x{code:x}")
+
+
+def head_loads(wl, dev):
+    """Kept tiles of every (b, h) of a workload (pools + mask on the GPU), for the
+    strong-scaling split; every rank computes the same numbers."""
+    import adaptive_block_sparse_b200 as m
+    sh = m.Shape(wl.B, wl.H, wl.T, wl.Hg, wl.W, wl.D, wl.P)
+    q, k, _ = make_qkv(wl, device=dev)
+    qp = torch.empty(wl.B, wl.H, sh.nb, wl.D, dtype=torch.float64, device=dev)
+    kp = torch.empty_like(qp)
+    m.nabla_reorder(q, None, sh, pool_out=qp)
+    m.nabla_reorder(k, None, sh, pool_out=kp)
+    cnt = torch.empty(wl.B, wl.H, sh.nb, dtype=torch.int32, device=dev)
+    thr = wl.thrs[0] if len(wl.thrs) == 1 else 0.8
+    m.nabla_build_mask(None, None, sh, thr, wl.window, row_cnt=cnt, q_pool=qp, k_pool=kp)
+    loads = cnt.to(torch.int64).sum(dim=-1).reshape(-1).tolist()
+    del q, k, qp, kp, cnt
+    torch.cuda.empty_cache()
+    return loads
 
 
 def time_call(fn, iters, warm=2):
@@ -350,12 +372,13 @@ def oracle_sample(wl, q_nat, k_nat, v_nat, rcnt, budget_s=20.0):
 
 
 # --------------------------------------------------------------------------------------
-def workload_config(wl, thr, world, natural, scaling="weak"):
+def workload_config(wl, thr, world, scaling="weak"):
     """The ``config`` object of a bench line; both arms print the same one."""
     return {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.T, wl.Hg, wl.W],
             "D": wl.D, "P": wl.P, "thr": thr, "sta": list(wl.window),
-            "step": ("pool Q/K, mask, attn fwd on natural-order Q/K/V" if natural
-                     else "reorder+pool, mask, attn fwd, attn bwd"),
+            "step": ("pool Q/K, mask, attn fwd on natural-order Q/K/V" if not wl.backward
+                     else "pool Q/K, V to fp16, mask + lists, attn fwd and bwd on natural-order "
+                          "Q/K/V/dO"),
             "l2": "inputs larger than L2 (no flush)",
             "parallelism": (f"heads-replicated x{world}" if scaling == "weak"
                             else f"heads split over {world} ranks (LPT by kept tiles)")}
@@ -429,7 +452,7 @@ def run_reference(args, wl, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": workload_config(wl, thr, world, not wl.backward),
+            "config": workload_config(wl, thr, world),
             "kept_tiles": kept_all,
             "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": val,
                              "unit": "TFLOP/s"},
@@ -449,6 +472,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-side", action="store_true",
                     help="skip the side measurements (training step, forward vs sparsity)")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="weak: every rank runs the whole workload; strong: the workload's "
+                         "heads are split over the ranks (LPT by kept tiles)")
     args = ap.parse_args()
     wl = WORKLOADS[args.config]
     world, rank, local = init_dist() if args.impl == "ours" else (
@@ -459,7 +485,17 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     pk, pk_kind = peaks()
-    path = Path(wl, dev)
+    full_wl = wl
+    units = None
+    if args.scaling == "strong":
+        from adaptive_block_sparse_b200.sharding import lpt_assign
+        plan = lpt_assign(head_loads(wl, dev), world)
+        units = plan[rank]
+        args.no_side = True
+        if not units:
+            raise SystemExit(f"rank {rank} has no heads: {world} ranks for {wl.B * wl.H} heads")
+    path = Path(wl, dev, units=units)
+    wl = path.wl
 
     for _ in range(max(3, args.warmup)):
         path.step()
@@ -503,17 +539,12 @@ def main():
     m, sh = path.m, path.shape
     # the mask from bf16 Q and K (pooling included): natural order -> pool alone, then the
     # mask from the means; reordered order -> the mask call pools itself
-    if path.natural:
-        def mask_from_qk():
-            m.nabla_reorder(path.q, None, sh, pool_out=path.qp)
-            m.nabla_reorder(path.k, None, sh, pool_out=path.kp)
-            m.nabla_build_mask(None, None, sh, path.thr, wl.window, mask_bits=path.bits,
-                               row_idx=path.ridx, row_cnt=path.rcnt, q_pool=path.qp,
-                               k_pool=path.kp, workspace=path.mask_ws)
-    else:
-        def mask_from_qk():
-            m.nabla_build_mask(path.qf, path.kf, sh, path.thr, wl.window, mask_bits=path.bits,
-                               row_idx=path.ridx, row_cnt=path.rcnt, workspace=path.mask_ws)
+    def mask_from_qk():
+        m.nabla_reorder(path.q, None, sh, pool_out=path.qp)
+        m.nabla_reorder(path.k, None, sh, pool_out=path.kp)
+        m.nabla_build_mask(None, None, sh, path.thr, wl.window, mask_bits=path.bits,
+                           row_idx=path.ridx, row_cnt=path.rcnt, q_pool=path.qp,
+                           k_pool=path.kp, workspace=path.mask_ws)
     mask_ms = time_call(mask_from_qk, 5)
     mask_bytes = 2 * BH * wl.S * wl.D * 2 + BH * nb * sh.nw * 4
     # several thresholds from one pooled map (the pools of the step), against one mask
@@ -534,20 +565,17 @@ def main():
     sweep = {"thrs": list(sweep_thrs), "ms": sweep_ms, "ms_separate_calls": separate_ms,
              "sparsity": m.sparsity_curve(sw_cnt, sh)}
     del sw_bits, sw_cnt
-    # bytes of the pass before the mask: pooling of Q, K (natural path) or reorder of Q,
-    # K, V with pooling (training path)
-    reorder_bytes = (2 * BH * wl.S * wl.D * 2 if path.natural else 3 * 2 * BH * wl.S * wl.D * 2) \
+    # bytes of the pass before the mask: pooling of Q, K (+ V read and written as fp16 on
+    # the training path)
+    reorder_bytes = 2 * BH * wl.S * wl.D * 2 + (2 * BH * wl.S * wl.D * 2 if wl.backward else 0) \
         + 2 * BH * nb * wl.D * 8
     # all-ones mask (padding bits are ignored by the kernels)
     dense_bits = torch.full((wl.B, wl.H, nb, sh.nw), -1, dtype=torch.int32, device=dev)
     dense_iters = 2 if nb > 1000 else 5
-    if path.natural:
-        dense_call = lambda: m.nabla_attn_fwd(path.q, path.k, path.v, dense_bits, sh, o=path.o,
-                                              o_dtype=path.o_dtype, lse=path.lse,
-                                              workspace=path.fwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
-    else:
-        dense_call = lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, dense_bits, sh, o=path.o,
-                                              o_dtype=path.o_dtype, lse=path.lse, workspace=path.fwd_ws)
+    v_fwd = path.vh if wl.backward else path.v
+    dense_call = lambda: m.nabla_attn_fwd(path.q, path.k, v_fwd, dense_bits, sh, o=path.o,  # noqa: E731
+                                          o_dtype=path.o_dtype, lse=path.lse,
+                                          workspace=path.fwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
     dense_ms = time_call(dense_call, dense_iters, warm=1)
     dense_tflops = BH * nb * nb * fl_fwd / (dense_ms * 1e-3) / 1e12
     path.check_status()
@@ -581,13 +609,9 @@ def main():
             m.nabla_build_mask(None, None, sh, thr_s, wl.window, mask_bits=b_s, row_cnt=c_s,
                                q_pool=path.qp, k_pool=path.kp, workspace=path.mask_ws)
             kept_s = int(c_s.to(torch.int64).sum())
-            if path.natural:
-                call = lambda: m.nabla_attn_fwd(path.q, path.k, path.v, b_s, sh, o=path.o,  # noqa: E731
-                                                o_dtype=path.o_dtype, lse=path.lse,
-                                                workspace=path.fwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
-            else:
-                call = lambda: m.nabla_attn_fwd(path.qf, path.kf, path.vf, b_s, sh, o=path.o,  # noqa: E731
-                                                o_dtype=path.o_dtype, lse=path.lse, workspace=path.fwd_ws)
+            call = lambda: m.nabla_attn_fwd(path.q, path.k, v_fwd, b_s, sh, o=path.o,  # noqa: E731
+                                            o_dtype=path.o_dtype, lse=path.lse,
+                                            workspace=path.fwd_ws, layout=m.NABLA_LAYOUT_NATURAL)
             ms_s = time_call(call, 3, warm=1)
             tf = kept_s * fl_fwd / (ms_s * 1e-3) / 1e12
             fvs.append({"thr": thr_s, "sparsity": 1.0 - kept_s / (BH * nb * nb), "kept_tiles": kept_s,
@@ -671,9 +695,9 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": workload_config(wl, path.thr, world, path.natural),
+        "config": workload_config(full_wl, path.thr, world, args.scaling),
         "fwd_ms": fwd_ms, "fwd_tflops_kept": fwd_tflops,
         "dense_fwd_ms": dense_ms, "dense_tflops": dense_tflops, "speedup_vs_dense": dense_ms / fwd_ms,
         "mask_ms": mask_ms, "mask_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,

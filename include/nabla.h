@@ -80,12 +80,16 @@ const char *nabla_status_string(nabla_status s);
  *   NABLA_BF16; dst_dtype NABLA_BF16 (copy) or NABLA_F16 (converted on the way, for the
  *   V operand of the attention kernels; exact for 2^-14 <= |x| <= 65504, larger
  *   magnitudes become +-inf).
- * inverse != 0: dst[b,h,n(r),:] = src[b,h,r,:] (reordered -> natural), src_dtype ==
+ * inverse == 1: dst[b,h,n(r),:] = src[b,h,r,:] (reordered -> natural), src_dtype ==
  *   dst_dtype in {NABLA_BF16, NABLA_F16, NABLA_F32} (e.g. to restore an output O).
+ * inverse == 2: dst[b,h,n,:] = src[b,h,n,:] converted (natural order kept), src_dtype
+ *   NABLA_BF16, dst_dtype NABLA_BF16 or NABLA_F16: the fp16 V of the natural-layout
+ *   training path (see nabla_attn_bwd), in one pass, optionally with pool_out.
+ * Any other value of inverse: INVALID_ARG.
  * src, dst: [B,H,S,D] of those dtypes; must not overlap.  With inverse == 0 and pool_out
  *   given, dst may be NULL: only the block means are computed, src is read once and
  *   nothing is reordered (the natural-layout forward then reads src directly).
- * pool_out (nullable, only with inverse == 0): fp64 [B,H,nb,D], the mean of each
+ * pool_out (nullable, with inverse == 0 or 2): fp64 [B,H,nb,D], the mean of each
  *   block's N reordered token vectors (sum in token order in fp64, then / N), i.e.
  *   the pooled Q or K of [ZH-TS] "downsampling", ready for nabla_build_mask.
  * Errors: INVALID_ARG (nulls, overlap, shape), UNSUPPORTED (D, P), CUDA (launch).
@@ -209,6 +213,11 @@ nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v, nabla_d
  * device status word reports it (0x201).
  * row_* and col_* lists from nabla_build_mask / nabla_mask_lists.
  * dq, dk, dv : out f32 [B,H,S,D] (fully overwritten; deterministic, no atomics).
+ * layout     : token order of q, k, v, o, dout, lse, dq, dk and dv: NABLA_LAYOUT_REORDERED,
+ *              or NABLA_LAYOUT_NATURAL (the latent's natural order, as the natural-layout
+ *              forward reads and writes them; the fractal flatten of [ZH-TS] "token
+ *              reordering" is done by the backward's own gather into its fp16 copies, and
+ *              the gradients are written at the tokens' natural indices).
  * workspace  : >= nabla_bwd_workspace_bytes(s) bytes.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  * --------------------------------------------------------------------------------- */
@@ -218,8 +227,8 @@ nabla_status nabla_attn_bwd(const void *q, const void *k, const void *v, nabla_d
                             nabla_dtype o_dtype, const void *dout, const float *lse,
                             const int32_t *row_idx, const int32_t *row_cnt,
                             const int32_t *col_idx, const int32_t *col_cnt, nabla_shape s,
-                            float scale, float *dq, float *dk, float *dv, void *workspace,
-                            size_t workspace_bytes, nabla_stream_t stream);
+                            float scale, float *dq, float *dk, float *dv, nabla_layout layout,
+                            void *workspace, size_t workspace_bytes, nabla_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Allocation-free forward (no counterpart in the NABLA pages; a library convenience).

@@ -78,6 +78,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert ro(sd=F16) == INV                                              # forward needs bf16 source
     assert ro(dd=F32) == INV                                              # no f32 forward output
     assert ro(sd=F32, dd=BF, inv=1) == INV                                # inverse keeps the dtype
+    assert ro(inv=3) == INV                                               # unknown direction
+    assert ro(inv=-1) == INV
+    assert ro(inv=2, dd=F32) == INV                                       # keep-order: bf16 or fp16 out
+    assert ro(inv=2, dst=None, pool=A) == INV                             # keep-order needs dst
     win = nb._Window(0, 0, 0)
     ws_need = lib.nabla_mask_workspace_bytes(good)
     assert ws_need > 256
@@ -124,6 +128,24 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert fwd(vdt=1) == INV
     assert fwd(wsb=fws - 1) == WS
     assert fwd(layout=2) == INV                                            # unknown layout
+    bws = lib.nabla_bwd_workspace_bytes(good)
+    assert bws > 256
+
+    def bwd(q=A, lse=A, vdt=0, odt=0, cidx=A, scale=0.125, dq=Bp, layout=0, ws=Bp, wsb=bws):
+        return lib.nabla_attn_bwd(q, A, A, vdt, A, odt, A, lse, A, A, cidx, A, good, scale, dq, Bp,
+                                  Bp, layout, ws, wsb, st)
+    assert bwd(q=None) == INV
+    assert bwd(q=mis) == INV
+    assert bwd(lse=None) == INV
+    assert bwd(cidx=None) == INV
+    assert bwd(cidx=ctypes.c_void_p(0x10002)) == INV                      # lists need 4-byte alignment
+    assert bwd(vdt=1) == INV                                              # V is bf16 or fp16
+    assert bwd(odt=2) == INV                                              # O is bf16 or f32
+    assert bwd(scale=float("inf")) == INV
+    assert bwd(dq=None) == INV
+    assert bwd(layout=2) == INV                                           # unknown layout
+    assert bwd(wsb=bws - 1) == WS
+    assert bwd(ws=ctypes.c_void_p(0x20000010)) == WS                      # misaligned workspace
     assert lib.nabla_fwd_workspace_bytes(_shape(nb, D=96)) == 0
     assert lib.nabla_status_string(3) == b"NABLA_ERR_WORKSPACE"
     assert lib.nabla_selftest_bounded_wait(None, 256, st) == WS

@@ -103,15 +103,18 @@ def test_fullsize_mask_and_forward(name):
 
 
 def test_fullsize_backward():
+    """The training step as bench.py times it: natural-order Q, K, V (fp16 V), dO; the
+    gradients land at natural indices.  Two heads in full against the oracle gradients of
+    the reordered tensors, inverse-reordered."""
     wl, path = _run("train_mid")
     gm = bits_to_mask(path.bits, wl.nb)
     check_lists(path.cidx, path.ccnt, np.swapaxes(gm, -1, -2))
     scale = 1 / math.sqrt(wl.D)
     for b, h in ((0, 3), (1, 17)):
-        q, k, do = (_head(t, b, h, wl) for t in (path.qf, path.kf, path.do))
-        v = _head(path.v, b, h, wl, reorder=True)
+        q, k, v, do = (_head(t, b, h, wl, reorder=True) for t in (path.q, path.k, path.vh, path.do))
         ref = oracle.block_sparse_attention_bwd(q[None, None], k[None, None], v[None, None],
                                                 do[None, None], gm[b:b + 1, h:h + 1], wl.N, scale)
         for got, r, what in zip((path.dq, path.dk, path.dv), ref, ("dQ", "dK", "dV")):
-            mx, mean = check_close(to64(got[b, h]), r[0, 0], f"{what} train_mid head {b},{h}")
+            r_nat = oracle.inverse_reorder(r[0, 0][None, None], wl.T, wl.Hg, wl.W, wl.P)[0, 0]
+            mx, mean = check_close(to64(got[b, h]), r_nat, f"{what} train_mid head {b},{h}")
             print(f"train_mid {what} head {b},{h}: max err {mx:.2e} mean {mean:.2e}")

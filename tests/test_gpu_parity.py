@@ -350,3 +350,46 @@ def test_bwd_parity(data, name, thr, window):
     for got, ref, what in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
         mx, mean = check_close(to64(got), ref, f"{what} {name}")
         print(f"{name} {what}: max|ref| {np.abs(ref).max():.2f} max err {mx:.2e} mean err {mean:.2e}")
+
+
+@pytest.mark.parametrize("name,thr,window", [("small", 0.8, (3, 3, 3)), ("odd", 0.8, (1, 1, 1)),
+                                             ("odd64", 0.6, (0, 0, 0))])
+def test_bwd_natural_layout(data, name, thr, window):
+    """The training step without a materialised reorder: pools of the natural-order Q and K,
+    the mask from them, the natural-layout forward (f32 O and LSE at natural indices), and
+    the backward on natural-order Q, K, V, O, dO, LSE writing dQ, dK, dV at natural indices.
+    V is passed as fp16 (a cast in the natural order, exact for these inputs): the backward
+    takes Dr = rowsum(dO * O) from the forward's O, and with bf16 V (probabilities rounded
+    to 8 bits) O carries enough error to push dQ past the 2e-2 gate (measured 2.7e-2).
+    Against the oracle gradients of the reordered tensors, inverse-reordered."""
+    m = nbl()
+    wl = _wl(name)
+    shape = shape_of(wl)
+    q, k, v = data(wl)
+    va = v.to(torch.float16)
+    qp = torch.empty(wl.B, wl.H, wl.nb, wl.D, dtype=torch.float64, device=DEV)
+    kp = torch.empty_like(qp)
+    m.nabla_reorder(q, None, shape, pool_out=qp)
+    m.nabla_reorder(k, None, shape, pool_out=kp)
+    bits, ridx, rcnt, cidx, ccnt = gpu_mask(None, None, shape, thr, window, q_pool=qp, k_pool=kp)
+    nat = m.NABLA_LAYOUT_NATURAL
+    lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
+    fws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    o, _ = m.nabla_attn_fwd(q, k, va, bits, shape, o_dtype=m.NABLA_F32, lse=lse, workspace=fws,
+                            layout=nat)
+    g = torch.Generator(device=DEV).manual_seed(4242)
+    do = torch.randn(q.shape, generator=g, device=DEV, dtype=torch.float32).to(torch.bfloat16)
+    bws = torch.zeros(m.nabla_bwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    dq, dk, dv = m.nabla_attn_bwd(q, k, va, o, do, lse, ridx, rcnt, cidx, ccnt, shape, workspace=bws,
+                                  layout=nat)
+    torch.cuda.synchronize()
+    assert m.nabla_read_device_status(fws) == 0
+    assert m.nabla_read_device_status(bws) == 0
+    gm = bits_to_mask(bits, wl.nb)
+    T, Hg, W, P = wl.T, wl.Hg, wl.W, wl.P
+    rq, rk, rv = oracle.block_sparse_attention_bwd(
+        *(oracle.reorder(to64(x), T, Hg, W, P) for x in (q, k, v, do)), gm, wl.N, 1 / math.sqrt(wl.D))
+    for got, ref, what in ((dq, rq, "dQ"), (dk, rk, "dK"), (dv, rv, "dV")):
+        ref_nat = oracle.inverse_reorder(ref, T, Hg, W, P)
+        mx, mean = check_close(to64(got), ref_nat, f"natural {what} {name}")
+        print(f"natural {name} {what}: max|ref| {np.abs(ref).max():.2f} max err {mx:.2e} mean err {mean:.2e}")
