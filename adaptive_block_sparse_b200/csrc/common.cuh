@@ -52,7 +52,6 @@ enum : uint32_t {
   kDevTimeoutMeta = 0x109,
   kDevTimeoutSelftest = 0x10A,   // nabla_selftest_bounded_wait: the expected outcome
   kDevSelftestUnexpected = 0x10B,
-  kDevSmemAlign = 0x10C,   // dynamic shared memory not 1024-byte aligned (launch refused work)
   kDevFp16Range = 0x201,   // backward: an input exceeds the fp16 range (|x| > 65504)
 };
 
@@ -136,19 +135,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Non-blocking test: has the phase with the given parity completed?
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -478,43 +464,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe (relieves the special-function unit): Cody-Waite style range
-// reduction x = j + f, j = floor(x), f in [0, 1), then a degree-3 minimax polynomial for
-// 2^f (coefficients from a Remez fit of the relative error on [0, 1]; max relative error
-// 7.5e-5, far below the 2^-8 rounding of the bf16 probabilities it feeds), and j added to
-// the exponent field.  Valid for x <= 127; inputs below -126 are clamped (result ~1e-38).
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -126.0f);
-  const float j = floorf(x);
-  const float f = x - j;
-  float p = fmaf(0.07802452147006989f, f, 0.22606715559959412f);
-  p = fmaf(p, f, 0.6958335638046265f);
-  p = fmaf(p, f, 0.9999251961708069f);
-  return __int_as_float(__float_as_int(p) + (static_cast<int>(j) << 23));
-}
-
-// 2^x for a pair of values on the FMA and integer pipes (relieves the special-function
-// unit): x = j + f with j = x rounded to the nearest integer by the 1.5 * 2^23 shifter
-// (its low mantissa bits then hold j), f in [-0.5, 0.5]; 2^f from a degree-3 polynomial
-// (minimax fit of the relative error on [-0.5, 0.5], max relative error 7.5e-5, far below
-// the 2^-11 rounding of the fp16 probabilities it feeds); j is added to the exponent
-// field as (shifter bits << 23), the shifter's own bits falling off the top.  Inputs below
-// -126 are clamped (result ~1e-38).
-__device__ __forceinline__ float2 poly_exp2x2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 shifter = make_float2(12582912.0f, 12582912.0f);
-  const float2 t = __fadd2_rn(x, shifter);
-  const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
-  float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
-                        make_float2(0.2426111251115799f, 0.2426111251115799f));
-  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 #endif  // __CUDACC__

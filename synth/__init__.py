@@ -82,6 +82,10 @@ WORKLOADS = {
                            sigma=(1.0, 6.0), seed=1002),
     "train_mid": Workload("train_mid", B=2, H=24, T=11, Hg=32, W=56, D=128, thrs=(0.8,),
                           window=(3, 3, 3), sigma=(2.0, 2.0), backward=True, seed=1004),
+    # heads 0-11 of batch 0 of the training-like workload (identical draws), a smaller
+    # case for profiler captures of the backward
+    "train_mid_h12": Workload("train_mid_h12", B=1, H=12, T=11, Hg=32, W=56, D=128, thrs=(0.8,),
+                              window=(3, 3, 3), sigma=(2.0, 2.0), backward=True, seed=1004),
 }
 
 
