@@ -64,7 +64,8 @@ _sigs = {
     "nabla_reorder": (ctypes.c_int, [_vp, ctypes.c_int, _vp, ctypes.c_int, _vp, _Shape, _i32, _vp]),
     "nabla_mask_workspace_bytes": (_sz, [_Shape]),
     "nabla_build_mask": (ctypes.c_int, [_vp, _vp, _vp, _vp, _Shape, ctypes.c_double, _Window,
-                                        ctypes.c_double, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+                                        ctypes.c_double, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, _vp,
+                                        _sz, _vp]),
     "nabla_mask_lists": (ctypes.c_int, [_vp, _Shape, _vp, _vp, _vp, _vp, _vp]),
     "nabla_build_mask_sweep": (ctypes.c_int, [_vp, _vp, _vp, _vp, _Shape, _vp, ctypes.c_int, _Window,
                                               ctypes.c_double, _vp, _vp, _vp, _sz, _vp]),
@@ -198,8 +199,10 @@ def nabla_bwd_workspace_bytes(shape: Shape) -> int:
 
 def nabla_build_mask(q, k, shape: Shape, thr: float, window=(0, 0, 0), scale=None,
                      mask_bits=None, row_idx=None, row_cnt=None, col_idx=None, col_cnt=None,
-                     q_pool=None, k_pool=None, workspace=None, stream=None):
-    """NABLA block mask.  Returns (mask_bits, row_idx, row_cnt, col_idx, col_cnt)."""
+                     q_pool=None, k_pool=None, workspace=None, stream=None,
+                     layout=NABLA_LAYOUT_REORDERED):
+    """NABLA block mask.  Returns (mask_bits, row_idx, row_cnt, col_idx, col_cnt).
+    ``layout``: token order of ``q`` and ``k`` when they are read (no pools given)."""
     dev = next(t.device for t in (q, q_pool, mask_bits, workspace) if t is not None)
     BH = shape.B * shape.H
     if mask_bits is None:
@@ -211,7 +214,7 @@ def nabla_build_mask(q, k, shape: Shape, thr: float, window=(0, 0, 0), scale=Non
     _check(load_library().nabla_build_mask(_ptr(q), _ptr(k), _ptr(q_pool), _ptr(k_pool), shape.c(),
                                  float(thr), _Window(*window), float(scale), _ptr(mask_bits),
                                  _ptr(row_idx), _ptr(row_cnt), _ptr(col_idx), _ptr(col_cnt),
-                                 _ptr(workspace), workspace.numel(), _stream(stream)),
+                                 int(layout), _ptr(workspace), workspace.numel(), _stream(stream)),
            "nabla_build_mask")
     del BH
     return mask_bits, row_idx, row_cnt, col_idx, col_cnt

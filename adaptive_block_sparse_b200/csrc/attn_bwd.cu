@@ -173,22 +173,46 @@ struct BwdParams {
   NatMap nat;                // outputs at natural token indices when nat.on
 };
 
-// Walks the ascending union of two sorted lists; returns -1 at the end.  f: bit0 = in
-// the first list, bit1 = in the second.
-struct UnionWalk {
+// Walks the ascending union of two sorted lists with a whole warp; every lane gets the
+// same result, -1 at the end.  f: bit0 = in the first list, bit1 = in the second.  The
+// lists are read 32 entries at a time (one coalesced load per list), the next 32 already
+// in flight, so a step costs a few shuffles instead of a dependent global load.
+struct WarpUnion {
   const int32_t* l0;
   const int32_t* l1;
-  int c0, c1, a, b;
-  __device__ int next(uint32_t* f) {
-    if (a < c0 && b < c1) {
-      const int ja = l0[a], jb = l1[b];
-      if (ja < jb) { *f = 1; ++a; return ja; }
-      if (jb < ja) { *f = 2; ++b; return jb; }
-      *f = 3; ++a; ++b; return ja;
+  int c0, c1, a, b, base0, base1;
+  int v0, v1, n0, n1;        // this lane's entry of the current and of the next chunk
+  __device__ static int load(const int32_t* l, int c, int pos) { return pos < c ? __ldg(l + pos) : 0x7FFFFFFF; }
+  __device__ void init(const int32_t* list0, int cnt0, const int32_t* list1, int cnt1, int lane) {
+    l0 = list0;
+    l1 = list1;
+    c0 = cnt0;
+    c1 = cnt1;
+    a = b = base0 = base1 = 0;
+    v0 = load(l0, c0, lane);
+    v1 = load(l1, c1, lane);
+    n0 = load(l0, c0, 32 + lane);
+    n1 = load(l1, c1, 32 + lane);
+  }
+  __device__ int next(uint32_t* f, int lane) {
+    if (a - base0 == 32) {          // warp-uniform
+      base0 += 32;
+      v0 = n0;
+      n0 = load(l0, c0, base0 + 32 + lane);
     }
-    if (a < c0) { *f = 1; return l0[a++]; }
-    if (b < c1) { *f = 2; return l1[b++]; }
-    return -1;
+    if (b - base1 == 32) {
+      base1 += 32;
+      v1 = n1;
+      n1 = load(l1, c1, base1 + 32 + lane);
+    }
+    const int ja = __shfl_sync(0xffffffffu, v0, a - base0);
+    const int jb = __shfl_sync(0xffffffffu, v1, b - base1);
+    const int xa = a < c0 ? ja : 0x7FFFFFFF;
+    const int xb = b < c1 ? jb : 0x7FFFFFFF;
+    if (xa == 0x7FFFFFFF && xb == 0x7FFFFFFF) return -1;
+    if (xa < xb) { *f = 1; ++a; return xa; }
+    if (xb < xa) { *f = 2; ++b; return xb; }
+    *f = 3; ++a; ++b; return xa;
   }
 };
 
@@ -283,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // the whole warp walks the lists; lane 0 waits on the ring and issues the copies
     if (lane == 0) {
       tma_prefetch_desc(&map_q64);
       tma_prefetch_desc(&map_do64);
@@ -299,26 +324,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(sV + pn * 16384, &map_v64, kv_full, pn * 64, ka);
         tma_load_2d(sV + pn * 16384 + 8192, &map_v64, kv_full, pn * 64, kb);
       }
-      UnionWalk wk;
-      wk.l0 = prm.list_idx + (bh * nb + jab.x) * static_cast<long long>(nb);
-      wk.l1 = prm.list_idx + (bh * nb + (jab.y >= 0 ? jab.y : jab.x)) * static_cast<long long>(nb);
-      wk.c0 = min(max(prm.list_cnt[bh * nb + jab.x], 0), nb);
-      wk.c1 = jab.y >= 0 ? min(max(prm.list_cnt[bh * nb + jab.y], 0), nb) : 0;
-      wk.a = wk.b = 0;
-      int it = 0;
-      bool ended = false;
-      while (true) {
-        uint32_t f = 0;
-        const int i = wk.next(&f);
-        const int s = it % L::kStages;
-        const int n = it / L::kStages;
-        if (n > 0 && !mbar_wait(&empty[s], (n - 1) & 1, prm.status, kDevTimeoutKvEmpty)) break;
-        if (i < 0 || i >= nb) {
+    }
+    WarpUnion wk;
+    wk.init(prm.list_idx + (bh * nb + jab.x) * static_cast<long long>(nb),
+            min(max(prm.list_cnt[bh * nb + jab.x], 0), nb),
+            prm.list_idx + (bh * nb + (jab.y >= 0 ? jab.y : jab.x)) * static_cast<long long>(nb),
+            jab.y >= 0 ? min(max(prm.list_cnt[bh * nb + jab.y], 0), nb) : 0, lane);
+    int it = 0;
+    bool ended = false;
+    while (true) {
+      uint32_t f = 0;
+      const int i = wk.next(&f, lane);
+      const int s = it % L::kStages;
+      const int n = it / L::kStages;
+      int ok = 1;
+      if (lane == 0 && n > 0) ok = mbar_wait(&empty[s], (n - 1) & 1, prm.status, kDevTimeoutKvEmpty) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (i < 0 || i >= nb) {
+        if (lane == 0) {
           meta[s] = kEnd;
           mbar_arrive(&full[s]);
-          ended = true;
-          break;
         }
+        ended = true;
+        break;
+      }
+      if (lane == 0) {
         meta[s] = static_cast<uint32_t>(i) | (f << 28);
         unsigned char* st = sStage + s * L::kStageStride;
         mbar_arrive_expect_tx(&full[s], 2 * C::kTileBytes + 512);
@@ -328,8 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(st + C::kTileBytes, &map_do64, &full[s], 0, static_cast<int>(qrow), 0);
         bulk_load(st + 2 * C::kTileBytes, prm.lse2 + qrow, 256, &full[s]);
         bulk_load(st + 2 * C::kTileBytes + 256, prm.delta + qrow, 256, &full[s]);
-        ++it;
       }
+      ++it;
+    }
+    if (lane == 0) {
       // Copies still in flight: the last kStages iterations, except that placing the end
       // marker waited for the oldest of them to be consumed (its stage was reused), and a
       // parity wait on that stage would now look two phases back.
@@ -568,6 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // the whole warp walks the lists; lane 0 waits on the ring and issues the copies
     if (lane == 0) {
       tma_prefetch_desc(&map_q64);
       tma_prefetch_desc(&map_do64);
@@ -583,26 +616,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(sDO + pn * 16384, &map_do64, q_full, pn * 64, qa);
         tma_load_2d(sDO + pn * 16384 + 8192, &map_do64, q_full, pn * 64, qb);
       }
-      UnionWalk wk;
-      wk.l0 = prm.list_idx + (bh * nb + iab.x) * static_cast<long long>(nb);
-      wk.l1 = prm.list_idx + (bh * nb + (iab.y >= 0 ? iab.y : iab.x)) * static_cast<long long>(nb);
-      wk.c0 = min(max(prm.list_cnt[bh * nb + iab.x], 0), nb);
-      wk.c1 = iab.y >= 0 ? min(max(prm.list_cnt[bh * nb + iab.y], 0), nb) : 0;
-      wk.a = wk.b = 0;
-      int it = 0;
-      bool ended = false;
-      while (true) {
-        uint32_t f = 0;
-        const int j = wk.next(&f);
-        const int s = it % L::kStages;
-        const int n = it / L::kStages;
-        if (n > 0 && !mbar_wait(&empty[s], (n - 1) & 1, prm.status, kDevTimeoutKvEmpty)) break;
-        if (j < 0 || j >= nb) {
+    }
+    WarpUnion wk;
+    wk.init(prm.list_idx + (bh * nb + iab.x) * static_cast<long long>(nb),
+            min(max(prm.list_cnt[bh * nb + iab.x], 0), nb),
+            prm.list_idx + (bh * nb + (iab.y >= 0 ? iab.y : iab.x)) * static_cast<long long>(nb),
+            iab.y >= 0 ? min(max(prm.list_cnt[bh * nb + iab.y], 0), nb) : 0, lane);
+    int it = 0;
+    bool ended = false;
+    while (true) {
+      uint32_t f = 0;
+      const int j = wk.next(&f, lane);
+      const int s = it % L::kStages;
+      const int n = it / L::kStages;
+      int ok = 1;
+      if (lane == 0 && n > 0) ok = mbar_wait(&empty[s], (n - 1) & 1, prm.status, kDevTimeoutKvEmpty) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (j < 0 || j >= nb) {
+        if (lane == 0) {
           meta[s] = kEnd;
           mbar_arrive(&full[s]);
-          ended = true;
-          break;
         }
+        ended = true;
+        break;
+      }
+      if (lane == 0) {
         meta[s] = static_cast<uint32_t>(j) | (f << 28);
         unsigned char* st = sStage + s * L::kStageBytes;
         mbar_arrive_expect_tx(&full[s], 2 * C::kTileBytes);
@@ -610,8 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one copy per operand: all D columns of the 64 rows (panels 8 KB apart)
         tma_load_3d(st, &map_k64, &full[s], 0, krow, 0);
         tma_load_3d(st + C::kTileBytes, &map_v64, &full[s], 0, krow, 0);
-        ++it;
       }
+      ++it;
+    }
+    if (lane == 0) {
       // Copies still in flight (as in the dK/dV pass).
       const int keep = ended ? L::kStages - 1 : L::kStages;
       const int first = it > keep ? it - keep : 0;

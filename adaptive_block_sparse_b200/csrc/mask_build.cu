@@ -27,7 +27,10 @@
 
 namespace nabla {
 
-cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st);
+cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st, bool natural);
+cudaError_t mask_fast_prepare_tokens(const void* q, const void* k, bool natural, double* qp_out,
+                                     double* kp_out, const Dims& d, double scale, void* scratch,
+                                     uint32_t* status, cudaStream_t st);
 size_t mask_fast_scratch_bytes(const Dims& d);
 bool mask_fast_supported(const Dims& d);
 cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d, double scale,
@@ -504,11 +507,13 @@ extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const dou
                                          const double* k_pool, nabla_shape s, double thr,
                                          nabla_window sta, double scale, uint32_t* mask_bits,
                                          int32_t* row_idx, int32_t* row_cnt, int32_t* col_idx,
-                                         int32_t* col_cnt, void* workspace,
+                                         int32_t* col_cnt, nabla_layout layout, void* workspace,
                                          size_t workspace_bytes, nabla_stream_t stream) {
   Dims d;
   nabla_status rc = check_shape(s, &d);
   if (rc != NABLA_OK) return rc;
+  if (layout != NABLA_LAYOUT_REORDERED && layout != NABLA_LAYOUT_NATURAL) return NABLA_ERR_INVALID_ARG;
+  const bool natural = layout == NABLA_LAYOUT_NATURAL;
   if (!(thr >= 0.0 && thr <= 1.0)) return NABLA_ERR_INVALID_ARG;   // also rejects NaN
   if (!(scale > 0.0) || !isfinite(scale)) return NABLA_ERR_INVALID_ARG;
   const int sizes[3] = {sta.t, sta.h, sta.w};
@@ -555,27 +560,36 @@ extern "C" nabla_status nabla_build_mask(const void* q, const void* k, const dou
   cudaError_t e = cudaSuccess;
   const double* qp = q_pool;
   const double* kp = k_pool;
-  if (!qp) {
-    if ((e = pool_blocks_device(q, qp_ws, d, st)) != cudaSuccess) return cuda_status(e);
-    qp = qp_ws;
-  }
-  if (!kp) {
-    if ((e = pool_blocks_device(k, kp_ws, d, st)) != cudaSuccess) return cuda_status(e);
-    kp = kp_ws;
-  }
+  void* fast_scratch = static_cast<char*>(workspace) + kStatusBytes + 2 * pool_bytes;
   // Fast tier (tensor-core logits, certified fp32 cut) for every row, then the fp64
   // kernel for the rows it could not certify.  Without the fast tier: fp64 for all rows.
+  // Given Q and K but no pools, the fast tier pools them itself together with the fp16
+  // split of the means (one pass over each tensor).
   const int32_t* rlist = nullptr;
   const int32_t* rlist_cnt = nullptr;
   if (mask_fast_supported(d)) {
+    if (!qp && !kp) {
+      e = mask_fast_prepare_tokens(q, k, natural, qp_ws, kp_ws, d, scale, fast_scratch,
+                                   static_cast<uint32_t*>(workspace), st);
+      qp = qp_ws;
+      kp = kp_ws;
+    } else {
+      if (!qp && (e = pool_blocks_device(q, qp_ws, d, st, natural)) == cudaSuccess) qp = qp_ws;
+      if (e == cudaSuccess && !kp && (e = pool_blocks_device(k, kp_ws, d, st, natural)) == cudaSuccess) kp = kp_ws;
+      if (e == cudaSuccess)
+        e = mask_fast_prepare(qp, kp, d, scale, fast_scratch, static_cast<uint32_t*>(workspace), st);
+    }
+    if (e != cudaSuccess) return cuda_status(e);
     int32_t* rl = nullptr;
     int32_t* rc = nullptr;
-    e = mask_fast_run(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt,
-                      static_cast<char*>(workspace) + kStatusBytes + 2 * pool_bytes,
-                      static_cast<uint32_t*>(workspace), &rl, &rc, st);
+    e = mask_fast_select(d, scale, thr, sta, mask_bits, row_idx, row_cnt, fast_scratch, &rl, &rc, st);
     if (e != cudaSuccess) return cuda_status(e);
     rlist = rl;
     rlist_cnt = rc;
+  } else {
+    if (!qp && (e = pool_blocks_device(q, qp_ws, d, st, natural)) == cudaSuccess) qp = qp_ws;
+    if (e == cudaSuccess && !kp && (e = pool_blocks_device(k, kp_ws, d, st, natural)) == cudaSuccess) kp = kp_ws;
+    if (e != cudaSuccess) return cuda_status(e);
   }
   e = d.D == 64 ? launch_mask_rows<64>(qp, kp, d, scale, thr, sta, mask_bits, row_idx, row_cnt,
                                        rlist, rlist_cnt, st)
@@ -663,11 +677,11 @@ extern "C" nabla_status nabla_build_mask_sweep(const void* q, const void* k, con
     double* qp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes);
     double* kp_ws = reinterpret_cast<double*>(static_cast<char*>(workspace) + kStatusBytes + pool_bytes);
     if (!qp) {
-      if ((e = pool_blocks_device(q, qp_ws, d, st)) != cudaSuccess) return cuda_status(e);
+      if ((e = pool_blocks_device(q, qp_ws, d, st, false)) != cudaSuccess) return cuda_status(e);
       qp = qp_ws;
     }
     if (!kp) {
-      if ((e = pool_blocks_device(k, kp_ws, d, st)) != cudaSuccess) return cuda_status(e);
+      if ((e = pool_blocks_device(k, kp_ws, d, st, false)) != cudaSuccess) return cuda_status(e);
       kp = kp_ws;
     }
     if (fast && (e = mask_fast_prepare(qp, kp, d, scale, fast_scratch, static_cast<uint32_t*>(workspace), st)) !=

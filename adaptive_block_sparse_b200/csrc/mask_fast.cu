@@ -126,6 +126,79 @@ __global__ void __launch_bounds__(256) split_pools_kernel(
   }
 }
 
+// 1'. the same from the tokens: block means of bf16 Q or K (natural or reordered order)
+// summed in fp64 in token order (exact; the same values as the pooling pass's), written
+// as fp64 means (for the exact tier) and as the fp16 split with the norms, in one pass.
+// Lane l of a warp owns the 16-byte column chunk l % C (C = D / 8) of row l / C of the
+// warp's 32 / C rows of the padded grid [B*H, nbp]; padding rows get zero splits.
+// Either `norm` (per row, for Q) or `max_bits` (per head, for K) is given.
+template <int D, bool GATHER>
+__global__ void __launch_bounds__(128) pool_split_kernel(
+    const uint4* __restrict__ src, double* __restrict__ pool, __half* __restrict__ hi,
+    __half* __restrict__ lo, float* __restrict__ norm, uint32_t* __restrict__ max_bits, int Hg,
+    int W, int Hb, int Wb, int nb, int nbp, long long rows_pad) {
+  constexpr int C = D / 8;
+  constexpr int RPW = 32 / C;
+  const int lane = threadIdx.x & 31;
+  const int c = lane % C;
+  const long long g = (static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5)) * RPW + lane / C;
+  if (g >= rows_pad) return;               // whole rows of lanes leave together
+  const long long bh = g / nbp;
+  const int blk = static_cast<int>(g - bh * nbp);
+  const bool valid = blk < nb;
+  double m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = 0.0;
+  if (valid) {
+    const long long S = static_cast<long long>(nb) * 64;
+    const int t = blk / (Hb * Wb);
+    const int rem = blk - t * (Hb * Wb);
+    const int hb = rem / Wb;
+    const int wb = rem - hb * Wb;
+    const uint4* base = src + bh * S * C + c;
+#pragma unroll 2
+    for (int r = 0; r < 8; ++r) {            // patch row r: tokens 8 r .. 8 r + 7 of the block
+      const long long tok0 = GATHER ? (static_cast<long long>(t) * Hg + hb * 8 + r) * W + wb * 8
+                                    : static_cast<long long>(blk) * 64 + 8 * r;
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(base + (tok0 + u) * C);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          m[2 * k] += static_cast<double>(__uint_as_float(w[k] << 16));
+          m[2 * k + 1] += static_cast<double>(__uint_as_float(w[k] & 0xFFFF0000u));
+        }
+      }
+    }
+    double* out = pool + (bh * nb + blk) * D + c * 8;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      m[k] = m[k] / 64.0;
+      out[k] = m[k];
+    }
+  }
+  __half h8[8], l8[8];
+  double n2 = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    h8[k] = __double2half(m[k]);
+    l8[k] = __double2half(m[k] - static_cast<double>(__half2float(h8[k])));
+    n2 = fma(m[k], m[k], n2);
+  }
+  *reinterpret_cast<uint4*>(hi + g * D + c * 8) = *reinterpret_cast<const uint4*>(h8);
+  *reinterpret_cast<uint4*>(lo + g * D + c * 8) = *reinterpret_cast<const uint4*>(l8);
+#pragma unroll
+  for (int o = C / 2; o > 0; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+  if (c == 0 && valid) {
+    const float nrm = static_cast<float>(sqrt(n2)) * 1.0000001f;
+    if (norm != nullptr) norm[bh * nb + blk] = nrm;
+    if (max_bits != nullptr) atomicMax(&max_bits[bh], __float_as_uint(nrm));
+  }
+}
+
 // ------------------------------------------------------------------------------------
 // 2. pooled logits on the tensor cores
 // ------------------------------------------------------------------------------------
@@ -732,7 +805,50 @@ FastScratch fast_scratch(const Dims& d, void* scratch) {
 
 }  // namespace
 
-// Tiers 1-2a: split of the pooled means and the pooled logits (independent of thr).
+namespace {
+// Tier 2a: the pooled logits from the split (independent of thr).
+cudaError_t mask_fast_logits(const Dims& d, double scale, const FastScratch& f, uint32_t* status,
+                             cudaStream_t st) {
+  const int nbp = mask_fast_nbp(d.nb);
+  const long long rows_pad = static_cast<long long>(d.BH) * nbp;
+  CUtensorMap mqh, mql, mkh, mkl, mout;
+  if (!(make_map_16(&mqh, f.qh, rows_pad, d.D, 128, true) && make_map_16(&mql, f.ql, rows_pad, d.D, 128, true) &&
+        make_map_16(&mkh, f.kh, rows_pad, d.D, 128, true) && make_map_16(&mkl, f.kl, rows_pad, d.D, 128, true) &&
+        make_map_f32(&mout, f.logits, rows_pad, nbp)))
+    return cudaErrorInvalidValue;
+  const long long units = static_cast<long long>(d.BH) * (nbp / 128) * (nbp / 128);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
+  cudaError_t e;
+  if (d.D == 64) {
+    e = cudaFuncSetAttribute(pooled_logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             LogitCfg<64>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    pooled_logits_kernel<64><<<grid, kLogitThreads, LogitCfg<64>::kSmemBytes, st>>>(
+        mqh, mql, mkh, mkl, mout, nbp, units, static_cast<float>(scale), status);
+  } else {
+    e = cudaFuncSetAttribute(pooled_logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             LogitCfg<128>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    pooled_logits_kernel<128><<<grid, kLogitThreads, LogitCfg<128>::kSmemBytes, st>>>(
+        mqh, mql, mkh, mkl, mout, nbp, units, static_cast<float>(scale), status);
+  }
+  return cudaGetLastError();
+}
+
+template <int D, bool GATHER>
+void launch_pool_split(const void* x, double* pool, __half* hi, __half* lo, float* norm, uint32_t* max_bits,
+                       const Dims& d, cudaStream_t st) {
+  const int nbp = mask_fast_nbp(d.nb);
+  const long long rows_pad = static_cast<long long>(d.BH) * nbp;
+  constexpr int kRowsPerCta = 4 * (32 / (D / 8));
+  pool_split_kernel<D, GATHER><<<static_cast<unsigned>((rows_pad + kRowsPerCta - 1) / kRowsPerCta), 128, 0, st>>>(
+      static_cast<const uint4*>(x), pool, hi, lo, norm, max_bits, d.Hg, d.W, d.Hb, d.Wb, d.nb, nbp, rows_pad);
+}
+}  // namespace
+
+// Tiers 1-2a from fp64 pools: split of the pooled means, then the pooled logits.
 cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d, double scale,
                               void* scratch, uint32_t* status, cudaStream_t st) {
   const int nbp = mask_fast_nbp(d.nb);
@@ -748,30 +864,37 @@ cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d,
     split_pools_kernel<128><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, st>>>(
         qp, kp, d.nb, nbp, rows_pad, f.qh, f.ql, f.kh, f.kl, f.qnorm, f.kmax, vec16);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return mask_fast_logits(d, scale, f, status, st);
+}
 
-  CUtensorMap mqh, mql, mkh, mkl, mout;
-  if (!(make_map_16(&mqh, f.qh, rows_pad, d.D, 128, true) && make_map_16(&mql, f.ql, rows_pad, d.D, 128, true) &&
-        make_map_16(&mkh, f.kh, rows_pad, d.D, 128, true) && make_map_16(&mkl, f.kl, rows_pad, d.D, 128, true) &&
-        make_map_f32(&mout, f.logits, rows_pad, nbp)))
-    return cudaErrorInvalidValue;
-  const long long units = static_cast<long long>(d.BH) * (nbp / 128) * (nbp / 128);
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const unsigned grid = static_cast<unsigned>(units < sms ? units : sms);
+// Tiers 1-2a from the bf16 tokens (natural order when `natural`, else reordered): the
+// pools (written to qp_out / kp_out for the exact tier), their split and norms in one
+// pass per tensor, then the pooled logits.
+cudaError_t mask_fast_prepare_tokens(const void* q, const void* k, bool natural, double* qp_out,
+                                     double* kp_out, const Dims& d, double scale, void* scratch,
+                                     uint32_t* status, cudaStream_t st) {
+  const FastScratch f = fast_scratch(d, scratch);
+  cudaError_t e = cudaMemsetAsync(f.kmax, 0, static_cast<size_t>(d.BH) * 4, st);
+  if (e != cudaSuccess) return e;
   if (d.D == 64) {
-    e = cudaFuncSetAttribute(pooled_logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             LogitCfg<64>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    pooled_logits_kernel<64><<<grid, kLogitThreads, LogitCfg<64>::kSmemBytes, st>>>(
-        mqh, mql, mkh, mkl, mout, nbp, units, static_cast<float>(scale), status);
+    if (natural) {
+      launch_pool_split<64, true>(q, qp_out, f.qh, f.ql, f.qnorm, nullptr, d, st);
+      launch_pool_split<64, true>(k, kp_out, f.kh, f.kl, nullptr, f.kmax, d, st);
+    } else {
+      launch_pool_split<64, false>(q, qp_out, f.qh, f.ql, f.qnorm, nullptr, d, st);
+      launch_pool_split<64, false>(k, kp_out, f.kh, f.kl, nullptr, f.kmax, d, st);
+    }
   } else {
-    e = cudaFuncSetAttribute(pooled_logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             LogitCfg<128>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    pooled_logits_kernel<128><<<grid, kLogitThreads, LogitCfg<128>::kSmemBytes, st>>>(
-        mqh, mql, mkh, mkl, mout, nbp, units, static_cast<float>(scale), status);
+    if (natural) {
+      launch_pool_split<128, true>(q, qp_out, f.qh, f.ql, f.qnorm, nullptr, d, st);
+      launch_pool_split<128, true>(k, kp_out, f.kh, f.kl, nullptr, f.kmax, d, st);
+    } else {
+      launch_pool_split<128, false>(q, qp_out, f.qh, f.ql, f.qnorm, nullptr, d, st);
+      launch_pool_split<128, false>(k, kp_out, f.kh, f.kl, nullptr, f.kmax, d, st);
+    }
   }
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return mask_fast_logits(d, scale, f, status, st);
 }
 
 // Tier 2b: the certified cut for one thr from the logits mask_fast_prepare wrote.  Rows

@@ -176,8 +176,10 @@ cudaError_t launch_reorder(const void* src, void* dst, double* pool, const Dims&
 
 }  // namespace
 
-// Pools a reordered bf16 tensor into fp64 block means (used by the mask build).
-cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st) {
+// Pools a bf16 tensor (reordered, or in the natural order) into fp64 block means (used by
+// the mask build).
+cudaError_t pool_blocks_device(const void* x, double* pool, const Dims& d, cudaStream_t st, bool natural) {
+  if (natural) return d.D == 64 ? go_pool<64, true>(x, pool, d, st) : go_pool<128, true>(x, pool, d, st);
   return d.D == 64 ? go_pool<64, false>(x, pool, d, st) : go_pool<128, false>(x, pool, d, st);
 }
 

@@ -232,14 +232,19 @@ class Path:
     def launches_per_step(self):
         """Kernels of this library launched by one step (memsets not counted).
 
-        Inference: pool Q, pool K; mask (split, logits, select, fp64 rescue); forward
-        (schedule: per-head sort + head placement; attention).  Training: pool Q, pool K,
+        Inference: the mask (pooling + fp16 split of Q, of K, logits, select, fp64
+        rescue); forward (schedule: per-head sort + head placement; attention).  Training:
         V to fp16; the mask as above + column lists; forward; backward (2 schedules of 2
         launches, preprocess, dK/dV, dQ).
         """
         if not self.wl.backward:
-            return 2 + 4 + 3
-        return 3 + 4 + 1 + 3 + 7
+            return 5 + 3
+        return 1 + 5 + 1 + 3 + 7
+
+    def fill_pools(self):
+        """The fp64 pooled means of Q and K (for the measurements made from pools)."""
+        self.m.nabla_reorder(self.q, None, self.shape, pool_out=self.qp)
+        self.m.nabla_reorder(self.k, None, self.shape, pool_out=self.kp)
 
     def _mark(self, name, timing):
         if timing:
@@ -250,15 +255,14 @@ class Path:
     def step(self, timing=False):
         m, sh, wl = self.m, self.shape, self.wl
         self._mark("t0", timing)
-        m.nabla_reorder(self.q, None, sh, pool_out=self.qp)
-        m.nabla_reorder(self.k, None, sh, pool_out=self.kp)
         if wl.backward:
             m.nabla_reorder(self.v, self.vh, sh, inverse=m.REORDER_KEEP)
         self._mark("t_reorder", timing)
-        m.nabla_build_mask(None, None, sh, self.thr, wl.window, mask_bits=self.bits,
+        # the mask pools Q and K itself (natural order), one pass over each
+        m.nabla_build_mask(self.q, self.k, sh, self.thr, wl.window, mask_bits=self.bits,
                            row_idx=self.ridx, row_cnt=self.rcnt, col_idx=self.cidx,
-                           col_cnt=self.ccnt, q_pool=self.qp, k_pool=self.kp,
-                           workspace=self.mask_ws)
+                           col_cnt=self.ccnt, workspace=self.mask_ws,
+                           layout=m.NABLA_LAYOUT_NATURAL)
         self._mark("t_mask", timing)
         v = self.vh if wl.backward else self.v
         m.nabla_attn_fwd(self.q, self.k, v, self.bits, sh, o=self.o, o_dtype=self.o_dtype,
@@ -524,8 +528,8 @@ def main():
     ms = max_over_ranks(ms_local, world, dev)
     path.check_status()
     fwd_ms = statistics.mean(path.segment_ms("t_mask", "t_fwd"))
-    mask_ms_fused = statistics.mean(path.segment_ms("t_reorder", "t_mask"))
-    reorder_ms = statistics.mean(path.segment_ms("t0", "t_reorder"))
+    mask_ms_step = statistics.mean(path.segment_ms("t_reorder", "t_mask"))
+    v16_ms = statistics.mean(path.segment_ms("t0", "t_reorder")) if wl.backward else None
     bwd_ms = statistics.mean(path.segment_ms("t_fwd", "t_bwd")) if wl.backward else None
 
     fl_fwd = 4.0 * 64 * 64 * wl.D
@@ -537,16 +541,20 @@ def main():
 
     # ---- side measurements (outside the timed region) ----------------------------------------
     m, sh = path.m, path.shape
-    # the mask from bf16 Q and K (pooling included): natural order -> pool alone, then the
-    # mask from the means; reordered order -> the mask call pools itself
+    # the mask from bf16 Q and K in the natural order (the step's call: pooling included)
     def mask_from_qk():
-        m.nabla_reorder(path.q, None, sh, pool_out=path.qp)
-        m.nabla_reorder(path.k, None, sh, pool_out=path.kp)
-        m.nabla_build_mask(None, None, sh, path.thr, wl.window, mask_bits=path.bits,
-                           row_idx=path.ridx, row_cnt=path.rcnt, q_pool=path.qp,
-                           k_pool=path.kp, workspace=path.mask_ws)
+        m.nabla_build_mask(path.q, path.k, sh, path.thr, wl.window, mask_bits=path.bits,
+                           row_idx=path.ridx, row_cnt=path.rcnt, workspace=path.mask_ws,
+                           layout=m.NABLA_LAYOUT_NATURAL)
     mask_ms = time_call(mask_from_qk, 5)
     mask_bytes = 2 * BH * wl.S * wl.D * 2 + BH * nb * sh.nw * 4
+    # the same in two passes: the fp64 pools alone (the pooling pass of the reorder entry
+    # point), then the mask from the pools
+    pool_ms = time_call(path.fill_pools, 5)
+    pool_bytes = 2 * BH * wl.S * wl.D * 2 + 2 * BH * nb * wl.D * 8
+    mask_pools_ms = time_call(lambda: m.nabla_build_mask(
+        None, None, sh, path.thr, wl.window, mask_bits=path.bits, row_idx=path.ridx,
+        row_cnt=path.rcnt, q_pool=path.qp, k_pool=path.kp, workspace=path.mask_ws), 5)
     # several thresholds from one pooled map (the pools of the step), against one mask
     # call per threshold; the masks are the same bit for bit
     sweep_thrs = (0.5, 0.7, 0.8, 0.9, 0.95)
@@ -565,10 +573,6 @@ def main():
     sweep = {"thrs": list(sweep_thrs), "ms": sweep_ms, "ms_separate_calls": separate_ms,
              "sparsity": m.sparsity_curve(sw_cnt, sh)}
     del sw_bits, sw_cnt
-    # bytes of the pass before the mask: pooling of Q, K (+ V read and written as fp16 on
-    # the training path)
-    reorder_bytes = 2 * BH * wl.S * wl.D * 2 + (2 * BH * wl.S * wl.D * 2 if wl.backward else 0) \
-        + 2 * BH * nb * wl.D * 8
     # all-ones mask (padding bits are ignored by the kernels)
     dense_bits = torch.full((wl.B, wl.H, nb, sh.nw), -1, dtype=torch.int32, device=dev)
     dense_iters = 2 if nb > 1000 else 5
@@ -702,8 +706,9 @@ def main():
         "dense_fwd_ms": dense_ms, "dense_tflops": dense_tflops, "speedup_vs_dense": dense_ms / fwd_ms,
         "mask_ms": mask_ms, "mask_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
         "mask_frac_hbm": mask_bytes / (mask_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-        "mask_ms_from_pools": mask_ms_fused, "mask_sweep_from_pools": sweep, "reorder_ms": reorder_ms,
-        "reorder_gbs": reorder_bytes / (reorder_ms * 1e-3) / 1e9,
+        "mask_ms_in_step": mask_ms_step, "mask_ms_from_pools": mask_pools_ms,
+        "pool_ms": pool_ms, "pool_gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
+        "mask_sweep_from_pools": sweep, "v_to_f16_ms": v16_ms,
         "bwd_ms": bwd_ms, "bwd_tflops_kept": bwd_tflops,
         "kept_tiles": kept, "sparsity": sparsity, "sparsity_per_head": per_head,
         "near_threshold_blocks": near,

@@ -110,7 +110,9 @@ nabla_status nabla_reorder(const void *src, nabla_dtype src_dtype, void *dst,
  * ascending CDF at j is > 1 - thr).  thr >= 1 keeps every block; thr == 0 keeps none,
  * so the result is the pure STA mask.  The decision is taken in fp64.
  *
- * q, k       : bf16 [B,H,S,D] reordered (read only when the matching pool is NULL).
+ * q, k       : bf16 [B,H,S,D] in the token order given by layout (read only when the
+ *              matching pool is NULL; given both without pools, the call pools them in
+ *              the same pass that prepares its tensor-core operands).
  * q_pool,
  * k_pool     : nullable fp64 [B,H,nb,D] block means from nabla_reorder; when given, the
  *              call reads them instead of q / k (q / k may then be NULL).
@@ -127,6 +129,8 @@ nabla_status nabla_reorder(const void *src, nabla_dtype src_dtype, void *dst,
  * col_idx,
  * col_cnt    : out, nullable: the transpose (query blocks that keep key block j,
  *              ascending), same shapes and the same rule; used by the backward pass.
+ * layout     : token order of q and k: NABLA_LAYOUT_REORDERED or NABLA_LAYOUT_NATURAL
+ *              (each 8 x 8 patch of a frame gathered as it is read); ignored for pools.
  * workspace  : >= nabla_mask_workspace_bytes(s) bytes, 256-byte aligned.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  * --------------------------------------------------------------------------------- */
@@ -135,8 +139,8 @@ nabla_status nabla_build_mask(const void *q, const void *k, const double *q_pool
                               const double *k_pool, nabla_shape s, double thr,
                               nabla_window sta, double scale, uint32_t *mask_bits,
                               int32_t *row_idx, int32_t *row_cnt, int32_t *col_idx,
-                              int32_t *col_cnt, void *workspace, size_t workspace_bytes,
-                              nabla_stream_t stream);
+                              int32_t *col_cnt, nabla_layout layout, void *workspace,
+                              size_t workspace_bytes, nabla_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Several thresholds on one pooled map ("mask reuse").

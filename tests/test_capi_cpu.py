@@ -86,9 +86,9 @@ def test_host_validation_rejects_bad_arguments(lib):
     ws_need = lib.nabla_mask_workspace_bytes(good)
     assert ws_need > 256
 
-    def bm(thr=0.5, window=win, scale=0.125, bits=A, ridx=None, rcnt=None, ws=Bp, wsb=ws_need):
+    def bm(thr=0.5, window=win, scale=0.125, bits=A, ridx=None, rcnt=None, ws=Bp, wsb=ws_need, layout=0):
         return lib.nabla_build_mask(A, A, None, None, good, thr, window, scale, bits, ridx, rcnt,
-                                    None, None, ws, wsb, st)
+                                    None, None, layout, ws, wsb, st)
     assert bm(thr=1.5) == INV
     assert bm(thr=-0.1) == INV
     assert bm(thr=float("nan")) == INV
@@ -100,6 +100,7 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert bm(wsb=ws_need - 1) == WS
     assert bm(ws=None) == WS
     assert bm(ws=ctypes.c_void_p(0x20000010)) == WS                       # misaligned workspace
+    assert bm(layout=2) == INV                                            # unknown layout
     thr3 = (ctypes.c_double * 3)(0.5, 0.8, 0.95)
 
     def sw(thrs=thr3, n=3, window=win, bits=A, ws=Bp, wsb=ws_need, qp=A):

@@ -165,6 +165,12 @@ def test_mask_parity(data, name, thr, window):
     # the pooled means from the fused reorder give the identical mask
     bits2, *_ = gpu_mask(None, None, shape, thr, window, cols=False, q_pool=qp, k_pool=kp)
     assert torch.equal(bits2, bits)
+    # so do Q and K in the natural token order, pooled by the mask build itself
+    m = nbl()
+    bits3, ridx3, rcnt3, cidx3, ccnt3 = gpu_mask(q, k, shape, thr, window, layout=m.NABLA_LAYOUT_NATURAL)
+    assert torch.equal(bits3, bits)
+    assert torch.equal(rcnt3, rcnt) and torch.equal(ccnt3, ccnt)
+    check_lists(ridx3, rcnt3, gm)
 
 
 # Degenerate rows for the cut: head 0 has Q = K = 0 (every block of a row has the same
