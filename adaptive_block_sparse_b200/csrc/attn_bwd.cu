@@ -37,6 +37,8 @@ namespace nabla {
 bool make_map_16(CUtensorMap* map, const void* base, long long rows, int D, int box_rows,
                  bool fp16);
 bool make_map_kv(CUtensorMap* map, const void* base, long long rows, int D, bool fp16);
+bool make_map_f32(CUtensorMap* map, const void* base, long long rows, int D);
+bool make_map_nat_f32(CUtensorMap* map, const void* base, long long frames, int Hg, int W, int D);
 
 namespace {
 
@@ -233,6 +235,32 @@ struct BwdCfg {
 // 16 of the 32 columns it read, [32h, 32h+16).
 __device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 2 ? kk * 8 : 32 + (kk - 2) * 8; }
 
+// Epilogue store of 32 f32 columns [x0, x0 + 32) of a warp's 32 rows (this lane's row:
+// v[0..31], already scaled): the rows are staged in the 128-byte-swizzled layout of a
+// tiled copy at `stage` (4 KB, used once), and one lane stores them with TMA -- rows
+// 32 q32 .. 32 q32 + 31 of block `blk` of head bh: 32 reordered rows, or a 4 x 8 token
+// part of the block's 8 x 8 patch.  The copy runs on after the CTA has moved on; the
+// CTA waits only for it to have read the staging before it exits.
+__device__ __forceinline__ void store_rows_f32(const CUtensorMap* map, unsigned char* stage, const uint32_t (&v)[32],
+                                               int lane, int x0, long long bh, int blk, int q32,
+                                               const NatMap& nat, int T) {
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch)
+    *reinterpret_cast<uint4*>(stage + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+        make_uint4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if (nat.on) {
+      const int tf = blk / nat.HW, rr = blk - tf * nat.HW, hb = rr / nat.Wb, wb = rr - hb * nat.Wb;
+      tma_store_4d(map, stage, x0, wb * 8, hb * 8 + 4 * q32, static_cast<int>(bh * T + tf));
+    } else {
+      tma_store_2d(map, stage, x0, static_cast<int>(bh * nat.S + static_cast<long long>(blk) * 64 + 32 * q32));
+    }
+    bulk_commit_group();
+  }
+}
+
 // -------------------------------------------------------------------------------------
 // 2. dK / dV over column lists
 // -------------------------------------------------------------------------------------
@@ -256,7 +284,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_q64,
                          const __grid_constant__ CUtensorMap map_do64,
                          const __grid_constant__ CUtensorMap map_k64,
-                         const __grid_constant__ CUtensorMap map_v64, const BwdParams prm) {
+                         const __grid_constant__ CUtensorMap map_v64,
+                         const __grid_constant__ CUtensorMap map_out0,
+                         const __grid_constant__ CUtensorMap map_out1, const BwdParams prm) {
   using C = BwdCfg<D>;
   using L = DkdvLayout<D>;
   extern __shared__ unsigned char smem_raw[];
@@ -495,28 +525,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       have = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, prm.status, kDevTimeoutOBar));
       tc_fence_after();
     }
+    if (have) {
+      // Every MMA has completed and every copy into the stage ring has landed and been
+      // read (the last accumulation waited for all of them), so the ring is free: each
+      // warp stages its 32 rows x 64 columns of dV and dK there (4 KB per 32 columns).
+      unsigned char* stage = sStage + mw * (D / 2) * 4 * 32 * 2;
 #pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-      float* out = which == 0 ? prm.out0 : prm.out1;
-      const float mul = which == 0 ? 1.f : prm.scale;
-      const uint32_t colbase = (which == 0 ? C::kColAcc0 : C::kColAcc1) + (D / 2) * h;
+      for (int which = 0; which < 2; ++which) {
+        const float mul = which == 0 ? 1.f : prm.scale;
+        const uint32_t colbase = (which == 0 ? C::kColAcc0 : C::kColAcc1) + (D / 2) * h;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D / 2; c0 += 32) {
-        uint32_t ov[32];
-        if (have) {
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+          uint32_t ov[32];
           tmem_ld32(tmem + lane_base + colbase + c0, ov);
           tmem_wait_ld();
-        } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) ov[c] = 0u;
+          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * mul);
+          if (valid)   // warp-uniform: a warp's rows are one block
+            store_rows_f32(which == 0 ? &map_out0 : &map_out1, stage, ov, lane, (D / 2) * h + c0, bh, blk,
+                           (mw & 3) & 1, prm.nat, prm.T);
+          stage += 4096;
         }
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(out + tok * D + (D / 2) * h + c0);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            dst[c] = make_float4(__uint_as_float(ov[4 * c]) * mul, __uint_as_float(ov[4 * c + 1]) * mul,
-                                 __uint_as_float(ov[4 * c + 2]) * mul, __uint_as_float(ov[4 * c + 3]) * mul);
-        }
+      }
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+    } else {
+      // no step, or a wait gave up: zeros, stored directly (copies may still be landing
+      // in the stage ring)
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        float* out = which == 0 ? prm.out0 : prm.out1;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D / 2; c0 += 4)
+          if (valid) *reinterpret_cast<float4*>(out + tok * D + (D / 2) * h + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
   }
@@ -549,7 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap map_q64,
                        const __grid_constant__ CUtensorMap map_do64,
                        const __grid_constant__ CUtensorMap map_k64,
-                       const __grid_constant__ CUtensorMap map_v64, const BwdParams prm) {
+                       const __grid_constant__ CUtensorMap map_v64,
+                       const __grid_constant__ CUtensorMap map_out0, const BwdParams prm) {
   using C = BwdCfg<D>;
   using L = DqLayout<D>;
   extern __shared__ unsigned char smem_raw[];
@@ -774,24 +816,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       have = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, prm.status, kDevTimeoutOBar));
       tc_fence_after();
     }
+    if (have) {
+      // the stage ring is free (as in the dK/dV pass): 32 rows x 64 columns of dQ per warp
+      unsigned char* stage = sStage + mw * (D / 2) * 4 * 32;
 #pragma unroll 1
-    for (int c0 = 0; c0 < D / 2; c0 += 32) {
-      uint32_t ov[32];
-      if (have) {
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        uint32_t ov[32];
         tmem_ld32(tmem + lane_base + C::kColAcc0 + (D / 2) * h + c0, ov);
         tmem_wait_ld();
-      } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) ov[c] = 0u;
+        for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * prm.scale);
+        if (valid)
+          store_rows_f32(&map_out0, stage, ov, lane, (D / 2) * h + c0, bh, blk, (mw & 3) & 1, prm.nat, prm.T);
+        stage += 4096;
       }
-      if (valid) {
-        float4* dst = reinterpret_cast<float4*>(prm.out0 + otok * D + (D / 2) * h + c0);
-        const float mul = prm.scale;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          dst[c] = make_float4(__uint_as_float(ov[4 * c]) * mul, __uint_as_float(ov[4 * c + 1]) * mul,
-                               __uint_as_float(ov[4 * c + 2]) * mul, __uint_as_float(ov[4 * c + 3]) * mul);
-      }
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+    } else {
+#pragma unroll 1
+      for (int c0 = 0; c0 < D / 2; c0 += 4)
+        if (valid) *reinterpret_cast<float4*>(prm.out0 + otok * D + (D / 2) * h + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   tc_fence_before();
@@ -848,6 +892,15 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
             make_map_kv(&mq3, q16, rows, D, true) && make_map_kv(&mdo3, do16, rows, D, true) &&
             make_map_kv(&mk3, k16, rows, D, true) && make_map_kv(&mv3, v16, rows, D, true);
   if (!*map_ok) return cudaErrorInvalidValue;
+  // f32 gradient maps for the epilogues' tiled stores
+  CUtensorMap mdq, mdk, mdv;
+  const long long frames = static_cast<long long>(d.BH) * d.T;
+  *map_ok = natural ? (make_map_nat_f32(&mdq, dq, frames, d.Hg, d.W, D) &&
+                       make_map_nat_f32(&mdk, dk, frames, d.Hg, d.W, D) &&
+                       make_map_nat_f32(&mdv, dv, frames, d.Hg, d.W, D))
+                    : (make_map_f32(&mdq, dq, rows, D) && make_map_f32(&mdk, dk, rows, D) &&
+                       make_map_f32(&mdv, dv, rows, D));
+  if (!*map_ok) return cudaErrorInvalidValue;
 
   BwdParams p;
   p.delta = delta;
@@ -871,7 +924,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DkdvLayout<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq3, mdo3, mk64, mv64, p);
+  attn_bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kSmemBytes, st>>>(mq3, mdo3, mk64, mv64, mdv, mdk, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   p.order = order_rows;
@@ -882,7 +935,7 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, int v_f16, c
   e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DqLayout<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk3, mv3, p);
+  attn_bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kSmemBytes, st>>>(mq64, mdo64, mk3, mv3, mdq, p);
   return cudaGetLastError();
 }
 
