@@ -7,24 +7,26 @@
 //
 //  * work tile = 128 query rows = two query blocks of one head (M = 128 MMAs): the same
 //    patch in frames 2u and 2u + 1 (tile_blocks()).  The tile walks the ascending union
-//    of the two blocks' kept key blocks, read from the mask bitmask, two key blocks per
-//    step (N = 128 keys per MMA); a half of the rows whose block does not keep a key
-//    block is masked (-inf);
+//    of the two blocks' kept key blocks, read from the mask bitmask, one key block per
+//    step (N = 64 keys per S MMA); the half of the rows whose block does not keep a key
+//    block skips its softmax (P = 0);
 //  * persistent: one CTA per SM runs two independent pipelines ("slots"), each taking
 //    tiles through an atomic counter in the schedule's order (heads by their longest
-//    tile, tiles longest first inside a head).  A slot owns
-//    a Q buffer, one K and one V stage, a TMEM score buffer and a TMEM accumulator; per
-//    step its chain is S = Q K^T (tcgen05.mma) -> softmax -> O += P V with P read from
-//    TMEM.  The two chains share the tensor core: while one slot runs its softmax, the
-//    other's MMAs run, and a tile change in one slot is covered by the other;
+//    tile, tiles longest first inside a head).  A slot owns a Q buffer, two K and two V
+//    stages, two TMEM score buffers and a TMEM accumulator; per step its chain is
+//    S = Q K^T (tcgen05.mma) -> softmax -> O += P V with P read from TMEM, and S of the
+//    next step is issued before P V of this one, into the other score buffer.  The two
+//    chains share the tensor core: while one slot runs its softmax, the other's MMAs
+//    run, and a tile change in one slot is covered by the other;
 //  * per slot: a streamer warp fetches the tiles (the union of the two bitmask rows is
 //    counted and walked warp-cooperatively, the tile's Q prefetched into L2) and loads
-//    Q, K and V with TMA (128-byte swizzle); one lane of an issuer warp issues the MMAs;
-//    a softmax warpgroup (one query row per thread, TMEM lane = row) holds a whole row
-//    of 128 scores in registers, rescales O only when a row maximum grows by more than
-//    2^8, rounds P to the V operand's 16-bit type (the row sum takes the rounded
-//    weights), and at the end of the tile normalises O, releases the accumulator and
-//    writes O through a shared-memory staging area with tiled TMA stores, and the LSE;
+//    Q, K and V with TMA (128-byte swizzle, one copy per K or V block); one lane of an
+//    issuer warp issues the MMAs; a softmax warpgroup (one query row per thread, TMEM
+//    lane = row) holds the row's 64 scores of a step in registers, rescales O only when
+//    a row maximum grows by more than 2^8, rounds P to the V operand's 16-bit type (the
+//    row sum takes the rounded weights), and at the end of the tile normalises O,
+//    releases the accumulator and writes O through a shared-memory staging area with
+//    tiled TMA stores, and the LSE;
 //  * the producer warps give registers to the softmax warpgroups (setmaxnreg);
 //  * every barrier wait is bounded; on a timeout a kernel records a status code, stops,
 //    drains its own copies and MMAs and frees TMEM.
@@ -573,10 +575,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk;
             if constexpr (VF16) {
               pk = pack_f16x2(pr.x, pr.y);
-              acc = __fadd2_rn(acc, make_float2(f16lo(pk), f16hi(pk)));
+              add_halves_f16(acc, pk);
             } else {
               pk = pack_bf16x2(pr.x, pr.y);
-              acc = __fadd2_rn(acc, make_float2(bf16lo(pk), bf16hi(pk)));
+              add_halves_bf16(acc, pk);
             }
             sv[e] = pk;
           }

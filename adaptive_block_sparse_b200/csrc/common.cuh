@@ -441,17 +441,21 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The two fp16 halves of a packed pair, widened to f32 (exact).
-__device__ __forceinline__ float f16lo(uint32_t v) {
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+// acc.x += low half, acc.y += high half of a packed 16-bit pair, each widened to f32
+// (exact) inside one mixed-precision add (round to nearest): the same values as unpacking
+// and adding, one instruction per element instead of two.
+__device__ __forceinline__ void add_halves_bf16(float2& acc, uint32_t v) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "r"(v));
 }
-__device__ __forceinline__ float f16hi(uint32_t v) {
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+__device__ __forceinline__ void add_halves_f16(float2& acc, uint32_t v) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %1, hi, %1;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "r"(v));
 }
-
-// The two bf16 halves of a packed pair, widened to f32 (exact).
-__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
 // max of three (one instruction on sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
