@@ -44,7 +44,8 @@ constexpr int kSoftmaxWarp0 = 4;          // warps 4..7 = slot 0, 8..11 = slot 1
 constexpr int kMetaRing = 3;              // tile descriptors per slot
 constexpr int kMetaInts = 8;              // item, bh, block a, block b, steps
 // Registers per thread: the block launches with kLaunchRegs x 384; the producer warps
-// (0-3) give registers up so that each softmax thread can hold a row of 128 scores.
+// (0-3) give registers up to the softmax warps (a row's 64 scores of a step, the packed
+// weights, the epilogue's packed O row).
 constexpr int kLaunchRegs = 168;
 constexpr int kRegProducer = 56;
 constexpr int kRegSoftmax = 224;

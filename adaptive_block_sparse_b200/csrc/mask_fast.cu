@@ -10,9 +10,11 @@
 // Computing it in fp64 on CUDA cores is slow, so this tier decides every row whose cut
 // is unambiguous at a proven error bound, and hands the others to the fp64 kernel:
 //
-//  1. split_pools_kernel: the fp64 block means q, k are split into fp16 pairs
-//     q = q_hi + q_lo + r (|r| <= 2^-22 |q|), padded to a multiple of 256 rows; row
-//     norms |q_i| and the per-head maximum |k_j| are kept for the error bound.
+//  1. pool_split_kernel (from the bf16 tokens: the fp64 block means, written out for the
+//     fp64 tier, in the same pass) or split_pools_kernel (from given means): the means
+//     q, k are split into fp16 pairs q = q_hi + q_lo + r (|r| <= 2^-22 |q|), padded to a
+//     multiple of 256 rows; row norms |q_i| and the per-head maximum |k_j| are kept for
+//     the error bound.
 //  2. pooled_logits_kernel: A = scale * (q_hi k_hi^T + (q_hi k_lo^T + q_lo k_hi^T)) with
 //     tcgen05 (M = 128, N = 128, K = 16 per instruction, fp32 accumulate in TMEM; the
 //     dominant q_hi k_hi^T term has its own accumulator), written to an fp32 scratch by
