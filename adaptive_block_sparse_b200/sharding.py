@@ -8,7 +8,7 @@ sharded by sequence (rank r holding a contiguous range of S/N tokens of every he
 exchanges them once before attention and once after:
 
     [B, H, S/N, D] per rank  --all-to-all-->  every token of this rank's heads
-    hot path on the rank's heads (pool, mask, forward in the natural token order)
+    hot path on the rank's heads (mask with its pooling, forward; natural token order)
     this rank's heads          --all-to-all-->  [B, H, S/N, D] per rank
 
 Two ways to assign heads to ranks:
@@ -110,17 +110,12 @@ def units_to_seq(y, plan, B, H, group=None):
 
 
 def nabla_local_heads(q, k, v, shape, thr, window=(0, 0, 0), scale=None):
-    """The hot path on one rank's heads, natural token order in and out: fp64 pools of Q
-    and K, the block mask from them, the forward reading Q, K, V in place.  Returns bf16 O
-    [B, h, S, D]."""
+    """The hot path on one rank's heads, natural token order in and out: the block mask
+    from Q and K (pooled by the mask build itself), the forward reading Q, K, V in place.
+    Returns bf16 O [B, h, S, D]."""
     import adaptive_block_sparse_b200 as m
-    dev = q.device
-    qp = torch.empty(shape.B, shape.H, shape.nb, shape.D, dtype=torch.float64, device=dev)
-    kp = torch.empty_like(qp)
-    m.nabla_reorder(q, None, shape, pool_out=qp)
-    m.nabla_reorder(k, None, shape, pool_out=kp)
-    bits, _, _, _, _ = m.nabla_build_mask(None, None, shape, thr, window, scale=scale,
-                                          q_pool=qp, k_pool=kp)
+    bits, _, _, _, _ = m.nabla_build_mask(q, k, shape, thr, window, scale=scale,
+                                          layout=m.NABLA_LAYOUT_NATURAL)
     o, _ = m.nabla_attn_fwd(q, k, v, bits, shape, scale=scale, layout=m.NABLA_LAYOUT_NATURAL)
     return o
 
