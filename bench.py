@@ -380,9 +380,10 @@ def workload_config(wl, thr, world, scaling="weak"):
     """The ``config`` object of a bench line; both arms print the same one."""
     return {"workload": wl.name, "B": wl.B, "H": wl.H, "grid": [wl.T, wl.Hg, wl.W],
             "D": wl.D, "P": wl.P, "thr": thr, "sta": list(wl.window),
-            "step": ("pool Q/K, mask, attn fwd on natural-order Q/K/V" if not wl.backward
-                     else "pool Q/K, V to fp16, mask + lists, attn fwd and bwd on natural-order "
-                          "Q/K/V/dO"),
+            "step": ("mask from natural-order Q/K (pooling fused), attn fwd on natural-order "
+                     "Q/K/V" if not wl.backward
+                     else "V to fp16, mask + lists from natural-order Q/K (pooling fused), attn "
+                          "fwd and bwd on natural-order Q/K/V/dO"),
             "l2": "inputs larger than L2 (no flush)",
             "parallelism": (f"heads-replicated x{world}" if scaling == "weak"
                             else f"heads split over {world} ranks (LPT by kept tiles)")}
