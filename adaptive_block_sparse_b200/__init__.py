@@ -204,7 +204,6 @@ def nabla_build_mask(q, k, shape: Shape, thr: float, window=(0, 0, 0), scale=Non
     """NABLA block mask.  Returns (mask_bits, row_idx, row_cnt, col_idx, col_cnt).
     ``layout``: token order of ``q`` and ``k`` when they are read (no pools given)."""
     dev = next(t.device for t in (q, q_pool, mask_bits, workspace) if t is not None)
-    BH = shape.B * shape.H
     if mask_bits is None:
         mask_bits = torch.empty(shape.B, shape.H, shape.nb, shape.nw, dtype=torch.int32, device=dev)
     if workspace is None:
@@ -216,7 +215,6 @@ def nabla_build_mask(q, k, shape: Shape, thr: float, window=(0, 0, 0), scale=Non
                                  _ptr(row_idx), _ptr(row_cnt), _ptr(col_idx), _ptr(col_cnt),
                                  int(layout), _ptr(workspace), workspace.numel(), _stream(stream)),
            "nabla_build_mask")
-    del BH
     return mask_bits, row_idx, row_cnt, col_idx, col_cnt
 
 
