@@ -38,10 +38,6 @@ cudaError_t mask_fast_prepare(const double* qp, const double* kp, const Dims& d,
 cudaError_t mask_fast_select(const Dims& d, double scale, double thr, const nabla_window& w,
                              uint32_t* bits, int32_t* ridx, int32_t* rcnt, void* scratch,
                              int32_t** rescue_list, int32_t** rescue_cnt, cudaStream_t st);
-cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, double scale, double thr,
-                          const nabla_window& w, uint32_t* bits, int32_t* ridx, int32_t* rcnt,
-                          void* scratch, uint32_t* status, int32_t** rescue_list,
-                          int32_t** rescue_cnt, cudaStream_t st);
 
 namespace {
 

@@ -937,14 +937,4 @@ cudaError_t mask_fast_select(const Dims& d, double scale, double thr, const nabl
   return e;
 }
 
-// Runs tiers 1-2 (split, logits, certified select) for one thr.
-cudaError_t mask_fast_run(const double* qp, const double* kp, const Dims& d, double scale, double thr,
-                          const nabla_window& w, uint32_t* bits, int32_t* ridx, int32_t* rcnt,
-                          void* scratch, uint32_t* status, int32_t** rescue_list,
-                          int32_t** rescue_cnt, cudaStream_t st) {
-  cudaError_t e = mask_fast_prepare(qp, kp, d, scale, scratch, status, st);
-  if (e != cudaSuccess) return e;
-  return mask_fast_select(d, scale, thr, w, bits, ridx, rcnt, scratch, rescue_list, rescue_cnt, st);
-}
-
 }  // namespace nabla
