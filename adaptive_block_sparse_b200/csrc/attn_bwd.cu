@@ -10,7 +10,9 @@
 //   dS = P * (dP - Dr),  dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
 //
 // Deterministic, no floating-point atomics, three launches:
-//   1. preprocess: Dr = rowsum(dO * O) and LSE in log2 units (HBM-bound);
+//   1. preprocess: Dr = rowsum(dO * O), LSE in log2 units and fp16 copies of Q, K, V, dO
+//      in the fractal block order, gathered from the natural token order when the
+//      tensors come in it (HBM-bound);
 //   2. dK/dV: one CTA per pair of key blocks (the same patch in frames 2u and 2u + 1, as
 //      the forward pairs query blocks: their column lists overlap most; 128 key rows ->
 //      M = 128 MMAs) walks the ascending union of the two blocks' query-block (column)
@@ -20,10 +22,12 @@
 //      accumulate in TMEM;
 //   3. dQ: one CTA per pair of query blocks walks the union of the row lists:
 //      S = Q K^T and dP = dO V^T into TMEM, dS written back over dP, dQ += dS K.
-// Warp roles: warp 0 = TMA producer (four-stage ring), warp 1 = MMA issuer and TMEM owner,
-// warps 4-11 = element-wise math (a key or query row per TMEM lane, each 64-wide tile
-// split in two column halves between warps w and w + 4) and epilogue.  Every wait is
-// bounded.
+// Warp roles: warp 0 = TMA producer (four-stage ring; the whole warp walks the lists, 32
+// entries per load), warp 1 = MMA issuer and TMEM owner, warps 4-11 = element-wise math
+// (a key or query row per TMEM lane, each 64-wide tile split in two column halves between
+// warps w and w + 4) and epilogue (fp32 gradients staged in the freed ring and stored
+// with tiled TMA stores, at the natural token indices when the tensors came in that
+// order).  Every wait is bounded.
 #include <math.h>
 
 #include <cudaTypedefs.h>
