@@ -149,7 +149,13 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
       widen(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(v) + sbase), t);
       *reinterpret_cast<uint4*>(v16 + base) = to_f16(t);
     } else if (nat.on) {   // an fp16 V in the natural order is gathered as it is
-      *reinterpret_cast<uint4*>(v16 + base) = *reinterpret_cast<const uint4*>(static_cast<const __half*>(v) + sbase);
+      const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __half*>(v) + sbase);
+      // an infinite or NaN half (exponent bits all set) is out of the range
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        range_ok = range_ok && (w[i] & 0x7C00u) != 0x7C00u && (w[i] & 0x7C000000u) != 0x7C000000u;
+      *reinterpret_cast<uint4*>(v16 + base) = u;
     }
   }
 #pragma unroll

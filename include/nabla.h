@@ -214,7 +214,8 @@ nabla_status nabla_attn_fwd(const void *q, const void *k, const void *v, nabla_d
  * q, k, dout: bf16 [B,H,S,D]; v: bf16 or fp16 (v_dtype); o: forward output (o_dtype);
  * lse: forward LSE.  The MMAs run on fp16 copies of Q, K, V and dO made in the
  * workspace (P and dS rounded to fp16): inputs must satisfy |x| <= 65504, otherwise the
- * device status word reports it (0x201).
+ * device status word reports it (0x201); an fp16 V is checked for infinite or NaN
+ * values when it is gathered (natural layout) and used as given in the reordered layout.
  * row_* and col_* lists from nabla_build_mask / nabla_mask_lists.
  * dq, dk, dv : out f32 [B,H,S,D] (fully overwritten; deterministic, no atomics).
  * layout     : token order of q, k, v, o, dout, lse, dq, dk and dv: NABLA_LAYOUT_REORDERED,

@@ -399,3 +399,34 @@ def test_bwd_natural_layout(data, name, thr, window):
         ref_nat = oracle.inverse_reorder(ref, T, Hg, W, P)
         mx, mean = check_close(to64(got), ref_nat, f"natural {what} {name}")
         print(f"natural {name} {what}: max|ref| {np.abs(ref).max():.2f} max err {mx:.2e} mean err {mean:.2e}")
+
+
+def test_bwd_reports_fp16_range():
+    """The backward's fp16 copies: a bf16 input beyond the fp16 range, or an infinite value
+    in a natural-order fp16 V, is reported in the status word (0x201); in-range inputs are
+    not."""
+    m = nbl()
+    wl = _wl("tiny")
+    shape = shape_of(wl)
+    q0, k0, v0 = make_qkv(wl, device=DEV)
+    nat = m.NABLA_LAYOUT_NATURAL
+    bits, ridx, rcnt, cidx, ccnt = gpu_mask(q0, k0, shape, 0.8, layout=nat)
+    g = torch.Generator(device=DEV).manual_seed(5)
+    do = torch.randn(q0.shape, generator=g, device=DEV).to(torch.bfloat16)
+
+    def status_of(q, k, v):
+        lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
+        o, _ = m.nabla_attn_fwd(q, k, v, bits, shape, o_dtype=m.NABLA_F32, lse=lse, layout=nat)
+        bws = torch.zeros(m.nabla_bwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+        m.nabla_attn_bwd(q, k, v, o, do, lse, ridx, rcnt, cidx, ccnt, shape, workspace=bws, layout=nat)
+        torch.cuda.synchronize()
+        return m.nabla_read_device_status(bws)
+
+    v16 = v0.to(torch.float16)
+    assert status_of(q0, k0, v16) == 0
+    big = q0.clone()
+    big[0, 1, 7, 3] = 1.0e5                       # representable in bf16, not in fp16
+    assert status_of(big, k0, v16) == 0x201
+    vinf = v16.clone()
+    vinf[0, 0, 100, 5] = float("inf")
+    assert status_of(q0, k0, vinf) == 0x201
