@@ -654,6 +654,30 @@ def main():
                                  "algorithmic_per_launch": f"{tk} kept 64x64 tiles x {int(fl_b)} FLOP"}})
             del tpath
             torch.cuda.empty_cache()
+        if wl.name == "wan720p":
+            # the hybrid mask on the same shape (NABLA at thr 0.7 OR a 3x3x5 STA window):
+            # the same step, timed beside the headline
+            swl = WORKLOADS["wan720p_sta"]
+            spath = Path(swl, dev)
+            for _ in range(3):
+                spath.step()
+            torch.cuda.synchronize()
+            spath.check_status()
+            spath.ev = {}
+            for _ in range(10):
+                spath.step(timing=True)
+            torch.cuda.synchronize()
+            spath.check_status()
+            sk = spath.kept_pairs()
+            s_fwd = statistics.mean(spath.segment_ms("t_mask", "t_fwd"))
+            side["sta_hybrid"] = {
+                "workload": swl.name, "thr": spath.thr, "sta": list(swl.window), "kept_tiles": sk,
+                "sparsity": 1.0 - sk / (BH * nb * nb), "step_ms": statistics.mean(spath.segment_ms("t0", "t_fwd")),
+                "mask_ms": statistics.mean(spath.segment_ms("t_reorder", "t_mask")), "fwd_ms": s_fwd,
+                "fwd_tflops_kept": sk * fl_fwd / (s_fwd * 1e-3) / 1e12,
+                "fwd_frac": sk * fl_fwd / (s_fwd * 1e-3) / 1e12 / pk["bf16_tflops"]}
+            del spath
+            torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers --------------------------------
     # Every step copies its own inputs host -> device and its result back inside the timed
