@@ -678,6 +678,34 @@ def main():
                 "fwd_frac": sk * fl_fwd / (s_fwd * 1e-3) / 1e12 / pk["bf16_tflops"]}
             del spath
             torch.cuda.empty_cache()
+            # the small configuration's threshold sweep, each forward next to the dense one
+            # on the same tensors (natural layout)
+            mwl = WORKLOADS["small"]
+            msh = m.Shape(mwl.B, mwl.H, mwl.T, mwl.Hg, mwl.W, mwl.D, mwl.P)
+            mq, mk, mv = make_qkv(mwl, device=dev)
+            mws = torch.zeros(m.nabla_fwd_workspace_bytes(msh), dtype=torch.uint8, device=dev)
+            mo = torch.empty_like(mq)
+            mnb = msh.nb
+            mdense = torch.full((mwl.B, mwl.H, mnb, msh.nw), -1, dtype=torch.int32, device=dev)
+            dms = time_call(lambda: m.nabla_attn_fwd(mq, mk, mv, mdense, msh, o=mo, workspace=mws,
+                                                     layout=m.NABLA_LAYOUT_NATURAL), 20, warm=3)
+            rows = []
+            for thr_m in mwl.thrs:
+                mc = torch.empty(mwl.B, mwl.H, mnb, dtype=torch.int32, device=dev)
+                mb, *_ = m.nabla_build_mask(mq, mk, msh, thr_m, mwl.window, row_cnt=mc,
+                                            layout=m.NABLA_LAYOUT_NATURAL)
+                kept_m = int(mc.to(torch.int64).sum())
+                sms_ = time_call(lambda: m.nabla_attn_fwd(mq, mk, mv, mb, msh, o=mo, workspace=mws,
+                                                          layout=m.NABLA_LAYOUT_NATURAL), 20, warm=3)
+                rows.append({"thr": thr_m, "kept_tiles": kept_m,
+                             "sparsity": 1.0 - kept_m / (mwl.B * mwl.H * mnb * mnb),
+                             "ms": sms_, "dense_ms": dms, "speedup_vs_dense": dms / sms_})
+            code = m.nabla_read_device_status(mws)
+            if code:
+                raise RuntimeError(f"device status 0x{code:x}")
+            side["small_thr_sweep"] = {"workload": mwl.name, "l2": "inputs fit in L2 (25 MB)",
+                                       "rows": rows}
+            del mq, mk, mv, mo, mdense, mws
 
     # ---- end to end through the public API with host buffers --------------------------------
     # Every step copies its own inputs host -> device and its result back inside the timed
