@@ -20,7 +20,8 @@
 // of the probabilities (non-negative doubles order like their bit patterns) where the
 // "mass at or above" crosses thr until it holds at most a few blocks; those are ranked
 // (probability descending, index ascending) and walked in order.  The logits are
-// computed with fp64 tensor-core MMA (m8n8k4), two key tiles per warp at a time.
+// computed with fp64 tensor-core MMA (m8n8k4), two key tiles per warp at a time, the
+// dims permuted so that each key's mean is read in whole 128-byte lines.
 #include <math.h>
 
 #include "common.cuh"
@@ -105,33 +106,56 @@ __global__ void __launch_bounds__(kThreads, 2) mask_rows_kernel(
   // ---- pooled logits A = Qp Kp^T * scale (fp64 tensor-core MMA, m8n8k4) ---------------
   // The (up to 8) rows of the group are the M = 8 side; each warp takes 8 key blocks at a
   // time (N = 8) and walks D in steps of 4.  Fragments: A[row = lane/4][k = lane%4],
-  // B[k = lane%4][key = lane/4], C[row = lane/4][key = 2*(lane%4) + {0,1}].
+  // B[k = lane%4][key = lane/4], C[row = lane/4][key = 2*(lane%4) + {0,1}].  The dot
+  // product runs over the D dims in a permuted order: step kk, lane k takes dim
+  // 16 (kk / 4) + 4 k + kk % 4, so that over four steps the four lanes of a key read one
+  // 128-byte line of the key's mean, each lane 32 contiguous bytes (two 16-byte loads when
+  // the means are 16-byte aligned), instead of 32 bytes of the line per step.
   __syncthreads();
   {
     const int gid = lane >> 2, tig = lane & 3;
     double afrag[D / 4];
 #pragma unroll
-    for (int kk = 0; kk < D / 4; ++kk) afrag[kk] = qs[gid * D + kk * 4 + tig];
+    for (int kk = 0; kk < D / 4; ++kk) afrag[kk] = qs[gid * D + 16 * (kk >> 2) + 4 * tig + (kk & 3)];
+    const bool vec = (reinterpret_cast<uintptr_t>(kpool) & 15) == 0;   // uniform
     // Two 8-key tiles per iteration: two independent accumulation chains, their key
     // loads in flight together.
     for (int jt = warp; jt * 8 < nb; jt += 2 * kWarps) {
       const int jt2 = jt + kWarps;
       const bool two = jt2 * 8 < nb;               // warp-uniform
       const int key = jt * 8 + gid, key2 = jt2 * 8 + gid;
-      const double* kr = kpool + (bh * nb + (key < nb ? key : 0)) * D + tig;
-      const double* kr2 = kpool + (bh * nb + (key2 < nb ? key2 : 0)) * D + tig;
+      const bool v1 = key < nb, v2 = two && key2 < nb;
+      const double* kr = kpool + (bh * nb + (v1 ? key : 0)) * D + 4 * tig;
+      const double* kr2 = kpool + (bh * nb + (v2 ? key2 : 0)) * D + 4 * tig;
       double c0 = 0.0, c1 = 0.0, c2 = 0.0, c3 = 0.0;
 #pragma unroll
-      for (int kk = 0; kk < D / 4; ++kk) {
-        const double b = key < nb ? __ldg(kr + kk * 4) : 0.0;
-        const double b2 = (two && key2 < nb) ? __ldg(kr2 + kk * 4) : 0.0;
-        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                     : "+d"(c0), "+d"(c1)
-                     : "d"(afrag[kk]), "d"(b));
-        if (two)
+      for (int g4 = 0; g4 < D / 16; ++g4) {
+        double b[4], b2[4];
+        if (vec) {
+          const double2 z = make_double2(0.0, 0.0);
+          const double2 x0 = v1 ? __ldg(reinterpret_cast<const double2*>(kr + 16 * g4)) : z;
+          const double2 x1 = v1 ? __ldg(reinterpret_cast<const double2*>(kr + 16 * g4 + 2)) : z;
+          const double2 y0 = v2 ? __ldg(reinterpret_cast<const double2*>(kr2 + 16 * g4)) : z;
+          const double2 y1 = v2 ? __ldg(reinterpret_cast<const double2*>(kr2 + 16 * g4 + 2)) : z;
+          b[0] = x0.x; b[1] = x0.y; b[2] = x1.x; b[3] = x1.y;
+          b2[0] = y0.x; b2[1] = y0.y; b2[2] = y1.x; b2[3] = y1.y;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            b[e] = v1 ? __ldg(kr + 16 * g4 + e) : 0.0;
+            b2[e] = v2 ? __ldg(kr2 + 16 * g4 + e) : 0.0;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
           asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                       : "+d"(c2), "+d"(c3)
-                       : "d"(afrag[kk]), "d"(b2));
+                       : "+d"(c0), "+d"(c1)
+                       : "d"(afrag[4 * g4 + e]), "d"(b[e]));
+          if (two)
+            asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                         : "+d"(c2), "+d"(c3)
+                         : "d"(afrag[4 * g4 + e]), "d"(b2[e]));
+        }
       }
       if (gid < nrows) {
         const int key0 = jt * 8 + 2 * tig;

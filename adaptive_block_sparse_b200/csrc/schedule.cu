@@ -23,7 +23,7 @@ namespace {
 __global__ void __launch_bounds__(512) sched_head_sort_kernel(const int32_t* __restrict__ cnt,
                                                               const uint32_t* __restrict__ bits,
                                                               int nb, int nw, int npairs, int npow2,
-                                                              int T, int HW, int frame_pairs,
+                                                              int T, int HW, int frame_pairs, int vec4,
                                                               int32_t* __restrict__ sorted,
                                                               int32_t* __restrict__ head_len) {
   extern __shared__ unsigned long long keys[];
@@ -41,10 +41,32 @@ __global__ void __launch_bounds__(512) sched_head_sort_kernel(const int32_t* __r
       if (bits != nullptr) {
         const uint32_t* r0 = bits + (bh * nb + i0) * static_cast<long long>(nw);
         const uint32_t* r1 = i1 >= 0 ? bits + (bh * nb + i1) * static_cast<long long>(nw) : nullptr;
-        for (int w = 0; w < nw; ++w) {
-          uint32_t u = r0[w] | (r1 ? r1[w] : 0u);
-          if (w == nw - 1 && (nb & 31)) u &= (1u << (nb & 31)) - 1u;
-          c += __popc(u);
+        const uint32_t tail = (nb & 31) ? (1u << (nb & 31)) - 1u : ~0u;
+        if (vec4) {
+          // rows of whole 16-byte words: eight of them (both rows) in flight at a time
+          const uint4* a4 = reinterpret_cast<const uint4*>(r0);
+          const uint4* b4 = reinterpret_cast<const uint4*>(r1);
+          const int n4 = nw >> 2;
+          for (int w4 = 0; w4 < n4; w4 += 8) {
+            uint4 xa[8], xb[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              xa[i] = w4 + i < n4 ? __ldg(a4 + w4 + i) : make_uint4(0u, 0u, 0u, 0u);
+              xb[i] = (r1 != nullptr && w4 + i < n4) ? __ldg(b4 + w4 + i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t last = w4 + i == n4 - 1 ? tail : ~0u;   // word nw - 1 is the .w part
+              c += __popc(xa[i].x | xb[i].x) + __popc(xa[i].y | xb[i].y) + __popc(xa[i].z | xb[i].z) +
+                   __popc((xa[i].w | xb[i].w) & last);
+            }
+          }
+        } else {
+          for (int w = 0; w < nw; ++w) {
+            uint32_t u = r0[w] | (r1 ? r1[w] : 0u);
+            if (w == nw - 1) u &= tail;
+            c += __popc(u);
+          }
         }
       } else {
         c = min(max(cnt[bh * nb + i0], 0), nb);
@@ -130,8 +152,10 @@ cudaError_t build_schedule(const int32_t* cnt, const uint32_t* bits, const Dims&
   cudaError_t e = cudaFuncSetAttribute(sched_head_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  // 16-byte loads of the bitmask rows when every row starts on a 16-byte boundary
+  const int vec4 = bits != nullptr && (d.nw & 3) == 0 && (reinterpret_cast<uintptr_t>(bits) & 15) == 0;
   sched_head_sort_kernel<<<d.BH, 512, smem, st>>>(cnt, bits, d.nb, d.nw, npairs, npow2, d.T,
-                                                   d.Hb * d.Wb, frame_pairs ? 1 : 0, sorted, head_len);
+                                                   d.Hb * d.Wb, frame_pairs ? 1 : 0, vec4, sorted, head_len);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   sched_head_place_kernel<<<d.BH, 256, 0, st>>>(sorted, head_len, d.BH, npairs, order);
