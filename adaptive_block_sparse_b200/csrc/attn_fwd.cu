@@ -362,13 +362,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         ++nq;
-        // the next tile's descriptor, while this tile's copies run
-        if (!end && fetched == c + 1) {
-          const int f = fetch(fetched);
-          if (f < 0) { ok = false; break; }
-          ++fetched;
-          if (f == 0) end = true;
-        }
         WarpBitWalk wk;
         wk.init(prm.bits + (static_cast<long long>(t.bh) * nb + t.ia) * nw,
                 t.ib >= 0 ? prm.bits + (static_cast<long long>(t.bh) * nb + t.ib) * nw : nullptr, nw, nb);
@@ -404,8 +397,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!load_k(j_next)) { ok = false; break; }
           }
           if (!load_v(j)) { ok = false; break; }
+          // the next tile's descriptor, once this tile's first K, V (and second K) are on
+          // their way
+          if (k == 0 && !end && fetched == c + 1) {
+            const int fr = fetch(fetched);
+            if (fr < 0) { ok = false; break; }
+            ++fetched;
+            if (fr == 0) end = true;
+          }
         }
         if (!ok) break;
+        if (!end && fetched == c + 1) {     // a tile without steps
+          const int fr = fetch(fetched);
+          if (fr < 0) break;
+          ++fetched;
+          if (fr == 0) end = true;
+        }
       }
       // Drain: copies still in flight must land before the CTA exits.
       if (nq > 0) mbar_wait(&B.q_full, (nq - 1) & 1, status, kDevTimeoutDrain);
