@@ -47,8 +47,8 @@ constexpr int kMetaInts = 8;              // item, bh, block a, block b, steps
 // (0-3) give registers up to the softmax warps (a row's 64 scores of a step, the packed
 // weights, the epilogue's packed O row).
 constexpr int kLaunchRegs = 168;
-constexpr int kRegProducer = 56;
-constexpr int kRegSoftmax = 224;
+constexpr int kRegProducer = 64;
+constexpr int kRegSoftmax = 216;
 static_assert(128 * kRegProducer + 256 * kRegSoftmax <= kThreads * kLaunchRegs,
               "register split exceeds the block's launch budget");
 
@@ -101,14 +101,55 @@ struct WarpBitWalk {
   const uint32_t* rb;
   int nw, w;
   uint32_t tail, a, b, cur;
+  // rows of up to 64 words are held in registers for the whole tile: lane l keeps words
+  // l and l + 32 of both rows, so moving to the next non-empty word takes a ballot and a
+  // shuffle instead of a dependent global load
+  bool reg;
+  uint32_t a0, a1, b0, b1;
   __device__ void init(const uint32_t* row_a, const uint32_t* row_b, int n_words, int nb) {
     ra = row_a; rb = row_b; nw = n_words; w = -1; cur = 0u; a = b = 0u;
     tail = (nb & 31) ? (1u << (nb & 31)) - 1u : ~0u;
+    reg = n_words <= 64;
+    a0 = a1 = b0 = b1 = 0u;
+    if (reg) {
+      const int l = static_cast<int>(threadIdx.x & 31);
+      if (l < nw) {
+        const uint32_t m = (l == nw - 1) ? tail : ~0u;
+        a0 = __ldg(ra + l) & m;
+        b0 = rb ? (__ldg(rb + l) & m) : 0u;
+      }
+      if (l + 32 < nw) {
+        const uint32_t m = (l + 32 == nw - 1) ? tail : ~0u;
+        a1 = __ldg(ra + l + 32) & m;
+        b1 = rb ? (__ldg(rb + l + 32) & m) : 0u;
+      }
+    }
   }
   __device__ int next(uint32_t* f) {
     while (cur == 0u) {
       const int base = w + 1;
       if (base >= nw) return -1;
+      if (reg) {
+        const int l = static_cast<int>(threadIdx.x & 31);
+        const uint32_t nz0 = __ballot_sync(0xffffffffu, l >= base && (a0 | b0) != 0u);
+        const uint32_t nz1 = __ballot_sync(0xffffffffu, l + 32 >= base && (a1 | b1) != 0u);
+        if (nz0 != 0u) {
+          const int src = __ffs(nz0) - 1;
+          w = src;
+          a = __shfl_sync(0xffffffffu, a0, src);
+          b = __shfl_sync(0xffffffffu, b0, src);
+        } else if (nz1 != 0u) {
+          const int src = __ffs(nz1) - 1;
+          w = 32 + src;
+          a = __shfl_sync(0xffffffffu, a1, src);
+          b = __shfl_sync(0xffffffffu, b1, src);
+        } else {
+          w = nw;
+          return -1;
+        }
+        cur = a | b;
+        continue;
+      }
       const int ww = base + static_cast<int>(threadIdx.x & 31);
       uint32_t xa = 0u, xb = 0u;
       if (ww < nw) {
