@@ -326,6 +326,50 @@ def test_fwd_dense_and_empty_rows(data):
                 assert torch.all(torch.isneginf(lse[:, :, r * 64:(r + 1) * 64]))
 
 
+def test_fwd_rows_beyond_64_mask_words(data):
+    """nb = 2176 (68 bitmask words per row): the forward's walk over the union of a tile's
+    two rows then reads the words from memory as it goes instead of holding them; kept
+    blocks sit in the first, middle and last words (the last one partly past nb)."""
+    m = nbl()
+    wl = WIDE
+    shape = shape_of(wl)
+    nb = wl.nb
+    assert shape.nw == 68
+    q, k, v = data(wl)
+    rng = np.random.default_rng(12)
+    mask = rng.random((1, 1, nb, nb)) < 4.0 / nb
+    ar = np.arange(nb)
+    mask[0, 0, ar, ar] = True                                   # no empty row
+    mask[0, 0, ar[::7], nb - 1] = True                          # the last, partial word
+    mask[0, 0, ar[::5], 2047] = True                            # either side of word 64
+    mask[0, 0, ar[::5], 2048] = True
+    mask[0, 0, ar[::3], 31] = True
+    bits = torch.from_numpy(oracle.pack_mask_bits(mask).view(np.int32)).to(DEV)
+    blocks = np.array([0, 1, 31, 63, 64, 1000, 1500, 2047, 2048, 2100, nb - 2, nb - 1])
+    rows = (blocks[:, None] * wl.N + np.arange(wl.N)[None, :]).reshape(-1)
+    scale = 1 / math.sqrt(wl.D)
+    qf, _ = gpu_reorder(q, shape)
+    kf, _ = gpu_reorder(k, shape)
+    vf, _ = gpu_reorder(v, shape)
+    vk, _ = gpu_reorder(v, shape, dtype=torch.float16)
+    O, L = oracle.block_sparse_attention_rows(to64(qf)[0, 0], to64(kf)[0, 0], to64(vf)[0, 0],
+                                              mask[0, 0], wl.N, scale, rows)
+    # reordered layout, fp16 V, f32 O
+    lse = torch.empty(wl.B, wl.H, wl.S, dtype=torch.float32, device=DEV)
+    ws = torch.zeros(m.nabla_fwd_workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    o, _ = m.nabla_attn_fwd(qf, kf, vk, bits, shape, o_dtype=m.NABLA_F32, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    assert m.nabla_read_device_status(ws) == 0
+    check_close(to64(o)[0, 0, rows], O, "O wide (reordered)")
+    check_lse(lse.cpu().numpy().astype(np.float64)[0, 0, rows], L)
+    # natural layout, bf16 V and O (the inference path)
+    o2, _ = m.nabla_attn_fwd(q, k, v, bits, shape, workspace=ws, layout=m.NABLA_LAYOUT_NATURAL)
+    torch.cuda.synchronize()
+    assert m.nabla_read_device_status(ws) == 0
+    perm = oracle.fractal_permutation(wl.T, wl.Hg, wl.W, wl.P)
+    check_close(to64(o2)[0, 0, perm[rows]], O, "O wide (natural)", storage_bf16=True)
+
+
 @pytest.mark.parametrize("name,thr,window", [("tiny", 0.8, (0, 0, 0)), ("small", 0.8, (3, 3, 3)),
                                              ("small", 0.95, (0, 0, 0)), ("odd", 0.8, (1, 1, 1)),
                                              ("odd64", 0.6, (0, 0, 0))])
