@@ -73,7 +73,7 @@ def peaks():
         with open(PEAKS_FILE) as f:
             p = json.load(f)
         return {k: float(p[k]) for k in FALLBACK}, "measured"
-    except Exception:
+    except (OSError, ValueError, KeyError, TypeError):
         return dict(FALLBACK), "fallback"
 
 
@@ -97,7 +97,7 @@ class ClockSampler:
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             threading.Thread(target=self._read, daemon=True).start()
-        except Exception:
+        except OSError:
             self.proc = None
 
     def _read(self):
@@ -110,7 +110,7 @@ class ClockSampler:
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
-        except Exception:
+        except subprocess.TimeoutExpired:
             self.proc.kill()
         time.sleep(0.05)
         sm, smax, reasons = [], [], set()
